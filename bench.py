@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE layer's forward + backward on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = moe_layer_fwd + moe_layer_bwd over one batch of the workload (default: the GPT-2-style
+GShard top-2 layer, T=4096, d=768, E=16, F=3072, GELU, capacity factor 1.25, bf16), inputs
+resident in HBM.  K steps are timed with CUDA events on the launching stream, one pair per step,
+with a 256 MiB write between steps to flush L2 (outside the timed pairs); the run is bracketed by
+a barrier and a device synchronise, and the max over ranks is taken.  value = tokens processed
+by all ranks / that time.  Several GPUs run independent replicas (the layer has no exchange step
+on one device), so scaling is weak.
+
+Also reported: e2e (the same step through the C ABI with the step's inputs copied from pinned
+host memory and its outputs read back inside the timed region), per-phase device times from the
+library's profiling events, the roofline of the dominant kernel, SM clocks sampled during the
+timed region, the number of library kernel launches in the timed region, and the CPU oracle
+timed on a bounded sample (rank 0, one GPU).
+
+--impl reference times the CPU oracle itself on this host's cores as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s fwd+bwd on 1 B200; % bf16 TC peak (GEMM), % HBM BW (rest)"
+FLUSH_BYTES = 256 << 20
+GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gpt2_gshard")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return j["hbm_gbs"], j["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_step(shape, inp, n_tok):
+    """One oracle forward + backward on the first n_tok tokens of the workload (capacity
+    recomputed for n_tok tokens).  Returns seconds."""
+    from mixture_experts_layer_23_b200.synth import to_f64
+    from oracle import moe_oracle as mo
+    dt = shape.dtype
+    x = to_f64(inp["x"][:n_tok], dt)
+    dy = to_f64(inp["dy"][:n_tok], dt) if inp["dy"] is not None else None
+    Wg = to_f64(inp["Wg"], dt)
+    W1, W2 = inp["_W1_64"], inp["_W2_64"]
+    W3 = inp.get("_W3_64")
+    t0 = time.perf_counter()
+    f = mo.layer_forward(x, Wg, inp["bias"], W1, W3, W2, k=shape.k, act=shape.act,
+                         gate_norm=shape.gate_norm, capacity_factor=shape.capacity_factor,
+                         n_shared=shape.n_shared)
+    if dy is not None:
+        mo.layer_backward(f, x, Wg, W1, W3, W2, dy)
+    return time.perf_counter() - t0
+
+
+def prepare_oracle_weights(shape, inp):
+    from mixture_experts_layer_23_b200.synth import to_f64
+    inp["_W1_64"] = to_f64(inp["W1"], shape.dtype)
+    inp["_W2_64"] = to_f64(inp["W2"], shape.dtype)
+    if inp["W3"] is not None:
+        inp["_W3_64"] = to_f64(inp["W3"], shape.dtype)
+
+
+def calibrate_sample(shape, inp, target_s):
+    """Token count whose oracle step takes about target_s seconds (>= 64, <= T)."""
+    n = min(shape.T, 256)
+    t = oracle_step(shape, inp, n)
+    want = int(n * target_s / max(t, 1e-3))
+    return max(64, min(shape.T, want)), t
+
+
+def cpu_baseline(shape, inp, target_s):
+    prepare_oracle_weights(shape, inp)
+    n, _ = calibrate_sample(shape, inp, target_s)
+    t = oracle_step(shape, inp, n)
+    return {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {n} of {shape.T} tokens, one float64 forward+backward of the same "
+                      f"layer (capacity recomputed for {n} tokens), {t:.1f} s"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from mixture_experts_layer_23_b200.configs import BY_NAME, WORKLOAD_TEXT
+    from mixture_experts_layer_23_b200.synth import make_inputs
+    shape = BY_NAME[args.workload]
+    inp = make_inputs(shape, 0)
+    prepare_oracle_weights(shape, inp)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n, _ = calibrate_sample(shape, inp, min(2.0, budget))
+    for _ in range(args.warmup):
+        oracle_step(shape, inp, n)
+    times = [oracle_step(shape, inp, n) for _ in range(args.steps)]
+    total = sum(times)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[shape.name], "name": shape.name, "T": shape.T,
+                   "d": shape.d, "E": shape.E, "k": shape.k, "d_ff": shape.d_ff},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"first {n} of {shape.T} tokens per step, float64 oracle "
+                                   "forward+backward (capacity recomputed for the sample)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.p = None
+        try:
+            self.p = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        out, _ = self.p.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def phase_work(shape, n_kept):
+    """Algorithmic work per phase: FLOPs for the GEMMs (kept rows only), bytes for the rest."""
+    b = 2 if shape.dtype == 1 else 4
+    T, d, F, S, E, k = shape.T, shape.d, shape.d_ff, shape.n_shared, shape.E, shape.k
+    rows = n_kept + S * T
+    g = 2 if shape.act == 1 else 1
+    Td, Nd = T * d * b, n_kept * d * b
+    return {
+        "router": ("hbm", Td + E * d * b + T * E * 4 + T * k * 8),
+        "dispatch": ("hbm", Td + Nd + T * k * 8),
+        "expert_up": ("tensor", 2.0 * rows * d * F * g),
+        "expert_down": ("tensor", 2.0 * rows * F * d),
+        "combine": ("hbm", Nd + S * Td + Td),
+        "combine_bwd": ("hbm", Td + 2 * Nd),
+        "router_bwd": ("hbm", Td + 2 * T * E * 4),
+        "dgrad_h": ("tensor", 2.0 * rows * d * F),
+        "dgrad_x": ("tensor", 2.0 * rows * F * d * g),
+        "wgrad_w1": ("tensor", 2.0 * rows * F * d * g),
+        "wgrad_w2": ("tensor", 2.0 * rows * d * F),
+        "undispatch": ("hbm", Nd + S * Td + Td),
+    }
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from mixture_experts_layer_23_b200 import build as moe_build
+    moe_build.build()
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.configs import BY_NAME, WORKLOAD_TEXT
+    from mixture_experts_layer_23_b200.layer import MoELayer, to_device
+    from mixture_experts_layer_23_b200.synth import make_inputs
+
+    shape = BY_NAME[args.workload]
+    inp = make_inputs(shape, 0)
+    w = {n: to_device(inp[n], shape, dev) for n in ("Wg", "W1", "W3", "W2")}
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
+    x = to_device(inp["x"], shape, dev)
+    dy = None if shape.fwd_only else to_device(inp["dy"], shape, dev)
+    layer = MoELayer(shape, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(x, w["Wg"], bias, w["W1"], w["W3"], w["W2"])
+        if dy is not None:
+            layer.backward(dy, x, w["Wg"], w["W1"], w["W3"], w["W2"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    st = layer.status()
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.STATUS_NAMES.get(st, st)}")
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    starts, ends = [mk() for _ in range(K)], [mk() for _ in range(K)]
+    nf, nb = len(moe.FWD_PHASES), len(moe.BWD_PHASES)
+    fev = [[mk() for _ in range(nf + 1)] for _ in range(K)]
+    bev = [[mk() for _ in range(nb + 1)] for _ in range(K)]
+    uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(uuid)
+    n0 = moe.kernel_launches()
+    for i in range(K):
+        moe.set_profile_events(fev[i], None if dy is None else bev[i])
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+        moe.set_profile_events(None, None)
+        flush.zero_()
+    launches = moe.kernel_launches() - n0
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    barrier()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    total_ms = max_over_ranks(total_ms)
+    st = layer.status()
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after timing: {moe.STATUS_NAMES.get(st, st)}")
+
+    # per-phase device times (average per launch)
+    phase_ms = {}
+    for j, name in enumerate(moe.FWD_PHASES):
+        phase_ms[name] = sum(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K)) / K
+    if dy is not None:
+        for j, name in enumerate(moe.BWD_PHASES):
+            phase_ms[name] = sum(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(K)) / K
+    n_kept = int(layer.view("kept").sum().item())
+    work = phase_work(shape, n_kept)
+    hbm_gbs, bf16_tf, peak_src = peaks()
+    phases = {}
+    for name, ms in phase_ms.items():
+        bound, amount = work[name]
+        if bound == "tensor":
+            ach = amount / (ms * 1e-3) / 1e12
+            phases[name] = {"ms": ms, "bound": bound, "achieved_tflops": ach,
+                            "frac": ach / bf16_tf}
+        else:
+            ach = amount / (ms * 1e-3) / 1e9
+            phases[name] = {"ms": ms, "bound": bound, "achieved_gbs": ach, "frac": ach / hbm_gbs}
+    top = max(phase_ms, key=phase_ms.get)
+    tb, tw = work[top]
+    if tb == "tensor":
+        ach = tw / (phase_ms[top] * 1e-3) / 1e12
+        roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16_tf,
+                "unit": "TFLOP/s", "frac": ach / bf16_tf, "traffic": None,
+                "peak_source": f"{peak_src} bf16 dense (burst)"}
+    else:
+        ach = tw / (phase_ms[top] * 1e-3) / 1e9
+        roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": ach / hbm_gbs, "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+
+    # end to end through the C ABI with host buffers
+    x_pin = x.cpu().pin_memory()
+    dy_pin = None if dy is None else dy.cpu().pin_memory()
+    y_host = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    dx_host = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+    h2d = x_pin.numel() * x_pin.element_size() + (0 if dy_pin is None else
+                                                  dy_pin.numel() * dy_pin.element_size())
+    d2h = y_host.numel() * y_host.element_size() + (0 if dy is None else
+                                                    dx_host.numel() * dx_host.element_size())
+    es, ee = [mk() for _ in range(K)], [mk() for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        es[i].record(stream)
+        x.copy_(x_pin, non_blocking=True)
+        if dy is not None:
+            dy.copy_(dy_pin, non_blocking=True)
+        step()
+        y_host.copy_(layer.y, non_blocking=True)
+        if dy is not None:
+            dx_host.copy_(layer.dx, non_blocking=True)
+        ee[i].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)))
+
+    value = world * shape.T * K / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if shape.dtype == 1 else "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[shape.name], "name": shape.name, "T": shape.T,
+                   "d": shape.d, "E": shape.E, "k": shape.k, "d_ff": shape.d_ff,
+                   "n_shared": shape.n_shared, "kept_assignments": n_kept,
+                   "gemm_engine": ["cuda_core", "tcgen05"][moe.gemm_engine(layer.cfg)],
+                   "l2": "flushed between timed steps (256 MiB write outside the timed events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "phases": phases,
+        "e2e": {"value": world * shape.T * K / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / K},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, inp, args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,381 @@
+// The C ABI of the MoE layer: argument checks, workspace layout and the call sequences of the
+// forward and backward passes.  Declarations and the contract are in include/moe.h.
+#include <math.h>
+#include <string.h>
+
+#include "launch.h"
+
+namespace moe {
+
+unsigned long long g_kernel_launches = 0;
+
+// Profiling hook (moe_set_profile_events): events recorded between the phases of a pass.
+static cudaEvent_t g_fwd_events[MOE_FWD_PHASES + 1];
+static cudaEvent_t g_bwd_events[MOE_BWD_PHASES + 1];
+static bool g_fwd_prof = false, g_bwd_prof = false;
+
+static inline moe_status mark_fwd(int i, cudaStream_t st) {
+  if (g_fwd_prof && cudaEventRecord(g_fwd_events[i], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+static inline moe_status mark_bwd(int i, cudaStream_t st) {
+  if (g_bwd_prof && cudaEventRecord(g_bwd_events[i], st) != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+static inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
+  if (!cfg || !out) return MOE_ERR_INVALID_ARG;
+  const moe_config_t& c = *cfg;
+  if (c.T < 1 || c.d < 1 || c.E < 1 || c.k < 1 || c.d_ff < 1 || c.n_shared < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c.k > c.E) return MOE_ERR_INVALID_ARG;
+  if (c.act != MOE_ACT_GELU && c.act != MOE_ACT_SWIGLU) return MOE_ERR_INVALID_ARG;
+  if (c.gate_norm != 0 && c.gate_norm != 1) return MOE_ERR_INVALID_ARG;
+  if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c.has_bias != 0 && c.has_bias != 1) return MOE_ERR_INVALID_ARG;
+  if (c.k > 8 || c.E > 256 || c.n_shared > 8 || c.T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
+  const int vec = (c.dtype == MOE_DTYPE_BF16) ? 8 : 4;
+  if (c.d % vec != 0 || c.d_ff % vec != 0) return MOE_ERR_UNSUPPORTED;
+
+  Dims D;
+  D.T = c.T; D.d = c.d; D.E = c.E; D.k = c.k; D.F = c.d_ff; D.S = c.n_shared;
+  D.E_tot = c.E + c.n_shared;
+  D.act = c.act; D.gate_norm = c.gate_norm; D.dtype = c.dtype; D.has_bias = c.has_bias;
+  D.elem = (c.dtype == MOE_DTYPE_BF16) ? 2 : 4;
+  if (c.capacity == MOE_DROPLESS) {
+    D.C = MOE_DROPLESS;
+  } else if (c.capacity >= 0) {
+    D.C = c.capacity;
+  } else {
+    if (!(c.capacity_factor > 0.f) || !isfinite(c.capacity_factor)) return MOE_ERR_INVALID_ARG;
+    const double cap = ceil((double)c.capacity_factor * c.k * c.T / c.E);
+    D.C = cap >= (double)MOE_DROPLESS ? (int64_t)MOE_DROPLESS : (int64_t)cap;
+  }
+  const int64_t kmax = D.C < D.T ? D.C : D.T;            // rows one expert can keep
+  D.T_pad = round_up(D.T, MOE_ROW_ALIGN);
+  D.routed_row0 = (int64_t)D.S * D.T_pad;
+  int64_t n_assign = (int64_t)D.T * D.k;
+  if ((int64_t)D.E * kmax < n_assign) n_assign = (int64_t)D.E * kmax;
+  const int64_t routed = (n_assign + (int64_t)(MOE_ROW_ALIGN - 1) * D.E) / MOE_ROW_ALIGN * MOE_ROW_ALIGN;
+  D.R = D.routed_row0 + routed;
+  if (D.R < MOE_ROW_ALIGN) D.R = MOE_ROW_ALIGN;
+  if (D.R >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  int64_t mg = round_up(kmax, MOE_ROW_ALIGN);
+  if (D.S > 0 && D.T_pad > mg) mg = D.T_pad;
+  D.max_group_rows = mg < MOE_ROW_ALIGN ? MOE_ROW_ALIGN : mg;
+  D.n_blk = (D.T + kDispatchTokensPerBlock - 1) / kDispatchTokensPerBlock;
+  D.n_tchunk = (D.T + kRouterBwdTokensPerChunk - 1) / kRouterBwdTokensPerChunk;
+  *out = D;
+  return MOE_OK;
+}
+
+ScratchLayout scratch_layout(const Dims& D) {
+  ScratchLayout S;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
+  const size_t R = (size_t)D.R, T = (size_t)D.T;
+  S.status = take(256);
+  S.blk_counts = take((size_t)D.n_blk * D.E * 4);
+  S.local_rank = 0;  // the dispatch keeps local ranks in the slot array
+  S.groups = take((size_t)D.E_tot * 16);
+  S.dO = take(R * D.d * D.elem);
+  S.dU = take(R * D.F * D.elem);
+  S.dV = (D.act == MOE_ACT_SWIGLU) ? take(R * D.F * D.elem) : 0;
+  S.dXd = take(R * D.d * D.elem);
+  S.dg = take(T * D.k * 4);
+  S.dlogits = take(T * D.E * 4);
+  S.dWg_part = take((size_t)D.n_tchunk * D.E * D.d * 4);
+  S.total = off;
+  return S;
+}
+
+moe_status ctx_layout(const Dims& D, moe_layout_t* L) {
+  memset(L, 0, sizeof(*L));
+  size_t off = 0;
+  auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
+  const size_t R = (size_t)D.R, T = (size_t)D.T;
+  L->capacity = D.C;
+  L->T_pad = D.T_pad;
+  L->rows = D.R;
+  L->routed_row0 = D.routed_row0;
+  L->max_group_rows = D.max_group_rows;
+  L->ctx_logits = take(T * D.E * 4);
+  L->ctx_topk_idx = take(T * D.k * 4);
+  L->ctx_topk_w = take(T * D.k * 4);
+  L->ctx_counts = take((size_t)D.E * 4);
+  L->ctx_kept = take((size_t)D.E * 4);
+  L->ctx_offsets = take((size_t)(D.E + 1) * 4);
+  L->ctx_slot = take(T * D.k * 4);
+  L->ctx_row_token = take(R * 4);
+  L->ctx_Xd = take(R * D.d * D.elem);
+  L->ctx_U = take(R * D.F * D.elem);
+  L->ctx_V = (D.act == MOE_ACT_SWIGLU) ? take(R * D.F * D.elem) : 0;
+  L->ctx_H = take(R * D.F * D.elem);
+  L->ctx_O = take(R * D.d * D.elem);
+  L->ctx_bytes = off;
+  L->scratch_bytes = scratch_layout(D).total;
+  return MOE_OK;
+}
+
+static inline bool misaligned(const void* p) { return ((uintptr_t)p & 15u) != 0; }
+
+// All listed pointers non-null and 16-byte aligned.
+static moe_status check_ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (misaligned(p)) return MOE_ERR_MISALIGNED;
+  }
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)                    \
+  do {                                   \
+    const moe_status s_ = (expr);        \
+    if (s_ != MOE_OK) return s_;         \
+  } while (0)
+
+// Expert FFN forward: the up-projection GEMM, then the down-projection GEMM.  With
+// phase_marks, the profiling event of phase 3 (expert_up) is recorded between the two.
+static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
+                             const void* W1, const void* W3, const void* W2, void* U, void* V,
+                             void* H, void* O, cudaStream_t st, bool phase_marks = false) {
+  MOE_TRY(launch_expert_up_simt(D, Xd, x, offsets, W1, W3, U, V, H, st));
+  if (phase_marks) MOE_TRY(mark_fwd(3, st));
+  return launch_expert_down_simt(D, H, offsets, W2, O, st);
+}
+
+// Expert FFN backward: dgrad through W2 and the activation, dgrad through W1 (and W3), then the
+// weight gradients; profiling phases 3..6 of the backward pass.
+static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, const void* Xd,
+                             const void* x, const int32_t* offsets, const void* W1,
+                             const void* W3, const void* W2, const void* U, const void* V,
+                             const void* H, void* dU, void* dV, void* dXd, float* dW1, float* dW3,
+                             float* dW2, cudaStream_t st) {
+  MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, U, V, dU, dV, st));
+  MOE_TRY(mark_bwd(3, st));
+  MOE_TRY(launch_dgrad_x_simt(D, dU, dV, offsets, W1, W3, dXd, st));
+  MOE_TRY(mark_bwd(4, st));
+  MOE_TRY(launch_wgrad_w13_simt(D, dU, dV, Xd, x, offsets, dW1, dW3, st));
+  MOE_TRY(mark_bwd(5, st));
+  MOE_TRY(launch_wgrad_w2_simt(D, H, dO, dy, offsets, dW2, st));
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_get_layout(const moe_config_t* cfg, moe_layout_t* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  return ctx_layout(D, out);
+}
+
+moe_status moe_workspace_size(const moe_config_t* cfg, size_t* ctx_bytes, size_t* scratch_bytes) {
+  if (!ctx_bytes || !scratch_bytes) return MOE_ERR_INVALID_ARG;
+  moe_layout_t L;
+  MOE_TRY(moe_get_layout(cfg, &L));
+  *ctx_bytes = L.ctx_bytes;
+  *scratch_bytes = L.scratch_bytes;
+  return MOE_OK;
+}
+
+moe_status moe_scratch_grad_offsets(const moe_config_t* cfg, size_t* dg_offset,
+                                    size_t* dlogits_offset) {
+  if (!dg_offset || !dlogits_offset) return MOE_ERR_INVALID_ARG;
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  const ScratchLayout S = scratch_layout(D);
+  *dg_offset = S.dg;
+  *dlogits_offset = S.dlogits;
+  return MOE_OK;
+}
+
+int32_t moe_gemm_engine(const moe_config_t* cfg) {
+  Dims D;
+  if (resolve_dims(cfg, &D) != MOE_OK) return -1;
+  return 0;
+}
+
+moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, const float* bias,
+                     float* logits, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({x, Wg, logits, topk_idx, topk_w}));
+  if (D.has_bias) MOE_TRY(check_ptrs({bias}));
+  return launch_router(D, x, Wg, bias, logits, topk_idx, topk_w, (cudaStream_t)stream);
+}
+
+moe_status moe_route_from_logits(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
+                                 float* topk_w, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({logits, topk_idx, topk_w}));
+  return launch_topk_from_logits(D, logits, topk_idx, topk_w, (cudaStream_t)stream);
+}
+
+moe_status moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                        int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
+                        int32_t* row_token, void* Xd, void* scratch, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({x, topk_idx, counts, kept, offsets, slot, row_token, Xd, scratch}));
+  const ScratchLayout S = scratch_layout(D);
+  return launch_dispatch(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
+                         (int32_t*)((char*)scratch + S.blk_counts), (cudaStream_t)stream);
+}
+
+moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x,
+                          const int32_t* offsets, const void* W1, const void* W3, const void* W2,
+                          void* U, void* V, void* H, void* O, void* scratch,
+                          moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({Xd, x, offsets, W1, W2, U, H, O, scratch}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, V}));
+  return expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, (cudaStream_t)stream);
+}
+
+moe_status moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot,
+                       const float* topk_w, void* y, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({O, slot, topk_w, y}));
+  return launch_combine(D, O, slot, topk_w, y, (cudaStream_t)stream);
+}
+
+moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
+                         const float* bias, const void* W1, const void* W3, const void* W2,
+                         void* y, void* ctx, void* scratch, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({x, Wg, W1, W2, y, ctx, scratch}));
+  if (D.has_bias) MOE_TRY(check_ptrs({bias}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3}));
+  moe_layout_t L;
+  ctx_layout(D, &L);
+  const ScratchLayout S = scratch_layout(D);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* c = (char*)ctx;
+  char* s = (char*)scratch;
+  if (cudaMemsetAsync(s + S.status, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  float* logits = (float*)(c + L.ctx_logits);
+  int32_t* idx = (int32_t*)(c + L.ctx_topk_idx);
+  float* w = (float*)(c + L.ctx_topk_w);
+  int32_t* counts = (int32_t*)(c + L.ctx_counts);
+  int32_t* kept = (int32_t*)(c + L.ctx_kept);
+  int32_t* offsets = (int32_t*)(c + L.ctx_offsets);
+  int32_t* slot = (int32_t*)(c + L.ctx_slot);
+  int32_t* row_token = (int32_t*)(c + L.ctx_row_token);
+  void* Xd = c + L.ctx_Xd;
+  void* U = c + L.ctx_U;
+  void* V = L.ctx_V ? c + L.ctx_V : nullptr;
+  void* H = c + L.ctx_H;
+  void* O = c + L.ctx_O;
+  MOE_TRY(mark_fwd(0, st));
+  MOE_TRY(launch_router(D, x, Wg, bias, logits, idx, w, st));
+  MOE_TRY(mark_fwd(1, st));
+  MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
+                          (int32_t*)(s + S.blk_counts), st));
+  MOE_TRY(mark_fwd(2, st));
+  MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, st, /*phase_marks=*/true));
+  MOE_TRY(mark_fwd(4, st));
+  MOE_TRY(launch_combine(D, O, slot, w, y, st));
+  MOE_TRY(mark_fwd(5, st));
+  return MOE_OK;
+}
+
+moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* dy, const void* x,
+                         const void* Wg, const void* W1, const void* W3, const void* W2,
+                         void* dx, float* dWg, float* dW1, float* dW3, float* dW2, void* scratch,
+                         moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({ctx, dy, x, Wg, W1, W2, dx, dWg, dW1, dW2, scratch}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, dW3}));
+  moe_layout_t L;
+  ctx_layout(D, &L);
+  const ScratchLayout S = scratch_layout(D);
+  cudaStream_t st = (cudaStream_t)stream;
+  const char* c = (const char*)ctx;
+  char* s = (char*)scratch;
+  const float* logits = (const float*)(c + L.ctx_logits);
+  const int32_t* idx = (const int32_t*)(c + L.ctx_topk_idx);
+  const float* w = (const float*)(c + L.ctx_topk_w);
+  const int32_t* kept = (const int32_t*)(c + L.ctx_kept);
+  const int32_t* offsets = (const int32_t*)(c + L.ctx_offsets);
+  const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
+  const void* Xd = c + L.ctx_Xd;
+  const void* U = c + L.ctx_U;
+  const void* V = L.ctx_V ? c + L.ctx_V : nullptr;
+  const void* H = c + L.ctx_H;
+  const void* O = c + L.ctx_O;
+  void* dO = s + S.dO;
+  void* dU = s + S.dU;
+  void* dV = S.dV ? s + S.dV : nullptr;
+  void* dXd = s + S.dXd;
+  float* dg = (float*)(s + S.dg);
+  float* dl = (float*)(s + S.dlogits);
+  float* part = (float*)(s + S.dWg_part);
+  MOE_TRY(mark_bwd(0, st));
+  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, kept, offsets, dg, dO, st));
+  MOE_TRY(mark_bwd(1, st));
+  MOE_TRY(launch_router_bwd(D, logits, idx, w, dg, x, dl, part, dWg, st));
+  MOE_TRY(mark_bwd(2, st));
+  MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, U, V, H, dU, dV, dXd, dW1, dW3, dW2,
+                     st));
+  MOE_TRY(mark_bwd(6, st));
+  MOE_TRY(launch_undispatch(D, dl, Wg, dXd, slot, dx, st));
+  MOE_TRY(mark_bwd(7, st));
+  return MOE_OK;
+}
+
+int64_t moe_kernel_launches(void) {
+  return (int64_t)__atomic_load_n(&g_kernel_launches, __ATOMIC_RELAXED);
+}
+
+moe_status moe_set_profile_events(void* const* fwd_events, void* const* bwd_events) {
+  g_fwd_prof = fwd_events != nullptr;
+  g_bwd_prof = bwd_events != nullptr;
+  for (int i = 0; g_fwd_prof && i <= MOE_FWD_PHASES; ++i) {
+    if (!fwd_events[i]) { g_fwd_prof = g_bwd_prof = false; return MOE_ERR_INVALID_ARG; }
+    g_fwd_events[i] = (cudaEvent_t)fwd_events[i];
+  }
+  for (int i = 0; g_bwd_prof && i <= MOE_BWD_PHASES; ++i) {
+    if (!bwd_events[i]) { g_fwd_prof = g_bwd_prof = false; return MOE_ERR_INVALID_ARG; }
+    g_bwd_events[i] = (cudaEvent_t)bwd_events[i];
+  }
+  return MOE_OK;
+}
+
+moe_status moe_read_status(moe_stream_t stream, void* scratch) {
+  if (!scratch) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, scratch, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemset(scratch, 0, 4) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_DEVICE_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

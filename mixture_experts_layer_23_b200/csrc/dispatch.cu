@@ -1,0 +1,169 @@
+// Capacity-limited dispatch of token rows into expert-contiguous buffers.
+//
+// Step 2 of the expert-parallel workflow (tutorial ch.4 "分布式训练", section "专家并行", part 二,
+// step 2) and the exchange of section "All-to-All 通信模式", part 二 (device i sends the subset
+// S_ik of its tokens to expert k's device).  On one GPU the exchange is a permutation in HBM;
+// the expert-contiguous buffer it fills is exactly what an all-to-all would send.
+//
+// Ranking rule: within one expert, assignments are ordered by token index; the first C are kept
+// ("drop by token order").  The rank must be bit-exact and deterministic, so it is computed as a
+// stable counting sort in three launches, none of which waits on another CTA:
+//   1. rank:    each CTA takes 256 tokens; per warp, a shared-memory bitmask per expert marks the
+//               lanes (tokens) that chose it, so a popcount of the lower lanes gives each
+//               assignment's rank inside the warp; warp bases make it a rank inside the CTA.
+//               The CTA's per-expert histogram goes to scratch.
+//   2. scan:    one CTA turns the histograms into per-CTA bases (exclusive scan over CTAs, token
+//               order), counts, kept = min(counts, C) and the 128-row aligned segment offsets.
+//   3. scatter: one warp per token finalises its slots and copies its x row (16-byte vectors,
+//               read once, written to each kept slot); extra CTAs zero the padding rows.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int DT = kDispatchTokensPerBlock;  // 256 tokens = 8 warps x 32 lanes
+static_assert(DT == 256, "rank kernel assumes 8 warps of 32 tokens");
+
+__global__ void __launch_bounds__(256)
+dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
+                     int32_t* __restrict__ blk_counts, int32_t* __restrict__ local_rank) {
+  __shared__ uint32_t mask[8][256];
+  __shared__ int32_t wbase[8][256];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int i = tid; i < 8 * 256; i += 256) (&mask[0][0])[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * DT + tid;
+  int e_of[8];
+  if (t < T_) {
+    for (int j = 0; j < k; ++j) {
+      e_of[j] = topk_idx[(int64_t)t * k + j];
+      if ((unsigned)e_of[j] < (unsigned)E) atomicOr(&mask[warp][e_of[j]], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += 256) {
+    int run = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w][e] = run;
+      run += __popc(mask[w][e]);
+    }
+    blk_counts[(int64_t)blockIdx.x * E + e] = run;
+  }
+  __syncthreads();
+  if (t < T_) {
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = e_of[j];
+      local_rank[(int64_t)t * k + j] =
+          ((unsigned)e < (unsigned)E) ? wbase[warp][e] + __popc(mask[warp][e] & below) : 0;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+dispatch_scan_kernel(int32_t* __restrict__ blk_counts, int n_blk, int E, int64_t C,
+                     int routed_row0, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+                     int32_t* __restrict__ offsets) {
+  __shared__ int32_t seg[257];
+  const int e = threadIdx.x;
+  if (e < E) {
+    int run = 0;
+    for (int b = 0; b < n_blk; ++b) {
+      const int c = blk_counts[(int64_t)b * E + e];
+      blk_counts[(int64_t)b * E + e] = run;  // becomes the CTA's base for this expert
+      run += c;
+    }
+    counts[e] = run;
+    const int kp = (int64_t)run < C ? run : (int)C;
+    kept[e] = kp;
+    seg[e] = (int)round_up(kp, MOE_ROW_ALIGN);
+  }
+  __syncthreads();
+  if (e == 0) {
+    int run = routed_row0;
+    for (int i = 0; i < E; ++i) {
+      offsets[i] = run;
+      run += seg[i];
+    }
+    offsets[E] = run;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
+                        const int32_t* __restrict__ blk_base, const int32_t* __restrict__ kept,
+                        const int32_t* __restrict__ offsets, int T_, int d, int E, int k,
+                        int64_t C, int n_tok_blocks, int shared_rows,
+                        int32_t* __restrict__ slot /* in: local rank, out: slot */,
+                        int32_t* __restrict__ row_token, T* __restrict__ Xd) {
+  constexpr int VN = Vec16<T>::N;
+  const int nv = d / VN;
+  const int lane = threadIdx.x & 31;
+  if ((int)blockIdx.x >= n_tok_blocks) {
+    // padding rows of routed expert e (or, for the last CTA, the shared rows' row_token)
+    const int e = blockIdx.x - n_tok_blocks;
+    if (e < E) {
+      const int r0 = offsets[e] + kept[e], r1 = offsets[e + 1];
+      for (int r = r0 + (threadIdx.x >> 5); r < r1; r += 8) {
+        if (lane == 0) row_token[r] = -1;
+        Vec16<T> z;
+        z.raw = make_uint4(0, 0, 0, 0);
+        for (int v = lane; v < nv; v += 32) st_vec(Xd + (int64_t)r * d + (int64_t)v * VN, z);
+      }
+    } else {
+      for (int r = threadIdx.x; r < shared_rows; r += blockDim.x) row_token[r] = -1;
+    }
+    return;
+  }
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T_) return;
+  int my_slot = -1;
+  if (lane < k) {
+    const int e = topk_idx[(int64_t)t * k + lane];
+    const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
+    const int pos = valid ? blk_base[(int64_t)(t / DT) * E + e] + slot[(int64_t)t * k + lane] : 0;
+    if (valid && (int64_t)pos < C) {
+      my_slot = offsets[e] + pos;
+      row_token[my_slot] = t;
+    }
+    slot[(int64_t)t * k + lane] = my_slot;
+  }
+  int s[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s[j] = __shfl_sync(0xffffffffu, my_slot, j);
+  const T* src = x + (int64_t)t * d;
+  for (int v = lane; v < nv; v += 32) {
+    const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < k && s[j] >= 0) st_vec(Xd + (int64_t)s[j] * d + (int64_t)v * VN, val);
+  }
+}
+
+}  // namespace
+
+moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
+                           int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                           void* Xd, int32_t* blk_counts, cudaStream_t st) {
+  dispatch_rank_kernel<<<D.n_blk, 256, 0, st>>>(topk_idx, D.T, D.E, D.k, blk_counts, slot);
+  MOE_LAUNCH_CHECK();
+  dispatch_scan_kernel<<<1, 256, 0, st>>>(blk_counts, D.n_blk, D.E, D.C, (int)D.routed_row0,
+                                          counts, kept, offsets);
+  MOE_LAUNCH_CHECK();
+  const int n_tok_blocks = (D.T + 7) / 8;
+  const int grid = n_tok_blocks + D.E + 1;
+  if (D.dtype == MOE_DTYPE_BF16)
+    dispatch_scatter_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        (const __nv_bfloat16*)x, topk_idx, blk_counts, kept, offsets, D.T, D.d, D.E, D.k, D.C,
+        n_tok_blocks, (int)D.routed_row0, slot, row_token, (__nv_bfloat16*)Xd);
+  else
+    dispatch_scatter_kernel<float><<<grid, 256, 0, st>>>(
+        (const float*)x, topk_idx, blk_counts, kept, offsets, D.T, D.d, D.E, D.k, D.C,
+        n_tok_blocks, (int)D.routed_row0, slot, row_token, (float*)Xd);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,43 @@
+// Internal launch functions of the MoE kernels (host side).  Each enqueues work on `st` and
+// returns MOE_ERR_CUDA if a launch fails.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+size_t router_smem_bytes(int E);
+moe_status launch_router(const Dims& D, const void* x, const void* Wg, const float* bias,
+                         float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
+moe_status launch_topk_from_logits(const Dims& D, const float* logits, int32_t* topk_idx,
+                                   float* topk_w, cudaStream_t st);
+moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
+                           int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                           void* Xd, int32_t* blk_counts, cudaStream_t st);
+moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
+                          void* y, cudaStream_t st);
+moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
+                              const float* topk_w, const int32_t* kept, const int32_t* offsets,
+                              float* dg, void* dO, cudaStream_t st);
+moe_status launch_router_bwd(const Dims& D, const float* logits, const int32_t* topk_idx,
+                             const float* topk_w, const float* dg, const void* x, float* dlogits,
+                             float* part, float* dWg, cudaStream_t st);
+moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
+                             const int32_t* slot, void* dx, cudaStream_t st);
+moe_status launch_expert_up_simt(const Dims& D, const void* Xd, const void* x,
+                                 const int32_t* offsets, const void* W1, const void* W3, void* U,
+                                 void* V, void* H, cudaStream_t st);
+moe_status launch_expert_down_simt(const Dims& D, const void* H, const int32_t* offsets,
+                                   const void* W2, void* O, cudaStream_t st);
+moe_status launch_dgrad_h_simt(const Dims& D, const void* dO, const void* dy,
+                               const int32_t* offsets, const void* W2, const void* U,
+                               const void* V, void* dU, void* dV, cudaStream_t st);
+moe_status launch_dgrad_x_simt(const Dims& D, const void* dU, const void* dV,
+                               const int32_t* offsets, const void* W1, const void* W3, void* dXd,
+                               cudaStream_t st);
+moe_status launch_wgrad_w13_simt(const Dims& D, const void* dU, const void* dV, const void* Xd,
+                                 const void* x, const int32_t* offsets, float* dW1, float* dW3,
+                                 cudaStream_t st);
+moe_status launch_wgrad_w2_simt(const Dims& D, const void* H, const void* dO, const void* dy,
+                                const int32_t* offsets, float* dW2, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,98 @@
+"""Device-side convenience around the C ABI: workspace allocation (torch), uploads of host
+inputs and typed views of the saved forward state.  Marshalling only; the layer's arithmetic
+is all in libmoe.so."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import moe
+from .configs import BF16, SWIGLU, LayerShape
+
+INT32 = torch.int32
+
+
+def act_dtype(shape: LayerShape):
+    return torch.bfloat16 if shape.dtype == BF16 else torch.float32
+
+
+def to_device(a, shape: LayerShape, device="cuda", pin=False):
+    """Storage-form numpy array (float32 or bf16 bits) -> torch tensor on `device`."""
+    if a is None:
+        return None
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(a))
+    if pin:
+        return t.pin_memory()
+    return t.to(device)
+
+
+class MoELayer:
+    """One layer's workspaces on one device."""
+
+    def __init__(self, shape: LayerShape, device="cuda", capacity=None):
+        self.shape = shape
+        self.cfg = moe.make_config(shape, capacity)
+        self.L = moe.get_layout(self.cfg)
+        self.device = torch.device(device)
+        self.dt = act_dtype(shape)
+        self.ctx = torch.empty(self.L.ctx_bytes, dtype=torch.uint8, device=self.device)
+        self.scratch = torch.zeros(self.L.scratch_bytes, dtype=torch.uint8, device=self.device)
+        T, d, E, F, Et = shape.T, shape.d, shape.E, shape.d_ff, shape.E_tot
+        self.y = torch.empty(T, d, dtype=self.dt, device=self.device)
+        self.dx = torch.empty(T, d, dtype=self.dt, device=self.device)
+        self.dWg = torch.empty(E, d, dtype=torch.float32, device=self.device)
+        self.dW1 = torch.empty(Et, F, d, dtype=torch.float32, device=self.device)
+        self.dW3 = (torch.empty(Et, F, d, dtype=torch.float32, device=self.device)
+                    if shape.act == SWIGLU else None)
+        self.dW2 = torch.empty(Et, d, F, dtype=torch.float32, device=self.device)
+
+    # typed views into ctx
+    def _view(self, off, dtype, shape):
+        n = int(np.prod(shape))
+        esz = torch.tensor([], dtype=dtype).element_size()
+        return self.ctx[off: off + n * esz].view(dtype).view(*shape)
+
+    def view(self, name):
+        s, L = self.shape, self.L
+        R = L.rows
+        table = {
+            "logits": (L.ctx_logits, torch.float32, (s.T, s.E)),
+            "topk_idx": (L.ctx_topk_idx, INT32, (s.T, s.k)),
+            "topk_w": (L.ctx_topk_w, torch.float32, (s.T, s.k)),
+            "counts": (L.ctx_counts, INT32, (s.E,)),
+            "kept": (L.ctx_kept, INT32, (s.E,)),
+            "offsets": (L.ctx_offsets, INT32, (s.E + 1,)),
+            "slot": (L.ctx_slot, INT32, (s.T, s.k)),
+            "row_token": (L.ctx_row_token, INT32, (R,)),
+            "Xd": (L.ctx_Xd, self.dt, (R, s.d)),
+            "U": (L.ctx_U, self.dt, (R, s.d_ff)),
+            "V": (L.ctx_V, self.dt, (R, s.d_ff)),
+            "H": (L.ctx_H, self.dt, (R, s.d_ff)),
+            "O": (L.ctx_O, self.dt, (R, s.d)),
+        }
+        off, dt, shp = table[name]
+        return self._view(off, dt, shp)
+
+    def scratch_view(self, name):
+        dg_off, dl_off = moe.scratch_grad_offsets(self.cfg)
+        s = self.shape
+        if name == "dg":
+            return self.scratch[dg_off: dg_off + s.T * s.k * 4].view(torch.float32).view(s.T, s.k)
+        if name == "dlogits":
+            return self.scratch[dl_off: dl_off + s.T * s.E * 4].view(torch.float32).view(s.T, s.E)
+        raise KeyError(name)
+
+    def forward(self, x, Wg, bias, W1, W3, W2, stream=None):
+        moe.layer_fwd(self.cfg, x, Wg, bias, W1, W3, W2, self.y, self.ctx, self.scratch, stream)
+        return self.y
+
+    def backward(self, dy, x, Wg, W1, W3, W2, stream=None):
+        moe.layer_bwd(self.cfg, self.ctx, dy, x, Wg, W1, W3, W2, self.dx, self.dWg, self.dW1,
+                      self.dW3, self.dW2, self.scratch, stream)
+        return self.dx
+
+    def status(self, stream=None) -> int:
+        return moe.read_status(self.scratch, stream)

@@ -206,7 +206,7 @@ def expert_backward(X, U, V, H, dO, W1e, W3e, W2e, act: int):
 
 def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
                   capacity_factor, n_shared: int = 0, identity_experts: bool = False,
-                  idx_override: np.ndarray | None = None):
+                  idx_override: np.ndarray | None = None, capacity_override=None):
     """Forward of the layer: route, dispatch under capacity, run experts, combine.
 
     Combine (Ch.4 "专家并行" 二 step 4: results return and sequence order is restored):
@@ -217,13 +217,14 @@ def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
     identity_experts: every expert returns its input (o = x), a pin of dispatch + combine.
     idx_override: route with these expert ids instead of re-selecting (used to compare against a
     device whose logits differ from the oracle's inside a near-tie).
+    capacity_override: an explicit capacity C instead of the one the capacity factor gives.
     """
     T, d = x.shape
     E = Wg.shape[0]
     logits = gate_logits(x, Wg, bias)
     idx = select_topk(logits, k) if idx_override is None else np.asarray(idx_override, np.int64)
     g = gate_weights(logits, idx, gate_norm)
-    C = capacity(capacity_factor, k, T, E)
+    C = capacity(capacity_factor, k, T, E) if capacity_override is None else capacity_override
     counts, kept, pos = dispatch(idx, E, C)
     y = np.zeros((T, d))
     cache = {}

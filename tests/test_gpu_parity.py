@@ -1,0 +1,174 @@
+"""CUDA path vs the CPU oracle, through the C ABI, on a B200.
+
+Routing ids, per-expert counts, kept counts, the slot map / drop mask and the dispatched rows
+must match bit-exactly; every float output and gradient must sit within max-abs error
+<= 1e-4 * max|ref| (fp32 layers) or 2e-2 * max|ref| (bf16 layers), per tensor.
+"""
+import numpy as np
+import pytest
+
+from mixture_experts_layer_23_b200.configs import (BF16, DROPLESS, FP32, GELU, LAYERS,
+                                                   PARITY_FP32, PARITY_SMALL, SWIGLU, LayerShape)
+from mixture_experts_layer_23_b200.synth import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("the gpu tests need a CUDA device")
+    from mixture_experts_layer_23_b200 import build
+    build.build()
+    yield
+
+
+def _parity():
+    import parity
+    return parity
+
+
+@pytest.mark.parametrize("shape", PARITY_SMALL + PARITY_FP32, ids=lambda s: s.name)
+def test_small_layers_match_oracle(shape):
+    _parity().full_compare(shape, seed=0)
+
+
+@pytest.mark.parametrize("shape", [s for s in LAYERS if s.name in
+                                   ("switch_tiny", "gpt2_gshard", "bert_large_skew")],
+                         ids=lambda s: s.name)
+def test_full_size_layers_match_oracle(shape):
+    """The three smaller named layers at full size, every element compared."""
+    _parity().full_compare(shape, seed=0)
+
+
+@pytest.mark.parametrize("shape", [s for s in LAYERS if s.name in
+                                   ("mixtral_dropless", "deepseek_v2")], ids=lambda s: s.name)
+def test_full_size_layers_sampled(shape):
+    """The two large named layers at full size: routing and dispatch in full, values sampled."""
+    _parity().sampled_compare(shape, seed=0)
+
+
+EDGE = [
+    LayerShape("one_token", T=1, d=64, E=4, k=2, d_ff=64, dtype=BF16),
+    LayerShape("single_expert_dense", T=130, d=64, E=1, k=1, d_ff=128, capacity_factor=1.0,
+               dtype=BF16),
+    LayerShape("k_equals_E", T=200, d=32, E=4, k=4, d_ff=48, gate_norm=1, capacity_factor=None,
+               act=SWIGLU, dtype=BF16),
+    LayerShape("ragged_bf16", T=333, d=40, E=5, k=2, d_ff=24, capacity_factor=0.9, dtype=BF16,
+               bias="zipf"),
+    LayerShape("ragged_fp32", T=129, d=12, E=3, k=2, d_ff=20, capacity_factor=1.1, dtype=FP32),
+    LayerShape("max_k_many_experts", T=300, d=32, E=256, k=8, d_ff=32, capacity_factor=2.0,
+               dtype=BF16, n_shared=1, act=SWIGLU, bias="normal"),
+    LayerShape("fp32_shared_only_top1", T=77, d=16, E=2, k=1, d_ff=8, n_shared=2,
+               capacity_factor=0.5, dtype=FP32),
+]
+
+
+@pytest.mark.parametrize("shape", EDGE, ids=lambda s: s.name)
+def test_edge_shapes(shape):
+    _parity().full_compare(shape, seed=3)
+
+
+def test_zero_capacity_drops_everything():
+    s = LayerShape("cap0", T=100, d=32, E=4, k=2, d_ff=32, n_shared=1, dtype=FP32)
+    gpu, _ = _parity().full_compare(s, seed=1, capacity=0)
+    assert np.all(gpu["slot"] == -1)
+    assert np.all(gpu["dW1"][:4] == 0) and np.all(gpu["dW2"][:4] == 0)
+
+
+def test_explicit_dropless_capacity():
+    s = LayerShape("dropless_explicit", T=150, d=32, E=4, k=2, d_ff=32, dtype=BF16)
+    gpu, _ = _parity().full_compare(s, seed=2, capacity=DROPLESS)
+    assert np.all(gpu["slot"] >= 0)
+
+
+def test_one_expert_takes_every_token():
+    s = LayerShape("hot_expert", T=400, d=64, E=8, k=2, d_ff=64, capacity_factor=1.0, dtype=BF16,
+                   bias="normal")
+    inp = make_inputs(s, 0)
+    inp["bias"] = np.zeros(8, np.float32)
+    inp["bias"][5] = 1000.0           # expert 5 is every token's first choice
+    gpu, _ = _parity().full_compare(s, inp=inp)
+    assert gpu["counts"][5] == 400 and gpu["kept"][5] == 100
+
+
+def test_exact_logit_ties_go_to_lower_index():
+    """Identical gate rows make exact logit ties: the lower expert index must win."""
+    s = LayerShape("ties", T=256, d=32, E=6, k=2, d_ff=32, capacity_factor=2.0, dtype=BF16)
+    inp = make_inputs(s, 4)
+    inp["Wg"][3] = inp["Wg"][1]
+    inp["Wg"][4] = inp["Wg"][1]
+    gpu, _ = _parity().full_compare(s, inp=inp)
+    idx = gpu["topk_idx"]
+    assert np.array_equal(gpu["logits"][:, 1], gpu["logits"][:, 3])
+    assert not np.any(idx == 4)                              # a tied higher index never wins
+    has3 = np.any(idx == 3, axis=1)
+    assert np.all(np.any(idx == 1, axis=1)[has3])            # 3 only ever beside its tie 1
+
+
+@pytest.mark.parametrize("shape", [PARITY_SMALL[1], PARITY_SMALL[4], PARITY_FP32[1]],
+                         ids=lambda s: s.name)
+def test_bitwise_deterministic(shape):
+    p = _parity()
+    inp = make_inputs(shape, 5)
+    a = p.run_gpu(shape, inp)
+    b = p.run_gpu(shape, inp)
+    for k in ("logits", "topk_idx", "topk_w", "slot", "Xd_bits", "y", "dx", "dWg", "dW1", "dW2",
+              "dg"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_route_and_route_from_logits_agree():
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import to_device
+    s = PARITY_SMALL[2]
+    inp = make_inputs(s, 0)
+    cfg = moe.make_config(s)
+    x, Wg = to_device(inp["x"], s), to_device(inp["Wg"], s)
+    bias = torch.from_numpy(inp["bias"]).cuda()
+    logits = torch.empty(s.T, s.E, device="cuda")
+    i1 = torch.empty(s.T, s.k, dtype=torch.int32, device="cuda")
+    w1 = torch.empty(s.T, s.k, device="cuda")
+    i2, w2 = torch.empty_like(i1), torch.empty_like(w1)
+    moe.route(cfg, x, Wg, bias, logits, i1, w1)
+    moe.route_from_logits(cfg, logits, i2, w2)
+    torch.cuda.synchronize()
+    assert torch.equal(i1, i2) and torch.equal(w1, w2)
+
+
+def test_step_entry_points_compose_to_the_layer():
+    """route -> dispatch -> expert_ffn -> combine equals moe_layer_fwd bit for bit."""
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import MoELayer, to_device
+    s = PARITY_SMALL[4]
+    inp = make_inputs(s, 0)
+    dev = {k: to_device(v, s) for k, v in inp.items() if k != "bias"}
+    bias = torch.from_numpy(inp["bias"]).cuda()
+    layer = MoELayer(s)
+    y_ref = layer.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"]).clone()
+    cfg, L = layer.cfg, layer.L
+    R = L.rows
+    dt = layer.dt
+    T, E, k, d, F = s.T, s.E, s.k, s.d, s.d_ff
+    logits = torch.empty(T, E, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    kept, offsets = torch.empty_like(counts), torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    slot = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    row_token = torch.empty(R, dtype=torch.int32, device="cuda")
+    Xd = torch.empty(R, d, dtype=dt, device="cuda")
+    U, V, H = (torch.empty(R, F, dtype=dt, device="cuda") for _ in range(3))
+    O = torch.empty(R, d, dtype=dt, device="cuda")
+    y = torch.empty(T, d, dtype=dt, device="cuda")
+    scratch = torch.zeros(L.scratch_bytes, dtype=torch.uint8, device="cuda")
+    moe.route(cfg, dev["x"], dev["Wg"], bias, logits, idx, w)
+    moe.dispatch(cfg, dev["x"], idx, counts, kept, offsets, slot, row_token, Xd, scratch)
+    moe.expert_ffn(cfg, Xd, dev["x"], offsets, dev["W1"], dev["W3"], dev["W2"], U, V, H, O, scratch)
+    moe.combine(cfg, O, slot, w, y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    assert torch.equal(slot, layer.view("slot"))
