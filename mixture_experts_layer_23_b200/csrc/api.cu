@@ -140,7 +140,13 @@ static moe_status check_ptrs(std::initializer_list<const void*> ps) {
 // phase_marks, the profiling event of phase 3 (expert_up) is recorded between the two.
 static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
                              const void* W1, const void* W3, const void* W2, void* U, void* V,
-                             void* H, void* O, cudaStream_t st, bool phase_marks = false) {
+                             void* H, void* O, uint32_t* status, cudaStream_t st,
+                             bool phase_marks = false) {
+  if (tc_supported(D)) {
+    MOE_TRY(launch_expert_up_tc(D, Xd, x, offsets, W1, W3, U, V, H, status, st));
+    if (phase_marks) MOE_TRY(mark_fwd(3, st));
+    return launch_expert_down_tc(D, H, offsets, W2, O, status, st);
+  }
   MOE_TRY(launch_expert_up_simt(D, Xd, x, offsets, W1, W3, U, V, H, st));
   if (phase_marks) MOE_TRY(mark_fwd(3, st));
   return launch_expert_down_simt(D, H, offsets, W2, O, st);
@@ -152,7 +158,17 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
                              const void* x, const int32_t* offsets, const void* W1,
                              const void* W3, const void* W2, const void* U, const void* V,
                              const void* H, void* dU, void* dV, void* dXd, float* dW1, float* dW3,
-                             float* dW2, cudaStream_t st) {
+                             float* dW2, uint32_t* status, cudaStream_t st) {
+  if (tc_supported(D)) {
+    MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, U, V, dU, dV, status, st));
+    MOE_TRY(mark_bwd(3, st));
+    MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
+    MOE_TRY(mark_bwd(4, st));
+    MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, status, st));
+    MOE_TRY(mark_bwd(5, st));
+    MOE_TRY(launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st));
+    return MOE_OK;
+  }
   MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, U, V, dU, dV, st));
   MOE_TRY(mark_bwd(3, st));
   MOE_TRY(launch_dgrad_x_simt(D, dU, dV, offsets, W1, W3, dXd, st));
@@ -199,7 +215,7 @@ moe_status moe_scratch_grad_offsets(const moe_config_t* cfg, size_t* dg_offset,
 int32_t moe_gemm_engine(const moe_config_t* cfg) {
   Dims D;
   if (resolve_dims(cfg, &D) != MOE_OK) return -1;
-  return 0;
+  return tc_supported(D) ? 1 : 0;
 }
 
 moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, const float* bias,
@@ -238,7 +254,9 @@ moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x
   MOE_TRY(resolve_dims(cfg, &D));
   MOE_TRY(check_ptrs({Xd, x, offsets, W1, W2, U, H, O, scratch}));
   if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, V}));
-  return expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, (cudaStream_t)stream);
+  const ScratchLayout S = scratch_layout(D);
+  return expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O,
+                    (uint32_t*)((char*)scratch + S.status), (cudaStream_t)stream);
 }
 
 moe_status moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot,
@@ -283,7 +301,8 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
                           (int32_t*)(s + S.blk_counts), st));
   MOE_TRY(mark_fwd(2, st));
-  MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, st, /*phase_marks=*/true));
+  MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, (uint32_t*)(s + S.status), st,
+                     /*phase_marks=*/true));
   MOE_TRY(mark_fwd(4, st));
   MOE_TRY(launch_combine(D, O, slot, w, y, st));
   MOE_TRY(mark_fwd(5, st));
@@ -328,7 +347,7 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   MOE_TRY(launch_router_bwd(D, logits, idx, w, dg, x, dl, part, dWg, st));
   MOE_TRY(mark_bwd(2, st));
   MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, U, V, H, dU, dV, dXd, dW1, dW3, dW2,
-                     st));
+                     (uint32_t*)(s + S.status), st));
   MOE_TRY(mark_bwd(6, st));
   MOE_TRY(launch_undispatch(D, dl, Wg, dXd, slot, dx, st));
   MOE_TRY(mark_bwd(7, st));

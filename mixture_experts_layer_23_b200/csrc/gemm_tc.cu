@@ -1,0 +1,833 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
+//
+// Step 3 of the expert-parallel workflow (tutorial ch.4 "分布式训练", section "专家并行", part 二,
+// step 3: each device runs its local experts on the tokens it received; part 一: each expert is
+// an MLP) and its backward (section "专家并行与数据并行的结合", part 三.3: expert weight gradients
+// are computed locally).  The Piper digest ("关键贡献", "关键要点") singles out thin expert GEMMs as
+// a cause of low GPU utilisation; here every expert's GEMM is one slice of a single persistent
+// launch, so a thin expert only costs its own tiles.
+//
+// One kernel, five kinds of grouped GEMM over the dispatched row space (bf16 in, fp32 accumulate):
+//   UP      : [U|V] = A W1^T (W3^T), epilogue H = gelu(U) or silu(U) * V      A = Xd (or x)
+//   DOWN    : O = H W2^T
+//   DGRAD_H : dH = A W2, epilogue dU = dH * gelu'(U)  or  dU, dV for SwiGLU   A = dO (or dy)
+//   DGRAD_X : dXd = dU W1 (+ dV W3)
+//   WGRAD   : dW1 = dU^T Xd, dW3 = dV^T Xd (which 0)  or  dW2 = dO^T H (which 2), fp32 out
+// Tiles are 128 x 256 (M x N), K in blocks of 64 (one 128-byte swizzle atom of bf16).
+//
+// CTA organisation (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: loads A and B tiles into a 4-stage shared-memory ring
+//   warp 1      owns the 512 TMEM columns (two 128x256 fp32 accumulators); one lane issues
+//               tcgen05.mma and commits each stage back to the producer
+//   warps 2..5  epilogue: tcgen05.ld the finished accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31 = tile rows), apply the fused activation, store to HBM
+// The two accumulators let the epilogue of one tile overlap the main loop of the next.
+// Every mbarrier wait is bounded: on timeout the kernel records MOE_STATUS_TIMEOUT in the status
+// word, drains its own copies and MMAs (with a bound), frees TMEM and returns.
+#include <cuda.h>  // CUtensorMap and its enums (types only; the encoder is fetched at run time)
+#include <string.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace tc {
+
+enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t A_BYTES = BM * BK * 2;           // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
+constexpr int MAX_GROUPS = 264;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4096;
+
+struct alignas(64) Params {
+  CUtensorMap a_main, a_alt, b_main, b_alt;
+  const int32_t* offsets;
+  const void* aux0;      // U (DGRAD_H epilogue)
+  const void* aux1;      // V (DGRAD_H epilogue, SwiGLU)
+  void* out0;            // U | O | dU | dXd | dW
+  void* out1;            // V | dV
+  void* out2;            // H
+  uint32_t* status;
+  unsigned long long timeout_ns;
+  long long T_pad;
+  int E, S, T;
+  int N;                 // output columns (row GEMMs: F or d; WGRAD: columns of the weight grad)
+  int Mw;                // WGRAD: rows of the weight grad
+  int K;                 // row GEMMs: inner dimension (d or F)
+  int act;
+  int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
+};
+
+// ----------------------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the CTA's abort flag) once the
+// time budget is spent, or as soon as another role of the CTA has aborted.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             unsigned long long budget_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > budget_ns) {
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 format: version 1 at bit 46,
+// layout type 2 = SWIZZLE_128B at bits 61..63).  K-major tiles: rows of 128 B, 8-row groups
+// 1024 B apart (SBO); LBO unused.  MN-major tiles: 64-element MN chunks LBO apart, 8-row K
+// groups 1024 B apart (SBO).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, M = 128, N = BN.
+__host__ __device__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
+  return (1u << 4)                       // D format fp32
+         | (1u << 7)                     // A format bf16
+         | (1u << 10)                    // B format bf16
+         | ((a_mn ? 1u : 0u) << 15)      // A major: 0 K, 1 MN
+         | ((b_mn ? 1u : 0u) << 16)      // B major
+         | ((uint32_t)(BN >> 3) << 17)   // N
+         | ((uint32_t)(BM >> 4) << 24);  // M
+}
+
+// ----------------------------------------------------------------------------- scheduling
+
+struct Tile {
+  int g, m, n;           // group, m tile, n tile
+  int a_row, o_row;      // first row of the group in input- / output-indexed buffers
+  int rows;              // group rows (multiple of 128)
+  bool shared;
+};
+
+// N columns one tile covers: a SwiGLU up-projection tile holds 128 columns of U and the same
+// 128 columns of V side by side.
+template <int KIND>
+__device__ __forceinline__ int tile_n(const Params& P) {
+  return (KIND == UP && P.act == MOE_ACT_SWIGLU) ? BN / 2 : BN;
+}
+
+template <int KIND>
+__device__ __forceinline__ int group_tiles(const Params& P, int rows) {
+  const int nt = (P.N + tile_n<KIND>(P) - 1) / tile_n<KIND>(P);
+  if (KIND == WGRAD) return ((P.Mw + BM - 1) / BM) * nt;
+  return (rows / BM) * nt;
+}
+
+__device__ __forceinline__ void group_rows(const Params& P, int g, int& a_row, int& o_row,
+                                           int& rows, bool& shared) {
+  if (g < P.E) {
+    a_row = P.offsets[g];
+    o_row = a_row;
+    rows = P.offsets[g + 1] - a_row;
+    shared = false;
+  } else {
+    a_row = 0;
+    o_row = (int)((g - P.E) * P.T_pad);
+    rows = (int)P.T_pad;
+    shared = true;
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, int n_groups,
+                                       int t) {
+  int lo = 0, hi = n_groups - 1;  // last g with tile_start[g] <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  Tile T;
+  T.g = lo;
+  group_rows(P, lo, T.a_row, T.o_row, T.rows, T.shared);
+  const int local = t - tile_start[lo];
+  const int mt = (KIND == WGRAD) ? (P.Mw + BM - 1) / BM : T.rows / BM;
+  T.m = local % mt;
+  T.n = local / mt;
+  return T;
+}
+
+template <int KIND>
+__device__ __forceinline__ int k_blocks(const Params& P, const Tile& t) {
+  if (KIND == WGRAD) return t.rows / BK;
+  if (KIND == DGRAD_X && P.act == MOE_ACT_SWIGLU) return 2 * (P.K / BK);
+  return P.K / BK;
+}
+
+// ----------------------------------------------------------------------------- producer
+
+template <int KIND>
+__device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int kb, uint8_t* sA,
+                                            uint8_t* sB, uint64_t* bar) {
+  const bool swiglu = P.act == MOE_ACT_SWIGLU;
+  const int k0 = kb * BK;
+  if (KIND == UP) {
+    const int n0 = t.n * (swiglu ? BN / 2 : BN);
+    if (t.shared) tma_load_2d(sA, &P.a_alt, bar, k0, t.m * BM);
+    else tma_load_2d(sA, &P.a_main, bar, k0, t.a_row + t.m * BM);
+    if (swiglu) {
+      tma_load_3d(sB, &P.b_main, bar, k0, n0, t.g);
+      tma_load_3d(sB + B_BYTES / 2, &P.b_alt, bar, k0, n0, t.g);
+    } else {
+      tma_load_3d(sB, &P.b_main, bar, k0, n0, t.g);
+    }
+  } else if (KIND == DOWN) {
+    tma_load_2d(sA, &P.a_main, bar, k0, t.o_row + t.m * BM);
+    tma_load_3d(sB, &P.b_main, bar, k0, t.n * BN, t.g);
+  } else if (KIND == DGRAD_H) {
+    if (t.shared) tma_load_2d(sA, &P.a_alt, bar, k0, t.m * BM);
+    else tma_load_2d(sA, &P.a_main, bar, k0, t.a_row + t.m * BM);
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j)
+      tma_load_3d(sB + j * 8192, &P.b_main, bar, t.n * BN + 64 * j, k0, t.g);
+  } else if (KIND == DGRAD_X) {
+    const int nkF = P.K / BK;
+    const bool second = kb >= nkF;
+    const int kk = (second ? kb - nkF : kb) * BK;
+    tma_load_2d(sA, second ? &P.a_alt : &P.a_main, bar, kk, t.o_row + t.m * BM);
+#pragma unroll
+    for (int j = 0; j < BN / 64; ++j)
+      tma_load_3d(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, t.n * BN + 64 * j, kk, t.g);
+  } else {  // WGRAD
+    const int m0 = t.m * BM, n0 = t.n * BN;
+    if (P.which == 0) {
+      // A = dU|dV rows of the group (row space), B = Xd rows (routed) or x (shared)
+#pragma unroll
+      for (int j = 0; j < BM / 64; ++j)
+        tma_load_2d(sA + j * 8192, &P.a_main, bar, m0 + 64 * j, t.o_row + k0);
+#pragma unroll
+      for (int j = 0; j < BN / 64; ++j) {
+        if (t.shared) tma_load_2d(sB + j * 8192, &P.b_alt, bar, n0 + 64 * j, k0);
+        else tma_load_2d(sB + j * 8192, &P.b_main, bar, n0 + 64 * j, t.a_row + k0);
+      }
+    } else {
+      // A = dO rows (routed) or dy (shared), B = H rows of the group
+#pragma unroll
+      for (int j = 0; j < BM / 64; ++j) {
+        if (t.shared) tma_load_2d(sA + j * 8192, &P.a_alt, bar, m0 + 64 * j, k0);
+        else tma_load_2d(sA + j * 8192, &P.a_main, bar, m0 + 64 * j, t.a_row + k0);
+      }
+#pragma unroll
+      for (int j = 0; j < BN / 64; ++j)
+        tma_load_2d(sB + j * 8192, &P.b_main, bar, n0 + 64 * j, t.o_row + k0);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- epilogue
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                      pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+}
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint4 u = s[q];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
+      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+}
+
+template <int KIND>
+__device__ __forceinline__ void epilogue_tile(const Params& P, const Tile& t, uint32_t tacc,
+                                              int nk, int quarter, int lane) {
+  const int r = quarter * 32 + lane;                // row inside the tile (= TMEM lane)
+  const uint32_t tl = tacc + ((uint32_t)(quarter * 32) << 16);
+  const bool swiglu = P.act == MOE_ACT_SWIGLU;
+  float v[32];
+  if (KIND == WGRAD) {
+    const int m = t.m * BM + r;   // rows >= Mw still join the warp-collective TMEM loads
+    float* out = reinterpret_cast<float*>(P.out0) + (size_t)t.g * P.Mw * P.N;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = t.n * BN + c * 32;
+      if (nk > 0) tmem_ld32(tl + c * 32, v);
+      else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+      if (m < P.Mw && n < P.N) {
+        float4* d = reinterpret_cast<float4*>(out + (size_t)m * P.N + n);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      }
+    }
+    return;
+  }
+  const size_t row = (size_t)t.o_row + (size_t)t.m * BM + r;
+  if (KIND == UP) {
+    const int F = P.N;
+    __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(P.out0);
+    __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(P.out1);
+    __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out2);
+    if (!swiglu) {
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n = t.n * BN + c * 32;
+        tmem_ld32(tl + c * 32, v);
+        if (n < F) {
+          store_bf16x32(U + row * F + n, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+          store_bf16x32(H + row * F + n, v);
+        }
+      }
+    } else {
+      float w[32];
+#pragma unroll 1
+      for (int c = 0; c < BN / 64; ++c) {
+        const int n = t.n * (BN / 2) + c * 32;
+        tmem_ld32(tl + c * 32, v);                 // U columns
+        tmem_ld32(tl + BN / 2 + c * 32, w);        // V columns
+        if (n < F) {
+          store_bf16x32(U + row * F + n, v);
+          store_bf16x32(V + row * F + n, w);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = v[i] * sigmoid_f(v[i]) * w[i];
+          store_bf16x32(H + row * F + n, v);
+        }
+      }
+    }
+  } else if (KIND == DGRAD_H) {
+    const int F = P.N;
+    const __nv_bfloat16* U = reinterpret_cast<const __nv_bfloat16*>(P.aux0);
+    const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(P.aux1);
+    __nv_bfloat16* dU = reinterpret_cast<__nv_bfloat16*>(P.out0);
+    __nv_bfloat16* dV = reinterpret_cast<__nv_bfloat16*>(P.out1);
+    float u[32];
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = t.n * BN + c * 32;
+      tmem_ld32(tl + c * 32, v);
+      if (n < F) {
+        load_bf16x32(U + row * F + n, u);
+        if (!swiglu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= gelu_grad_f(u[i]);
+          store_bf16x32(dU + row * F + n, v);
+        } else {
+          float w[32];
+          load_bf16x32(V + row * F + n, w);
+          float dv[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float s = sigmoid_f(u[i]);
+            dv[i] = v[i] * u[i] * s;
+            v[i] = v[i] * w[i] * s * (1.f + u[i] * (1.f - s));
+          }
+          store_bf16x32(dU + row * F + n, v);
+          store_bf16x32(dV + row * F + n, dv);
+        }
+      }
+    }
+  } else {  // DOWN, DGRAD_X: plain bf16 store
+    const int Nc = P.N;
+    __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(P.out0);
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      const int n = t.n * BN + c * 32;
+      tmem_ld32(tl + c * 32, v);
+      if (n < Nc) store_bf16x32(O + row * Nc + n, v);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------- kernel
+
+template <int KIND>
+__global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = bars;                 // [STAGES]
+  uint64_t* empty = bars + STAGES;       // [STAGES]
+  uint64_t* tfull = bars + 2 * STAGES;   // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* drain = tempty + 2;          // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* tile_start = reinterpret_cast<int*>(tmem_slot + 4);   // [MAX_GROUPS + 1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_groups = P.E + P.S;
+
+  // per-group tile counts, then an exclusive prefix (warp 0)
+  for (int g = threadIdx.x; g < n_groups; g += NUM_THREADS) {
+    int a_row, o_row, rows;
+    bool sh;
+    group_rows(P, g, a_row, o_row, rows, sh);
+    tile_start[g + 1] = group_tiles<KIND>(P, rows);
+  }
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    tile_start[0] = 0;
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  __syncthreads();
+  if (warp == 0) {
+    int carry = 0;
+    for (int base = 1; base <= n_groups; base += 32) {
+      const int i = base + lane;
+      int v = (i <= n_groups) ? tile_start[i] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (i <= n_groups) tile_start[i] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int n_tiles = tile_start[n_groups];
+  const unsigned long long budget = P.timeout_ns;
+  constexpr bool A_MN = (KIND == WGRAD);
+  constexpr bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == WGRAD);
+  constexpr uint32_t IDESC = make_idesc(A_MN, B_MN);
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t outstanding = 0;          // stages with a load in flight not yet seen consumed
+    uint32_t out_phase = 0;            // bit s: phase parity of stage s's last issued load
+    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+      const int nk = k_blocks<KIND>(P, tl);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) { ok = false; break; }
+        outstanding &= ~(1u << stage);
+        mbar_expect_tx(&full[stage], STAGE_BYTES);
+        uint8_t* sA = tiles + stage * STAGE_BYTES;
+        issue_loads<KIND>(P, tl, kb, sA, sA + A_BYTES, &full[stage]);
+        outstanding |= 1u << stage;
+        out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+    if (*abort_flag) {
+      // let our own copies land before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (outstanding & (1u << s)) {
+          volatile int never = 0;
+          wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
+        }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const uint32_t a_step = A_MN ? 2048u : 32u;   // bytes per UMMA_K = 16 step
+    const uint32_t b_step = B_MN ? 2048u : 32u;
+    const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
+    bool issued_any = false;
+    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+      const int nk = k_blocks<KIND>(P, tl);
+      if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, budget)) break;
+      tc_fence_after();
+      const uint32_t dtm = tmem_base + (uint32_t)(acc * BN);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!wait_bounded(&full[stage], phase, abort_flag, budget)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(tiles + stage * STAGE_BYTES);
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = sw128_desc(sa + k * a_step, a_lbo, 1024);
+          const uint64_t bd = sw128_desc(sb + k * b_step, b_lbo, 1024);
+          umma_bf16(dtm, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        issued_any = true;
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+      umma_commit(&tfull[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (*abort_flag && issued_any) {
+      umma_commit(drain);
+      volatile int never = 0;
+      wait_bounded(drain, 0, &never, 20000000ull);
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const int quarter = warp & 3;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+      const int nk = k_blocks<KIND>(P, tl);
+      if (!wait_bounded(&tfull[acc], acc_phase, abort_flag, budget)) break;
+      __syncwarp();
+      tc_fence_after();
+      epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, lane);
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) atomicOr(P.status, MOE_STATUS_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encoder() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 map, 128-byte swizzle.  dims/box innermost first; rank 2 or 3.
+static bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                     const uint32_t* box) {
+  EncodeTiledFn enc = encoder();
+  if (!enc || !base) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  gs[0] = dims[0] * 2;
+  if (rank == 3) gs[1] = dims[0] * dims[1] * 2;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                 uint32_t box_rows) {
+  const uint64_t d[2] = {inner, rows};
+  const uint32_t b[2] = {box_inner, box_rows};
+  return make_map(m, base, 2, d, b);
+}
+static bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                 uint32_t box_inner, uint32_t box_mid) {
+  const uint64_t d[3] = {inner, mid, outer};
+  const uint32_t b[3] = {box_inner, box_mid, 1};
+  return make_map(m, base, 3, d, b);
+}
+
+static int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+static unsigned long long g_timeout_ns = 2000000000ull;  // 2 s per wait
+
+template <int KIND>
+static moe_status launch(const Params& P, int max_tiles, cudaStream_t st) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    attr_done = true;
+  }
+  const int grid = max_tiles < num_sms() ? (max_tiles > 0 ? max_tiles : 1) : num_sms();
+  grouped_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(P);
+  return launch_status();
+}
+
+static Params base_params(const Dims& D, const int32_t* offsets, uint32_t* status) {
+  Params P;
+  memset(&P, 0, sizeof(P));
+  P.offsets = offsets;
+  P.status = status;
+  P.timeout_ns = g_timeout_ns;
+  P.T_pad = D.T_pad;
+  P.E = D.E;
+  P.S = D.S;
+  P.T = D.T;
+  P.act = D.act;
+  return P;
+}
+
+// Upper bound on the tiles of a row GEMM (every group at its largest).
+static int row_tiles_bound(const Dims& D, int n_tiles_n) {
+  return (int)((D.R / BM) * n_tiles_n);
+}
+
+}  // namespace tc
+
+bool tc_supported(const Dims& D) {
+  return D.dtype == MOE_DTYPE_BF16 && D.d % 64 == 0 && D.F % 64 == 0 && D.E + D.S <= tc::MAX_GROUPS &&
+         tc::encoder() != nullptr;
+}
+
+void tc_set_timeout_ns(unsigned long long ns) { tc::g_timeout_ns = ns; }
+
+using namespace tc;
+
+moe_status launch_expert_up_tc(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
+                               const void* W1, const void* W3, void* U, void* V, void* H,
+                               uint32_t* status, cudaStream_t st) {
+  Params P = base_params(D, offsets, status);
+  const bool sw = D.act == MOE_ACT_SWIGLU;
+  const uint32_t bbox = sw ? BN / 2 : BN;
+  bool ok = map2(&P.a_main, Xd, D.d, D.R, 64, BM) && map2(&P.a_alt, x, D.d, D.T, 64, BM) &&
+            map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, bbox);
+  if (sw) ok = ok && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, bbox);
+  if (!ok) return MOE_ERR_CUDA;
+  P.out0 = U;
+  P.out1 = V;
+  P.out2 = H;
+  P.N = D.F;
+  P.K = D.d;
+  const int nt = (D.F + bbox - 1) / bbox;
+  return launch<UP>(P, row_tiles_bound(D, nt), st);
+}
+
+moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* offsets,
+                                 const void* W2, void* O, uint32_t* status, cudaStream_t st) {
+  Params P = base_params(D, offsets, status);
+  if (!(map2(&P.a_main, H, D.F, D.R, 64, BM) && map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, BN)))
+    return MOE_ERR_CUDA;
+  P.out0 = O;
+  P.N = D.d;
+  P.K = D.F;
+  return launch<DOWN>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
+}
+
+moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, const int32_t* offsets,
+                             const void* W2, const void* U, const void* V, void* dU, void* dV,
+                             uint32_t* status, cudaStream_t st) {
+  Params P = base_params(D, offsets, status);
+  if (!(map2(&P.a_main, dO, D.d, D.R, 64, BM) && map2(&P.a_alt, dy, D.d, D.T, 64, BM) &&
+        map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, 64)))
+    return MOE_ERR_CUDA;
+  P.aux0 = U;
+  P.aux1 = V;
+  P.out0 = dU;
+  P.out1 = dV;
+  P.N = D.F;
+  P.K = D.d;
+  return launch<DGRAD_H>(P, row_tiles_bound(D, (D.F + BN - 1) / BN), st);
+}
+
+moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
+                             const void* W1, const void* W3, void* dXd, uint32_t* status,
+                             cudaStream_t st) {
+  Params P = base_params(D, offsets, status);
+  bool ok = map2(&P.a_main, dU, D.F, D.R, 64, BM) && map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, 64);
+  if (D.act == MOE_ACT_SWIGLU)
+    ok = ok && map2(&P.a_alt, dV, D.F, D.R, 64, BM) && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, 64);
+  if (!ok) return MOE_ERR_CUDA;
+  P.out0 = dXd;
+  P.N = D.d;
+  P.K = D.F;
+  return launch<DGRAD_X>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
+}
+
+// dW1 (and dW3) = dU^T X  -- M = F, N = d, K = the group's rows.
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xd,
+                               const void* x, const int32_t* offsets, float* dW1, float* dW3,
+                               uint32_t* status, cudaStream_t st) {
+  for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
+    Params P = base_params(D, offsets, status);
+    if (!(map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64) && map2(&P.b_main, Xd, D.d, D.R, 64, 64) &&
+          map2(&P.b_alt, x, D.d, D.T, 64, 64)))
+      return MOE_ERR_CUDA;
+    P.out0 = pass ? dW3 : dW1;
+    P.Mw = D.F;
+    P.N = D.d;
+    P.which = 0;
+    const int tiles = D.E_tot * ((D.F + BM - 1) / BM) * ((D.d + BN - 1) / BN);
+    const moe_status s = launch<WGRAD>(P, tiles, st);
+    if (s != MOE_OK) return s;
+  }
+  return MOE_OK;
+}
+
+// dW2 = dO^T H  -- M = d, N = F.
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, const void* dy,
+                              const int32_t* offsets, float* dW2, uint32_t* status,
+                              cudaStream_t st) {
+  Params P = base_params(D, offsets, status);
+  if (!(map2(&P.a_main, dO, D.d, D.R, 64, 64) && map2(&P.a_alt, dy, D.d, D.T, 64, 64) &&
+        map2(&P.b_main, H, D.F, D.R, 64, 64)))
+    return MOE_ERR_CUDA;
+  P.out0 = dW2;
+  P.Mw = D.d;
+  P.N = D.F;
+  P.which = 2;
+  const int tiles = D.E_tot * ((D.d + BM - 1) / BM) * ((D.F + BN - 1) / BN);
+  return launch<WGRAD>(P, tiles, st);
+}
+
+}  // namespace moe

@@ -40,4 +40,25 @@ moe_status launch_wgrad_w13_simt(const Dims& D, const void* dU, const void* dV, 
 moe_status launch_wgrad_w2_simt(const Dims& D, const void* H, const void* dO, const void* dy,
                                 const int32_t* offsets, float* dW2, cudaStream_t st);
 
+// tcgen05 engine (bf16, d and F multiples of 64)
+bool tc_supported(const Dims& D);
+void tc_set_timeout_ns(unsigned long long ns);
+moe_status launch_expert_up_tc(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
+                               const void* W1, const void* W3, void* U, void* V, void* H,
+                               uint32_t* status, cudaStream_t st);
+moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* offsets,
+                                 const void* W2, void* O, uint32_t* status, cudaStream_t st);
+moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, const int32_t* offsets,
+                             const void* W2, const void* U, const void* V, void* dU, void* dV,
+                             uint32_t* status, cudaStream_t st);
+moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
+                             const void* W1, const void* W3, void* dXd, uint32_t* status,
+                             cudaStream_t st);
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xd,
+                               const void* x, const int32_t* offsets, float* dW1, float* dW3,
+                               uint32_t* status, cudaStream_t st);
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, const void* dy,
+                              const int32_t* offsets, float* dW2, uint32_t* status,
+                              cudaStream_t st);
+
 }  // namespace moe

@@ -39,13 +39,22 @@ def test_small_layers_match_oracle(shape):
                          ids=lambda s: s.name)
 def test_full_size_layers_match_oracle(shape):
     """The three smaller named layers at full size, every element compared."""
+    _assert_engine(shape)
     _parity().full_compare(shape, seed=0)
+
+
+def _assert_engine(shape):
+    """bf16 layers with d, F multiples of 64 must run on the tcgen05 engine, fp32 on CUDA cores."""
+    from mixture_experts_layer_23_b200 import moe
+    want = 1 if (shape.dtype == BF16 and shape.d % 64 == 0 and shape.d_ff % 64 == 0) else 0
+    assert moe.gemm_engine(moe.make_config(shape)) == want
 
 
 @pytest.mark.parametrize("shape", [s for s in LAYERS if s.name in
                                    ("mixtral_dropless", "deepseek_v2")], ids=lambda s: s.name)
 def test_full_size_layers_sampled(shape):
     """The two large named layers at full size: routing and dispatch in full, values sampled."""
+    _assert_engine(shape)
     _parity().sampled_compare(shape, seed=0)
 
 
