@@ -52,7 +52,7 @@ typedef enum {
   MOE_ERR_INVALID_ARG = 1,         /* null pointer, non-positive size, k > E, ... */
   MOE_ERR_UNSUPPORTED = 2,         /* valid but outside this build's limits (see moe_config_t) */
   MOE_ERR_MISALIGNED = 3,          /* a pointer is not 16-byte aligned */
-  MOE_ERR_WORKSPACE_TOO_SMALL = 4, /* reserved: sizes are not passed in, see moe_workspace_size */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4, /* the library's fixed scratch is too small (moe_dispatch_noalloc) */
   MOE_ERR_CUDA = 5,                /* a CUDA launch or runtime call failed */
   MOE_ERR_DEVICE_TIMEOUT = 6       /* a bounded device-side wait gave up (moe_read_status) */
 } moe_status;
@@ -116,6 +116,26 @@ moe_status moe_route_from_logits(const moe_config_t* cfg, const float* logits, i
 moe_status moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                         int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
                         int32_t* row_token, void* Xd, void* scratch, moe_stream_t stream);
+
+/* moe_dispatch for callers that cannot allocate device memory.  The pages have no counterpart to
+ * this entry point; it exists for deployments, not for the method.
+ * Some callers cannot hand the library a scratch buffer: a host framework that owns all device
+ * memory through its own fixed pool and does not expose it to plug-ins, a deployment whose memory
+ * is budgeted once at start-up so a later allocation could fail, or a latency-critical loop that
+ * cannot afford an allocation's cost.  This call takes the same arguments as moe_dispatch minus
+ * `scratch`, produces identical outputs, and allocates nothing: the per-CTA expert histograms live
+ * in a fixed 256 KB array inside the library, which every GPU that loads the library holds until
+ * the process exits.
+ * Limit: ceil(T / 256) * E <= 65536 (for example T = 65536 with E = 256, or T = 2^20 with E = 16);
+ * larger configs return MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ * The first call on a device looks up the array's device address with that device current; make
+ * that first call before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (for example on two streams) race
+ * and corrupt each other's results, so serialise them.  The array keeps the last call's contents;
+ * each call rewrites every entry it reads, so nothing needs clearing. */
+moe_status moe_dispatch_noalloc(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                                int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
+                                int32_t* row_token, void* Xd, moe_stream_t stream);
 
 /* Step 3, the expert FFNs as grouped GEMMs over the row space.
  * GELU: U = Xd W1_e^T, H = gelu(U);  SwiGLU: U = Xd W1_e^T, V = Xd W3_e^T, H = silu(U) * V;

@@ -16,6 +16,8 @@
 //               order), counts, kept = min(counts, C) and the 128-row aligned segment offsets.
 //   3. scatter: one warp per token finalises its slots and copies its x row (16-byte vectors,
 //               read once, written to each kept slot); extra CTAs zero the padding rows.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -166,4 +168,55 @@ moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx
   return MOE_OK;
 }
 
+// ----------------------------------------------------------------------------- no-allocation form
+//
+// moe_dispatch_noalloc: the same dispatch for callers that cannot allocate device memory.  The
+// per-CTA expert histograms (the only scratch the dispatch needs) live in a fixed array inside
+// this library instead of a caller-supplied buffer.  Every device that loads the library holds the
+// array (256 KB) until the process exits.  All calls share it, so calls that overlap on the GPU
+// race; it keeps the last call's contents, and needs no clearing because the rank kernel writes
+// every entry a call reads before the scan reads it.
+
+constexpr int kNoAllocMaxHistogram = 1 << 16;  // int32 entries: ceil(T / 256) * E must fit
+static __device__ __align__(256) int32_t g_noalloc_histogram[kNoAllocMaxHistogram];
+
+// Device address of the array on the current device, looked up once per device (with that device
+// current, on its first call).  In host code the array's name is only a host-side stand-in, so the
+// kernels must be given this address, never the name.
+static moe_status noalloc_histogram(int32_t** out) {
+  constexpr int kMaxDevices = 64;
+  static int32_t* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_histogram) != cudaSuccess || !p) return MOE_ERR_CUDA;
+    addr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = addr[dev];
+  return MOE_OK;
+}
+
 }  // namespace moe
+
+extern "C" moe_status moe_dispatch_noalloc(const moe_config_t* cfg, const void* x,
+                                           const int32_t* topk_idx, int32_t* counts, int32_t* kept,
+                                           int32_t* offsets, int32_t* slot, int32_t* row_token,
+                                           void* Xd, moe_stream_t stream) {
+  moe::Dims D;
+  const moe_status s = moe::resolve_dims(cfg, &D);
+  if (s != MOE_OK) return s;
+  const void* ptrs[] = {x, topk_idx, counts, kept, offsets, slot, row_token, Xd};
+  for (const void* p : ptrs) {
+    if (!p) return MOE_ERR_INVALID_ARG;
+    if (((uintptr_t)p & 15u) != 0) return MOE_ERR_MISALIGNED;
+  }
+  if ((int64_t)D.n_blk * D.E > moe::kNoAllocMaxHistogram) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  int32_t* hist = nullptr;
+  const moe_status h = moe::noalloc_histogram(&hist);
+  if (h != MOE_OK) return h;
+  return moe::launch_dispatch(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd, hist,
+                              (cudaStream_t)stream);
+}

@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_bwd",
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
-           "moe_kernel_launches", "moe_set_profile_events")
+           "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -67,6 +67,7 @@ def _load():
         "moe_route": [CP, P, P, P, P, P, P, P],
         "moe_route_from_logits": [CP, P, P, P, P],
         "moe_dispatch": [CP, P, P, P, P, P, P, P, P, P, P],
+        "moe_dispatch_noalloc": [CP, P, P, P, P, P, P, P, P, P],
         "moe_expert_ffn": [CP, P, P, P, P, P, P, P, P, P, P, P, P],
         "moe_combine": [CP, P, P, P, P, P],
         "moe_layer_fwd": [CP, P, P, P, P, P, P, P, P, P, P],
@@ -171,6 +172,13 @@ def dispatch(cfg, x, topk_idx, counts, kept, offsets, slot, row_token, Xd, scrat
     _check(_lib.moe_dispatch(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(counts), _p(kept),
                              _p(offsets), _p(slot), _p(row_token), _p(Xd), _p(scratch),
                              _stream(stream)), "moe_dispatch")
+
+
+def dispatch_noalloc(cfg, x, topk_idx, counts, kept, offsets, slot, row_token, Xd, stream=None):
+    """moe_dispatch without a scratch argument (for callers that cannot allocate; see moe.h)."""
+    _check(_lib.moe_dispatch_noalloc(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(counts), _p(kept),
+                                     _p(offsets), _p(slot), _p(row_token), _p(Xd),
+                                     _stream(stream)), "moe_dispatch_noalloc")
 
 
 def expert_ffn(cfg, Xd, x, offsets, W1, W3, W2, U, V, H, O, scratch, stream=None):
