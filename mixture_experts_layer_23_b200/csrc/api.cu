@@ -224,6 +224,9 @@ moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, con
   MOE_TRY(resolve_dims(cfg, &D));
   MOE_TRY(check_ptrs({x, Wg, logits, topk_idx, topk_w}));
   if (D.has_bias) MOE_TRY(check_ptrs({bias}));
+  if (router_tc_supported(D))
+    return launch_router_tc(D, x, Wg, bias, logits, topk_idx, topk_w, nullptr,
+                            (cudaStream_t)stream);
   return launch_router(D, x, Wg, bias, logits, topk_idx, topk_w, (cudaStream_t)stream);
 }
 
@@ -296,7 +299,10 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   void* H = c + L.ctx_H;
   void* O = c + L.ctx_O;
   MOE_TRY(mark_fwd(0, st));
-  MOE_TRY(launch_router(D, x, Wg, bias, logits, idx, w, st));
+  if (router_tc_supported(D))
+    MOE_TRY(launch_router_tc(D, x, Wg, bias, logits, idx, w, (uint32_t*)(s + S.status), st));
+  else
+    MOE_TRY(launch_router(D, x, Wg, bias, logits, idx, w, st));
   MOE_TRY(mark_fwd(1, st));
   MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
                           (int32_t*)(s + S.blk_counts), st));
@@ -342,9 +348,9 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   float* dl = (float*)(s + S.dlogits);
   float* part = (float*)(s + S.dWg_part);
   MOE_TRY(mark_bwd(0, st));
-  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, kept, offsets, dg, dO, st));
+  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, dg, dl, dO, st));
   MOE_TRY(mark_bwd(1, st));
-  MOE_TRY(launch_router_bwd(D, logits, idx, w, dg, x, dl, part, dWg, st));
+  MOE_TRY(launch_router_wgrad(D, dl, x, part, dWg, st));
   MOE_TRY(mark_bwd(2, st));
   MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, U, V, H, dU, dV, dXd, dW1, dW3, dW2,
                      (uint32_t*)(s + S.status), st));

@@ -16,11 +16,11 @@ moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx
 moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
                           void* y, cudaStream_t st);
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
-                              const float* topk_w, const int32_t* kept, const int32_t* offsets,
-                              float* dg, void* dO, cudaStream_t st);
-moe_status launch_router_bwd(const Dims& D, const float* logits, const int32_t* topk_idx,
-                             const float* topk_w, const float* dg, const void* x, float* dlogits,
-                             float* part, float* dWg, cudaStream_t st);
+                              const float* topk_w, const int32_t* topk_idx, const float* logits,
+                              const int32_t* kept, const int32_t* offsets, float* dg,
+                              float* dlogits, void* dO, cudaStream_t st);
+moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
+                               float* dWg, cudaStream_t st);
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
                              const int32_t* slot, void* dx, cudaStream_t st);
 moe_status launch_expert_up_simt(const Dims& D, const void* Xd, const void* x,
@@ -40,9 +40,14 @@ moe_status launch_wgrad_w13_simt(const Dims& D, const void* dU, const void* dV, 
 moe_status launch_wgrad_w2_simt(const Dims& D, const void* H, const void* dO, const void* dy,
                                 const int32_t* offsets, float* dW2, cudaStream_t st);
 
+// tcgen05 router (bf16, d a multiple of 64, E <= 256); status may be null
+bool router_tc_supported(const Dims& D);
+moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const float* bias,
+                            float* logits, int32_t* topk_idx, float* topk_w, uint32_t* status,
+                            cudaStream_t st);
+
 // tcgen05 engine (bf16, d and F multiples of 64)
 bool tc_supported(const Dims& D);
-void tc_set_timeout_ns(unsigned long long ns);
 moe_status launch_expert_up_tc(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
                                const void* W1, const void* W3, void* U, void* V, void* H,
                                uint32_t* status, cudaStream_t st);

@@ -4,10 +4,12 @@
 // step 1: a small router, replicated on every device, gates the local tokens).  The top-k gate is
 // the Tutel gate_type {'type': 'top', 'k': ...} of section "框架".
 //
-// One CTA owns 64 tokens: it computes their [64 x E] logit tile on CUDA cores (fp32 FMA, x and
-// Wg staged through shared memory), adds the constant bias, writes the logits, and then each warp
-// runs softmax and a warp-shuffle top-k over its tokens' rows straight from shared memory.
+// This is the CUDA-core form (fp32 layers and shapes the tensor-core router does not take): one
+// CTA owns 64 tokens, computes their [64 x E] logit tile with fp32 FMA (x and Wg staged through
+// shared memory), adds the constant bias and writes the logits; then one thread per token runs
+// the serial softmax + top-k of route_serial.cuh over its row in shared memory.
 #include "common.cuh"
+#include "route_serial.cuh"
 
 namespace moe {
 namespace {
@@ -16,71 +18,6 @@ constexpr int RT_TOK = 64;   // tokens per CTA
 constexpr int RT_EC = 64;    // experts per GEMM pass
 constexpr int RT_BK = 32;    // d per smem stage
 constexpr int RT_THREADS = 256;
-
-// Top-k + gate weights of one token whose E logits are readable at `row` (smem or global).
-// Lane l holds logits l, l+32, ...  Selection key: larger logit first, equal logits -> lower
-// expert index.  Writes topk_idx / topk_w for this token.
-__device__ __forceinline__ void topk_row(const float* row, int E, int k, int gate_norm,
-                                         int32_t* idx_out, float* w_out) {
-  const int lane = threadIdx.x & 31;
-  float v[8];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    v[i] = (e < E) ? row[e] : -INFINITY;
-  }
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, v[i]);
-  m = warp_max(m);
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E) s += expf(v[i] - m);
-  }
-  s = warp_sum(s);
-
-  float chosen_l[8];
-  int chosen_e[8];
-  for (int j = 0; j < k; ++j) {
-    // lane-local best among untaken entries (entries scan in increasing expert index)
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u)) {
-        if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    chosen_l[j] = bv;
-    chosen_e[j] = be;
-  }
-  if (lane == 0) {
-    if (gate_norm == 0) {
-      for (int j = 0; j < k; ++j) {
-        idx_out[j] = chosen_e[j];
-        w_out[j] = expf(chosen_l[j] - m) / s;
-      }
-    } else {
-      float z = 0.f;
-      for (int j = 0; j < k; ++j) z += expf(chosen_l[j] - chosen_l[0]);
-      for (int j = 0; j < k; ++j) {
-        idx_out[j] = chosen_e[j];
-        w_out[j] = expf(chosen_l[j] - chosen_l[0]) / z;
-      }
-    }
-  }
-}
 
 template <typename T>
 __global__ void __launch_bounds__(RT_THREADS)
@@ -137,21 +74,25 @@ router_fwd_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
     const int r = i / E, e = i % E;
     if (t0 + r < T_) logits[(int64_t)(t0 + r) * E + e] = ls[r * (E + 1) + e];
   }
-  const int warp = tid >> 5;
-  for (int r = warp; r < RT_TOK; r += RT_THREADS / 32) {
-    const int t = t0 + r;
-    if (t >= T_) break;
-    topk_row(ls + r * (E + 1), E, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
+  if (tid < RT_TOK && t0 + tid < T_) {
+    const int t = t0 + tid;
+    TopK8 st;
+    topk_init(st);
+    for (int e = 0; e < E; ++e) topk_push(st, ls[tid * (E + 1) + e], e);
+    topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
   }
 }
 
 __global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T_, int E, int k,
                                         int gate_norm, int32_t* __restrict__ topk_idx,
                                         float* __restrict__ topk_w) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (warp >= T_) return;
-  topk_row(logits + (int64_t)warp * E, E, k, gate_norm, topk_idx + (int64_t)warp * k,
-           topk_w + (int64_t)warp * k);
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T_) return;
+  const float* row = logits + (int64_t)t * E;
+  TopK8 st;
+  topk_init(st);
+  for (int e = 0; e < E; ++e) topk_push(st, row[e], e);
+  topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
 }
 
 }  // namespace
@@ -185,8 +126,8 @@ moe_status launch_router(const Dims& D, const void* x, const void* Wg, const flo
 
 moe_status launch_topk_from_logits(const Dims& D, const float* logits, int32_t* topk_idx,
                                    float* topk_w, cudaStream_t st) {
-  const int threads = 256;
-  const int grid = (int)(((int64_t)D.T * 32 + threads - 1) / threads);
+  const int threads = 128;
+  const int grid = (D.T + threads - 1) / threads;
   topk_from_logits_kernel<<<grid, threads, 0, st>>>(logits, D.T, D.E, D.k, D.gate_norm, topk_idx,
                                                     topk_w);
   MOE_LAUNCH_CHECK();

@@ -5,81 +5,13 @@
 // where the experts are, and the replicated router (part 三.2) gets its gradient like any
 // other replicated parameter.  Selection and drops are piecewise constant, so no gradient flows
 // through the chosen indices:
-//   gate_norm 0: p = softmax(l), dp[e] = sum_j [idx_j = e] dg_j, dl = p * (dp - <p, dp>)
-//   gate_norm 1: w = softmax(l[chosen]), dl[chosen] = w * (dg - <w, dg>), 0 elsewhere
+//   (the softmax backward, dl from dg, runs inside the combine backward kernel)
 //   dWg = dl^T x (two-level fixed-order reduction, bit-reproducible)
 //   dx  = dl Wg + sum_j dXd[slot_j] + sum_s dXd[shared row of t]   (a gather, no atomics)
 #include "common.cuh"
 
 namespace moe {
 namespace {
-
-__global__ void __launch_bounds__(256)
-router_dlogits_kernel(const float* __restrict__ logits, const int32_t* __restrict__ topk_idx,
-                      const float* __restrict__ topk_w, const float* __restrict__ dg, int T_,
-                      int E, int k, int gate_norm, float* __restrict__ dlogits) {
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T_) return;
-  int my_e = -1;
-  float my_dg = 0.f, my_w = 0.f;
-  if (lane < k) {
-    my_e = topk_idx[(int64_t)t * k + lane];
-    my_dg = dg[(int64_t)t * k + lane];
-    my_w = topk_w[(int64_t)t * k + lane];
-  }
-  const float* row = logits + (int64_t)t * E;
-  float* out = dlogits + (int64_t)t * E;
-  if (gate_norm == 0) {
-    float l[8];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      l[i] = (e < E) ? row[e] : -INFINITY;
-      m = fmaxf(m, l[i]);
-    }
-    m = warp_max(m);
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      l[i] = (e < E) ? expf(l[i] - m) : 0.f;  // unnormalised p
-      s += l[i];
-    }
-    s = warp_sum(s);
-    const float inv = 1.f / s;
-    float dp[8];
-    float dot = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      l[i] *= inv;
-      dp[i] = 0.f;
-    }
-    for (int j = 0; j < k; ++j) {
-      const int ej = __shfl_sync(0xffffffffu, my_e, j);
-      const float gj = __shfl_sync(0xffffffffu, my_dg, j);
-      if ((ej & 31) == lane) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i == (ej >> 5)) dp[i] += gj;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) dot += l[i] * dp[i];
-    dot = warp_sum(dot);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) out[e] = l[i] * (dp[i] - dot);
-    }
-  } else {
-    float wd = warp_sum(my_w * my_dg);  // lanes >= k contribute 0
-    for (int e = lane; e < E; e += 32) out[e] = 0.f;
-    __syncwarp();
-    if (lane < k) out[my_e] = my_w * (my_dg - wd);
-  }
-}
 
 // Partial dWg over one chunk of tokens and 64 columns of d: part[c][e][i] = sum_t dl[t,e] x[t,i].
 template <typename T>
@@ -194,12 +126,8 @@ undispatch_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
 
 }  // namespace
 
-moe_status launch_router_bwd(const Dims& D, const float* logits, const int32_t* topk_idx,
-                             const float* topk_w, const float* dg, const void* x, float* dlogits,
-                             float* part, float* dWg, cudaStream_t st) {
-  router_dlogits_kernel<<<(D.T + 7) / 8, 256, 0, st>>>(logits, topk_idx, topk_w, dg, D.T, D.E, D.k,
-                                                       D.gate_norm, dlogits);
-  MOE_LAUNCH_CHECK();
+moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
+                               float* dWg, cudaStream_t st) {
   dim3 grid(D.n_tchunk, (D.d + 63) / 64);
   if (D.dtype == MOE_DTYPE_BF16)
     router_wgrad_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(

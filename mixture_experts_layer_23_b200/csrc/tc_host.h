@@ -1,0 +1,27 @@
+// Host-side helpers of the tcgen05 kernels (see tc_host.cu).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+namespace tc {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encoder();
+// bf16 tensor map with 128-byte swizzle; dims and box innermost first, rank 2 or 3.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box);
+bool map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+          uint32_t box_rows);
+bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+          uint32_t box_inner, uint32_t box_mid);
+int num_sms();
+// Time budget of every bounded device wait in the tcgen05 kernels (default 2 s).
+unsigned long long wait_budget_ns();
+void set_wait_budget_ns(unsigned long long ns);
+
+}  // namespace tc
+}  // namespace moe

@@ -1,0 +1,29 @@
+// Host driver for the library's per-token softmax + top-k routine (route_serial.cuh), compiled as
+// plain C++: reads "T E k gate_norm" and T*E logits from stdin, prints for each token its k expert
+// ids and k gate weights.  Used by tests/test_route_serial_host.py against the CPU oracle.
+#define __device__
+#define __forceinline__ inline
+#include <cstdio>
+#include <vector>
+
+#include "../../mixture_experts_layer_23_b200/csrc/route_serial.cuh"
+
+int main() {
+  int T, E, k, gate_norm;
+  if (scanf("%d %d %d %d", &T, &E, &k, &gate_norm) != 4) return 1;
+  std::vector<float> row(E);
+  for (int t = 0; t < T; ++t) {
+    for (int e = 0; e < E; ++e)
+      if (scanf("%f", &row[e]) != 1) return 1;
+    moe::TopK8 st;
+    moe::topk_init(st);
+    for (int e = 0; e < E; ++e) moe::topk_push(st, row[e], e);
+    int idx[8];
+    float w[8];
+    moe::topk_finish(st, k, gate_norm, idx, w);
+    for (int j = 0; j < k; ++j) printf("%d ", idx[j]);
+    for (int j = 0; j < k; ++j) printf("%.9g ", w[j]);
+    printf("\n");
+  }
+  return 0;
+}

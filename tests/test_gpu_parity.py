@@ -71,6 +71,12 @@ EDGE = [
                dtype=BF16, n_shared=1, act=SWIGLU, bias="normal"),
     LayerShape("fp32_shared_only_top1", T=77, d=16, E=2, k=1, d_ff=8, n_shared=2,
                capacity_factor=0.5, dtype=FP32),
+    # tensor-core router at its widest (E = 256 experts, N = 256 accumulator columns), k = 8
+    LayerShape("wide_router_tc", T=300, d=64, E=256, k=8, d_ff=64, capacity_factor=2.0,
+               dtype=BF16, bias="normal"),
+    # tensor-core router with E not a multiple of 16 and a ragged last token tile
+    LayerShape("odd_experts_tc", T=517, d=128, E=13, k=3, d_ff=128, capacity_factor=1.1,
+               dtype=BF16, bias="zipf"),
 ]
 
 
