@@ -44,16 +44,22 @@ constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 4096;
+// Epilogue staging: each epilogue warp owns a ring of NSLOT 4 KB slots (32 rows x 128 B, laid out
+// in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
+constexpr int NSLOT = 2;
+constexpr uint32_t SLOT_BYTES = 32 * 128;
+constexpr uint32_t RING_BYTES = 4 * NSLOT * SLOT_BYTES;
+constexpr size_t MISC_BYTES = 2048;   // barriers, TMEM slot, abort flag, tile prefix
+constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + MISC_BYTES;
+static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
+static_assert(8 * 5 * STAGES + 64 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc area too small");
 
 struct alignas(64) Params {
   CUtensorMap a_main, a_alt, b_main, b_alt;
+  CUtensorMap o0, o1, o2;  // output tensor maps (TMA stores), see the epilogue of each kind
   const int32_t* offsets;
   const void* aux0;      // U (DGRAD_H epilogue)
   const void* aux1;      // V (DGRAD_H epilogue, SwiGLU)
-  void* out0;            // U | O | dU | dXd | dW
-  void* out1;            // V | dV
-  void* out2;            // H
   uint32_t* status;
   unsigned long long timeout_ns;
   long long T_pad;
@@ -200,134 +206,256 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 }
 
 // ----------------------------------------------------------------------------- epilogue
+//
+// Warp q (TMEM lane quarter) owns rows 32q..32q+31 of the tile; lane = row.  A chunk is 64 bf16
+// (or 32 fp32) columns: each lane writes its 128-byte row into a staging slot with the 128-byte
+// swizzle (16-byte unit c of row r lands at unit c ^ (r % 8): conflict-free), the warp fences the
+// writes into the async proxy, and lane 0 hands the 32 x 128 B box to a TMA store.  Stores that
+// fall outside the tensor (a partial last N tile) are clipped by TMA.
+
+struct Ring {
+  uint8_t* base;
+  int next;  // slots taken so far; slot = next % NSLOT.  Stores are issued in take order.
+};
+
+// Take the next slot.  AHEAD = slots taken earlier whose stores are not issued yet.  Take j
+// reuses the slot of take j - NSLOT, whose store must have finished reading shared memory; at
+// this point j - AHEAD stores have been issued, so at most NSLOT - 1 - AHEAD may still be pending.
+template <int AHEAD = 0>
+__device__ __forceinline__ uint8_t* ring_take(Ring& r, int lane) {
+  static_assert(AHEAD < NSLOT, "more slots held than the ring has");
+  if (r.next >= NSLOT && lane == 0) bulk_wait_read<NSLOT - 1 - AHEAD>();
+  __syncwarp();
+  uint8_t* p = r.base + (r.next % NSLOT) * SLOT_BYTES;
+  ++r.next;
+  return p;
+}
+__device__ __forceinline__ void ring_store_2d(Ring& r, const CUtensorMap* map, uint8_t* slot,
+                                              int c0, int c1, int lane) {
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, slot, c0, c1);
+    bulk_commit();
+  }
+}
+__device__ __forceinline__ void ring_store_3d(Ring& r, const CUtensorMap* map, uint8_t* slot,
+                                              int c0, int c1, int c2, int lane) {
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(map, slot, c0, c1, c2);
+    bulk_commit();
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
+// row r of a slot <- 64 values as bf16
+__device__ __forceinline__ void slot_put_bf16(uint8_t* slot, int r, const float* v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    d[q] = make_uint4(pack_bf16(v[8 * q + 0], v[8 * q + 1]), pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                      pack_bf16(v[8 * q + 4], v[8 * q + 5]), pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(slot + r * 128 + ((c ^ (r & 7)) << 4)) =
+        make_uint4(pack_bf16(v[8 * c + 0], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                   pack_bf16(v[8 * c + 4], v[8 * c + 5]), pack_bf16(v[8 * c + 6], v[8 * c + 7]));
 }
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s = reinterpret_cast<const uint4*>(src);
+// half h (32 columns) of row r of a slot <- 32 values as bf16
+__device__ __forceinline__ void slot_put_bf16_half(uint8_t* slot, int r, int h, const float* v) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 u = s[q];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  for (int c = 0; c < 4; ++c) {
+    const int cc = 4 * h + c;
+    *reinterpret_cast<uint4*>(slot + r * 128 + ((cc ^ (r & 7)) << 4)) =
+        make_uint4(pack_bf16(v[8 * c + 0], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                   pack_bf16(v[8 * c + 4], v[8 * c + 5]), pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+  }
+}
+// row r of a slot <- 32 fp32 values
+__device__ __forceinline__ void slot_put_f32(uint8_t* slot, int r, const float* v) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
-      v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<float4*>(slot + r * 128 + ((c ^ (r & 7)) << 4)) =
+        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
+// 64 accumulator columns starting at taddr (two loads, one wait)
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  uint32_t a[32], b[32];
+  tmem_ld32_async(taddr, a);
+  tmem_ld32_async(taddr + 32, b);
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] = __uint_as_float(a[i]);
+    v[32 + i] = __uint_as_float(b[i]);
   }
 }
 
-template <int KIND>
-__device__ __forceinline__ void epilogue_tile(const Params& P, const Tile& t, uint32_t tacc,
-                                              int nk, int quarter, int lane) {
-  const int r = quarter * 32 + lane;                // row inside the tile (= TMEM lane)
-  const uint32_t tl = tacc + ((uint32_t)(quarter * 32) << 16);
-  const bool swiglu = P.act == MOE_ACT_SWIGLU;
-  float v[32];
-  if (KIND == WGRAD) {
-    const int m = t.m * BM + r;   // rows >= Mw still join the warp-collective TMEM loads
-    float* out = reinterpret_cast<float*>(P.out0) + (size_t)t.g * P.Mw * P.N;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int n = t.n * BN + c * 32;
-      if (nk > 0) tmem_ld32(tl + c * 32, v);
-      else {
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-      }
-      if (m < P.Mw && n < P.N) {
-        float4* d = reinterpret_cast<float4*>(out + (size_t)m * P.N + n);
-#pragma unroll
-        for (int q = 0; q < 8; ++q) d[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      }
-    }
-    return;
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
   }
-  const size_t row = (size_t)t.o_row + (size_t)t.m * BM + r;
-  if (KIND == UP) {
-    const int F = P.N;
-    __nv_bfloat16* U = reinterpret_cast<__nv_bfloat16*>(P.out0);
-    __nv_bfloat16* V = reinterpret_cast<__nv_bfloat16*>(P.out1);
-    __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.out2);
-    if (!swiglu) {
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n = t.n * BN + c * 32;
-        tmem_ld32(tl + c * 32, v);
-        if (n < F) {
-          store_bf16x32(U + row * F + n, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
-          store_bf16x32(H + row * F + n, v);
-        }
-      }
-    } else {
-      float w[32];
-#pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        const int n = t.n * (BN / 2) + c * 32;
-        tmem_ld32(tl + c * 32, v);                 // U columns
-        tmem_ld32(tl + BN / 2 + c * 32, w);        // V columns
-        if (n < F) {
-          store_bf16x32(U + row * F + n, v);
-          store_bf16x32(V + row * F + n, w);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = v[i] * sigmoid_f(v[i]) * w[i];
-          store_bf16x32(H + row * F + n, v);
-        }
-      }
-    }
-  } else if (KIND == DGRAD_H) {
-    const int F = P.N;
-    const __nv_bfloat16* U = reinterpret_cast<const __nv_bfloat16*>(P.aux0);
-    const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(P.aux1);
-    __nv_bfloat16* dU = reinterpret_cast<__nv_bfloat16*>(P.out0);
-    __nv_bfloat16* dV = reinterpret_cast<__nv_bfloat16*>(P.out1);
-    float u[32];
+}
+
+// Returns false if the wait for the accumulator timed out.
+template <int KIND>
+__device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
+                                              int q, int lane, Ring& ring, uint64_t* tfull,
+                                              uint32_t parity, volatile int* abort_flag) {
+  const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
+  const bool swiglu = P.act == MOE_ACT_SWIGLU;
+  float a[64];
+  if (KIND == WGRAD) {
+    if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+    __syncwarp();
+    tc_fence_after();
+    const int m_row0 = t.m * BM + q * 32;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       const int n = t.n * BN + c * 32;
-      tmem_ld32(tl + c * 32, v);
-      if (n < F) {
-        load_bf16x32(U + row * F + n, u);
+      if (n >= P.N) break;
+      if (nk > 0) {
+        uint32_t r[32];
+        tmem_ld32_async(tl + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) a[i] = 0.f;
+      }
+      uint8_t* slot = ring_take(ring, lane);
+      slot_put_f32(slot, lane, a);
+      ring_store_3d(ring, &P.o0, slot, n, m_row0, t.g, lane);
+    }
+    return true;
+  }
+  const int row0 = t.o_row + t.m * BM + q * 32;  // first output row of this warp's slab
+  if (KIND == DGRAD_H) {
+    // 32-column steps; U (and V) of the next step are loaded while this step computes, and the
+    // first step's are in flight before the wait for the accumulator.
+    const int F = P.N;
+    const size_t rowoff = (size_t)(row0 + lane) * F;
+    const uint4* U = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux0) + rowoff);
+    const uint4* V = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux1) + rowoff);
+    uint4 pu[4], pv[4];
+    int n = t.n * BN;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) pu[i] = U[n / 8 + i];
+    if (swiglu) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pv[i] = V[n / 8 + i];
+    }
+    if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+    __syncwarp();
+    tc_fence_after();
+#pragma unroll 1
+    for (int ch = 0; ch < BN / 64; ++ch) {
+      n = t.n * BN + ch * 64;
+      if (n >= F) break;
+      uint8_t* su = ring_take(ring, lane);
+      uint8_t* sv = swiglu ? ring_take<1>(ring, lane) : nullptr;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const int ns = n + 32 * h;
+        float u[32], v[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) unpack_bf16x8(pu[i], u + 8 * i);
+        if (swiglu) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) unpack_bf16x8(pv[i], v + 8 * i);
+        }
+        const int nn = ns + 32;
+        if (nn < F && nn < t.n * BN + BN) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) pu[i] = U[nn / 8 + i];
+          if (swiglu) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pv[i] = V[nn / 8 + i];
+          }
+        }
+        uint32_t r[32];
+        tmem_ld32_async(tl + ch * 64 + h * 32, r);
+        tmem_wait_ld();
         if (!swiglu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= gelu_grad_f(u[i]);
-          store_bf16x32(dU + row * F + n, v);
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * gelu_grad_f(u[i]);
+          slot_put_bf16_half(su, lane, h, a);
         } else {
-          float w[32];
-          load_bf16x32(V + row * F + n, w);
-          float dv[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float s = sigmoid_f(u[i]);
-            dv[i] = v[i] * u[i] * s;
-            v[i] = v[i] * w[i] * s * (1.f + u[i] * (1.f - s));
+            const float dh = __uint_as_float(r[i]);
+            a[i] = dh * v[i] * s * (1.f + u[i] * (1.f - s));  // dU
+            v[i] = dh * u[i] * s;                             // dV
           }
-          store_bf16x32(dU + row * F + n, v);
-          store_bf16x32(dV + row * F + n, dv);
+          slot_put_bf16_half(su, lane, h, a);
+          slot_put_bf16_half(sv, lane, h, v);
         }
       }
+      ring_store_2d(ring, &P.o0, su, n, row0, lane);
+      if (swiglu) ring_store_2d(ring, &P.o1, sv, n, row0, lane);
     }
-  } else {  // DOWN, DGRAD_X: plain bf16 store
-    const int Nc = P.N;
-    __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(P.out0);
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int n = t.n * BN + c * 32;
-      tmem_ld32(tl + c * 32, v);
-      if (n < Nc) store_bf16x32(O + row * Nc + n, v);
-    }
+    return true;
   }
+  if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+  __syncwarp();
+  tc_fence_after();
+  if (KIND == UP) {
+    const int F = P.N;
+    if (!swiglu) {
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 64; ++ch) {
+        const int n = t.n * BN + ch * 64;
+        if (n >= F) break;
+        tmem_ld64(tl + ch * 64, a);
+        uint8_t* slot = ring_take(ring, lane);
+        slot_put_bf16(slot, lane, a);
+        ring_store_2d(ring, &P.o0, slot, n, row0, lane);       // U
+#pragma unroll
+        for (int i = 0; i < 64; ++i) a[i] = gelu_f(a[i]);
+        slot = ring_take(ring, lane);
+        slot_put_bf16(slot, lane, a);
+        ring_store_2d(ring, &P.o2, slot, n, row0, lane);       // H
+      }
+    } else {
+      float v[64];
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 128; ++ch) {
+        const int n = t.n * (BN / 2) + ch * 64;
+        if (n >= F) break;
+        tmem_ld64(tl + ch * 64, a);                   // U columns
+        tmem_ld64(tl + BN / 2 + ch * 64, v);          // V columns
+        uint8_t* slot = ring_take(ring, lane);
+        slot_put_bf16(slot, lane, a);
+        ring_store_2d(ring, &P.o0, slot, n, row0, lane);       // U
+        slot = ring_take(ring, lane);
+        slot_put_bf16(slot, lane, v);
+        ring_store_2d(ring, &P.o1, slot, n, row0, lane);       // V
+#pragma unroll
+        for (int i = 0; i < 64; ++i) a[i] = a[i] * sigmoid_f(a[i]) * v[i];
+        slot = ring_take(ring, lane);
+        slot_put_bf16(slot, lane, a);
+        ring_store_2d(ring, &P.o2, slot, n, row0, lane);       // H
+      }
+    }
+    return true;
+  }
+  // DOWN, DGRAD_X: plain bf16 output
+#pragma unroll 1
+  for (int ch = 0; ch < BN / 64; ++ch) {
+    const int n = t.n * BN + ch * 64;
+    if (n >= P.N) break;
+    tmem_ld64(tl + ch * 64, a);
+    uint8_t* slot = ring_take(ring, lane);
+    slot_put_bf16(slot, lane, a);
+    ring_store_2d(ring, &P.o0, slot, n, row0, lane);
+  }
+  return true;
 }
 
 // ----------------------------------------------------------------------------- kernel
@@ -337,7 +465,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* tiles = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // 4 warps x NSLOT slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_base + RING_BYTES);
   uint64_t* full = bars;                 // [STAGES]
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
@@ -471,19 +600,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   } else if (warp >= 2) {
     // ---------------- epilogue
     const int quarter = warp & 3;
+    Ring ring{ring_base + (warp - 2) * NSLOT * SLOT_BYTES, 0};
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
       const int nk = k_blocks<KIND>(P, tl);
-      if (!wait_bounded(&tfull[acc], acc_phase, abort_flag, budget)) break;
-      __syncwarp();
-      tc_fence_after();
-      epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, lane);
+      if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, lane, ring,
+                               &tfull[acc], acc_phase, abort_flag))
+        break;
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait<0>();  // this warp's stores have completed
+    __syncwarp();
   }
   __syncwarp();
   tc_fence_before();
@@ -551,9 +682,9 @@ moe_status launch_expert_up_tc(const Dims& D, const void* Xd, const void* x, con
             map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, bbox);
   if (sw) ok = ok && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, bbox);
   if (!ok) return MOE_ERR_CUDA;
-  P.out0 = U;
-  P.out1 = V;
-  P.out2 = H;
+  ok = map2(&P.o0, U, D.F, D.R, 64, 32) && map2(&P.o2, H, D.F, D.R, 64, 32);
+  if (sw) ok = ok && map2(&P.o1, V, D.F, D.R, 64, 32);
+  if (!ok) return MOE_ERR_CUDA;
   P.N = D.F;
   P.K = D.d;
   const int nt = (D.F + bbox - 1) / bbox;
@@ -565,7 +696,7 @@ moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* of
   Params P = base_params(D, offsets, status);
   if (!(map2(&P.a_main, H, D.F, D.R, 64, BM) && map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, BN)))
     return MOE_ERR_CUDA;
-  P.out0 = O;
+  if (!map2(&P.o0, O, D.d, D.R, 64, 32)) return MOE_ERR_CUDA;
   P.N = D.d;
   P.K = D.F;
   return launch<DOWN>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
@@ -580,8 +711,8 @@ moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, cons
     return MOE_ERR_CUDA;
   P.aux0 = U;
   P.aux1 = V;
-  P.out0 = dU;
-  P.out1 = dV;
+  if (!map2(&P.o0, dU, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
+  if (D.act == MOE_ACT_SWIGLU && !map2(&P.o1, dV, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
   P.N = D.F;
   P.K = D.d;
   return launch<DGRAD_H>(P, row_tiles_bound(D, (D.F + BN - 1) / BN), st);
@@ -595,7 +726,7 @@ moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, cons
   if (D.act == MOE_ACT_SWIGLU)
     ok = ok && map2(&P.a_alt, dV, D.F, D.R, 64, BM) && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, 64);
   if (!ok) return MOE_ERR_CUDA;
-  P.out0 = dXd;
+  if (!map2(&P.o0, dXd, D.d, D.R, 64, 32)) return MOE_ERR_CUDA;
   P.N = D.d;
   P.K = D.F;
   return launch<DGRAD_X>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
@@ -610,7 +741,7 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
     if (!(map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64) && map2(&P.b_main, Xd, D.d, D.R, 64, 64) &&
           map2(&P.b_alt, x, D.d, D.T, 64, 64)))
       return MOE_ERR_CUDA;
-    P.out0 = pass ? dW3 : dW1;
+    if (!map3_f32(&P.o0, pass ? dW3 : dW1, D.d, D.F, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
     P.Mw = D.F;
     P.N = D.d;
     P.which = 0;
@@ -629,7 +760,7 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
   if (!(map2(&P.a_main, dO, D.d, D.R, 64, 64) && map2(&P.a_alt, dy, D.d, D.T, 64, 64) &&
         map2(&P.b_main, H, D.F, D.R, 64, 64)))
     return MOE_ERR_CUDA;
-  P.out0 = dW2;
+  if (!map3_f32(&P.o0, dW2, D.F, D.d, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
   P.Mw = D.d;
   P.N = D.F;
   P.which = 2;

@@ -20,7 +20,7 @@ EncodeTiledFn encoder() {
 
 // bf16 map, 128-byte swizzle.  dims/box innermost first; rank 2 or 3.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-              const uint32_t* box) {
+              const uint32_t* box, int elem) {
   EncodeTiledFn enc = encoder();
   if (!enc || !base) return false;
   cuuint64_t gd[3], gs[2];
@@ -29,9 +29,9 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
     gd[i] = dims[i];
     bx[i] = box[i];
   }
-  gs[0] = dims[0] * 2;
-  if (rank == 3) gs[1] = dims[0] * dims[1] * 2;
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+  gs[0] = dims[0] * elem;
+  if (rank == 3) gs[1] = dims[0] * dims[1] * elem;
+  return enc(m, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -47,6 +47,13 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64
   const uint64_t d[3] = {inner, mid, outer};
   const uint32_t b[3] = {box_inner, box_mid, 1};
   return make_map(m, base, 3, d, b);
+}
+
+bool map3_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+              uint32_t box_inner, uint32_t box_mid) {
+  const uint64_t d[3] = {inner, mid, outer};
+  const uint32_t b[3] = {box_inner, box_mid, 1};
+  return make_map(m, base, 3, d, b, 4);
 }
 
 int num_sms() {

@@ -12,12 +12,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encoder();
-// bf16 tensor map with 128-byte swizzle; dims and box innermost first, rank 2 or 3.
-bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box);
+// Tensor map with 128-byte swizzle over bf16 (elem 2) or fp32 (elem 4) data; dims and box
+// innermost first, rank 2 or 3.
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box,
+              int elem = 2);
 bool map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
           uint32_t box_rows);
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
           uint32_t box_inner, uint32_t box_mid);
+bool map3_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+              uint32_t box_inner, uint32_t box_mid);
 int num_sms();
 // Time budget of every bounded device wait in the tcgen05 kernels (default 2 s).
 unsigned long long wait_budget_ns();
