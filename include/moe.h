@@ -174,6 +174,10 @@ moe_status moe_scratch_grad_offsets(const moe_config_t* cfg, size_t* dg_offset,
  * if the stream reported an error, else MOE_OK. */
 moe_status moe_read_status(moe_stream_t stream, void* scratch);
 
+/* Name and description of the CUDA error behind the most recent MOE_ERR_CUDA in this process
+ * ("" if none).  Process-wide; the text stays valid until the next failure. */
+const char* moe_last_cuda_error(void);
+
 /* Static, human-readable name of a status code. */
 const char* moe_status_string(moe_status s);
 

@@ -1,6 +1,7 @@
 // The C ABI of the MoE layer: argument checks, workspace layout and the call sequences of the
 // forward and backward passes.  Declarations and the contract are in include/moe.h.
 #include <math.h>
+#include <stdio.h>
 #include <string.h>
 
 #include "launch.h"
@@ -8,6 +9,12 @@
 namespace moe {
 
 unsigned long long g_kernel_launches = 0;
+
+static char g_last_cuda_error[256] = "";
+void note_cuda_error(cudaError_t e) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
+           cudaGetErrorString(e));
+}
 
 // Profiling hook (moe_set_profile_events): events recorded between the phases of a pass.
 static cudaEvent_t g_fwd_events[MOE_FWD_PHASES + 1];
@@ -389,6 +396,8 @@ moe_status moe_read_status(moe_stream_t stream, void* scratch) {
   }
   return MOE_OK;
 }
+
+const char* moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {

@@ -128,20 +128,27 @@ moe_status ctx_layout(const Dims& D, moe_layout_t* L);
 
 namespace moe {
 extern unsigned long long g_kernel_launches;  // counted by MOE_LAUNCH_CHECK after each launch
+void note_cuda_error(cudaError_t e);          // remembered for moe_last_cuda_error
 }
 
 #define MOE_LAUNCH_CHECK()                                                   \
   do {                                                                       \
     __atomic_fetch_add(&moe::g_kernel_launches, 1ull, __ATOMIC_RELAXED);     \
     cudaError_t e_ = cudaGetLastError();                                     \
-    if (e_ != cudaSuccess) return MOE_ERR_CUDA;                              \
+    if (e_ != cudaSuccess) {                                                 \
+      moe::note_cuda_error(e_);                                              \
+      return MOE_ERR_CUDA;                                                   \
+    }                                                                        \
   } while (0)
 
 namespace moe {
 // Status of the launch just made (counts it, like MOE_LAUNCH_CHECK).
 inline moe_status launch_status() {
   __atomic_fetch_add(&g_kernel_launches, 1ull, __ATOMIC_RELAXED);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return MOE_OK;
+  note_cuda_error(e);
+  return MOE_ERR_CUDA;
 }
 }  // namespace moe
 

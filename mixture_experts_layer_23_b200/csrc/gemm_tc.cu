@@ -13,14 +13,20 @@
 //   DGRAD_H : dH = A W2, epilogue dU = dH * gelu'(U)  or  dU, dV for SwiGLU   A = dO (or dy)
 //   DGRAD_X : dXd = dU W1 (+ dV W3)
 //   WGRAD   : dW1 = dU^T Xd, dW3 = dV^T Xd (which 0)  or  dW2 = dO^T H (which 2), fp32 out
-// Tiles are 128 x 256 (M x N), K in blocks of 64 (one 128-byte swizzle atom of bf16).
+// Tiles are 256 x 256 (M x N) computed by a pair of CTAs on two SMs with tcgen05.mma.cta_group::2:
+// each CTA stages its own 128 rows of A and its half (128 rows) of B, the pair's leader issues the
+// MMA, and each CTA's TMEM receives its own 128 rows of the fp32 accumulator.  K advances in
+// blocks of 64 (one 128-byte swizzle atom of bf16).
 //
-// CTA organisation (192 threads, one CTA per SM, persistent over tiles):
-//   warp 0      TMA producer: loads A and B tiles into a 4-stage shared-memory ring
-//   warp 1      owns the 512 TMEM columns (two 128x256 fp32 accumulators); one lane issues
-//               tcgen05.mma and commits each stage back to the producer
-//   warps 2..5  epilogue: tcgen05.ld the finished accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31 = tile rows), apply the fused activation, store to HBM
+// CTA organisation (one CTA per SM, clusters of 2, persistent over tiles; see Cfg for the per-kind
+// numbers of epilogue warps and stages):
+//   warp 0      TMA producer: loads this CTA's A and B halves into a 5- or 6-stage ring;
+//               completion is counted on the leader CTA's barrier (cta_group::2 loads)
+//   warp 1      owns 512 TMEM columns (two 128x256 fp32 accumulators, allocated pair-wide); on the
+//               leader, one lane issues the MMAs and commits each stage back to both producers
+//   warps 2..    epilogue: tcgen05.ld the finished accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31 = tile rows; with 8 epilogue warps, warps 2..5 take the first half
+//               of the columns and 6..9 the second), apply the fused activation, store via TMA
 // The two accumulators let the epilogue of one tile overlap the main loop of the next.
 // Every mbarrier wait is bounded: on timeout the kernel records MOE_STATUS_TIMEOUT in the status
 // word, drains its own copies and MMAs (with a bound), frees TMEM and returns.
@@ -31,28 +37,45 @@
 #include "launch.h"
 #include "tc_host.h"
 #include "tc_ptx.cuh"
+#include "act_fast.cuh"
 
 namespace moe {
 namespace tc {
 
-enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
-
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int NUM_THREADS = 192;
+constexpr int BM = 128;           // rows per CTA
+constexpr int BMP = 2 * BM;        // rows per CTA-pair tile (MMA M)
+constexpr int BN = 256;            // MMA N (accumulator columns)
+constexpr int BNH = BN / 2;        // B rows staged by each CTA
+constexpr int BK = 64;
 constexpr uint32_t A_BYTES = BM * BK * 2;           // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr uint32_t B_BYTES = BNH * BK * 2;          // 16 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES; // per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
 // Epilogue staging: each epilogue warp owns a ring of NSLOT 4 KB slots (32 rows x 128 B, laid out
 // in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
 constexpr int NSLOT = 2;
 constexpr uint32_t SLOT_BYTES = 32 * 128;
-constexpr uint32_t RING_BYTES = 4 * NSLOT * SLOT_BYTES;
-constexpr size_t MISC_BYTES = 2048;   // barriers, TMEM slot, abort flag, tile prefix
-constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + MISC_BYTES;
-static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
-static_assert(8 * 5 * STAGES + 64 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc area too small");
+constexpr size_t MISC_BYTES = 1280;   // barriers, TMEM slot, abort flag, tile prefix
+
+enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
+
+// Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
+// up-projection's activation epilogue is the heaviest per output, so it gets 8 epilogue warps (two
+// per TMEM lane quarter, each taking half the columns) and 5 stages; the others keep 4 epilogue
+// warps and 6 stages of loads in flight.  10 warps cap each thread at 168 registers (each SM
+// sub-partition's register file holds 3 of the 10 warps).
+template <int KIND>
+struct Cfg {
+  static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
+  static constexpr int SPLIT = EPI_WARPS / 4;
+  static constexpr int STAGES = (KIND == UP) ? 5 : 6;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr uint32_t RING_BYTES = EPI_WARPS * NSLOT * SLOT_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + MISC_BYTES;
+  static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
+  static_assert(8 * (2 * STAGES + 5) + 16 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc too small");
+};
 
 struct alignas(64) Params {
   CUtensorMap a_main, a_alt, b_main, b_alt;
@@ -71,23 +94,19 @@ struct alignas(64) Params {
   int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
 };
 
-// Instruction descriptor of kind::f16: bf16 x bf16 -> fp32, M = 128, N = BN.
+// Instruction descriptor of the pair MMA: bf16 x bf16 -> fp32, M = 256 (two CTAs), N = BN.
 __host__ __device__ constexpr uint32_t make_idesc(bool a_mn, bool b_mn) {
-  return (1u << 4)                       // D format fp32
-         | (1u << 7)                     // A format bf16
-         | (1u << 10)                    // B format bf16
-         | ((a_mn ? 1u : 0u) << 15)      // A major: 0 K, 1 MN
-         | ((b_mn ? 1u : 0u) << 16)      // B major
-         | ((uint32_t)(BN >> 3) << 17)   // N
-         | ((uint32_t)(BM >> 4) << 24);  // M
+  return idesc_bf16(BMP, BN, a_mn, b_mn);
 }
 
 // ----------------------------------------------------------------------------- scheduling
 
 struct Tile {
-  int g, m, n;           // group, m tile, n tile
+  int g, m, n;           // group, m tile (256 rows), n tile
   int a_row, o_row;      // first row of the group in input- / output-indexed buffers
   int rows;              // group rows (multiple of 128)
+  int mrow;              // first row of this CTA's half, relative to the group (m * 256 + 128 * rank)
+  bool live;             // this CTA's half holds rows of the group
   bool shared;
 };
 
@@ -99,10 +118,14 @@ __device__ __forceinline__ int tile_n(const Params& P) {
 }
 
 template <int KIND>
+__device__ __forceinline__ int m_tiles(const Params& P, int rows) {
+  return ((KIND == WGRAD ? P.Mw : rows) + BMP - 1) / BMP;
+}
+
+template <int KIND>
 __device__ __forceinline__ int group_tiles(const Params& P, int rows) {
   const int nt = (P.N + tile_n<KIND>(P) - 1) / tile_n<KIND>(P);
-  if (KIND == WGRAD) return ((P.Mw + BM - 1) / BM) * nt;
-  return (rows / BM) * nt;
+  return m_tiles<KIND>(P, rows) * nt;
 }
 
 __device__ __forceinline__ void group_rows(const Params& P, int g, int& a_row, int& o_row,
@@ -121,8 +144,8 @@ __device__ __forceinline__ void group_rows(const Params& P, int g, int& a_row, i
 }
 
 template <int KIND>
-__device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, int n_groups,
-                                       int t) {
+__device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, int n_groups, int t,
+                                       int rank) {
   int lo = 0, hi = n_groups - 1;  // last g with tile_start[g] <= t
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -132,9 +155,11 @@ __device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, i
   T.g = lo;
   group_rows(P, lo, T.a_row, T.o_row, T.rows, T.shared);
   const int local = t - tile_start[lo];
-  const int mt = (KIND == WGRAD) ? (P.Mw + BM - 1) / BM : T.rows / BM;
+  const int mt = m_tiles<KIND>(P, T.rows);
   T.m = local % mt;
   T.n = local / mt;
+  T.mrow = T.m * BMP + rank * BM;
+  T.live = T.mrow < (KIND == WGRAD ? P.Mw : T.rows);
   return T;
 }
 
@@ -146,61 +171,60 @@ __device__ __forceinline__ int k_blocks(const Params& P, const Tile& t) {
 }
 
 // ----------------------------------------------------------------------------- producer
+//
+// Each CTA loads its own half: A rows [mrow, mrow + 128) and B rows [nb, nb + 128) with
+// nb = n0 + 128 * rank (for the SwiGLU up-projection: CTA 0 loads W1 rows, CTA 1 the same rows of
+// W3, which makes accumulator columns 0..127 U and 128..255 V).  bar: the leader's full barrier.
 
 template <int KIND>
-__device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int kb, uint8_t* sA,
-                                            uint8_t* sB, uint64_t* bar) {
+__device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int kb, int rank,
+                                            uint8_t* sA, uint8_t* sB, uint32_t bar) {
   const bool swiglu = P.act == MOE_ACT_SWIGLU;
   const int k0 = kb * BK;
+  const int nb = t.n * BN + rank * BNH;
   if (KIND == UP) {
-    const int n0 = t.n * (swiglu ? BN / 2 : BN);
-    if (t.shared) tma_load_2d(sA, &P.a_alt, bar, k0, t.m * BM);
-    else tma_load_2d(sA, &P.a_main, bar, k0, t.a_row + t.m * BM);
-    if (swiglu) {
-      tma_load_3d(sB, &P.b_main, bar, k0, n0, t.g);
-      tma_load_3d(sB + B_BYTES / 2, &P.b_alt, bar, k0, n0, t.g);
-    } else {
-      tma_load_3d(sB, &P.b_main, bar, k0, n0, t.g);
-    }
+    if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
+    else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
+    if (swiglu) tma_load_3d_pair(sB, rank ? &P.b_alt : &P.b_main, bar, k0, t.n * BNH, t.g);
+    else tma_load_3d_pair(sB, &P.b_main, bar, k0, nb, t.g);
   } else if (KIND == DOWN) {
-    tma_load_2d(sA, &P.a_main, bar, k0, t.o_row + t.m * BM);
-    tma_load_3d(sB, &P.b_main, bar, k0, t.n * BN, t.g);
+    tma_load_2d_pair(sA, &P.a_main, bar, k0, t.o_row + t.mrow);
+    tma_load_3d_pair(sB, &P.b_main, bar, k0, nb, t.g);
   } else if (KIND == DGRAD_H) {
-    if (t.shared) tma_load_2d(sA, &P.a_alt, bar, k0, t.m * BM);
-    else tma_load_2d(sA, &P.a_main, bar, k0, t.a_row + t.m * BM);
+    if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
+    else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
 #pragma unroll
-    for (int j = 0; j < BN / 64; ++j)
-      tma_load_3d(sB + j * 8192, &P.b_main, bar, t.n * BN + 64 * j, k0, t.g);
+    for (int j = 0; j < BNH / 64; ++j)
+      tma_load_3d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, k0, t.g);
   } else if (KIND == DGRAD_X) {
     const int nkF = P.K / BK;
     const bool second = kb >= nkF;
     const int kk = (second ? kb - nkF : kb) * BK;
-    tma_load_2d(sA, second ? &P.a_alt : &P.a_main, bar, kk, t.o_row + t.m * BM);
+    tma_load_2d_pair(sA, second ? &P.a_alt : &P.a_main, bar, kk, t.o_row + t.mrow);
 #pragma unroll
-    for (int j = 0; j < BN / 64; ++j)
-      tma_load_3d(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, t.n * BN + 64 * j, kk, t.g);
-  } else {  // WGRAD
-    const int m0 = t.m * BM, n0 = t.n * BN;
+    for (int j = 0; j < BNH / 64; ++j)
+      tma_load_3d_pair(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
+  } else {  // WGRAD: K runs over the group's rows; A and B are read MN-major
     if (P.which == 0) {
       // A = dU|dV rows of the group (row space), B = Xd rows (routed) or x (shared)
 #pragma unroll
       for (int j = 0; j < BM / 64; ++j)
-        tma_load_2d(sA + j * 8192, &P.a_main, bar, m0 + 64 * j, t.o_row + k0);
+        tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
 #pragma unroll
-      for (int j = 0; j < BN / 64; ++j) {
-        if (t.shared) tma_load_2d(sB + j * 8192, &P.b_alt, bar, n0 + 64 * j, k0);
-        else tma_load_2d(sB + j * 8192, &P.b_main, bar, n0 + 64 * j, t.a_row + k0);
+      for (int j = 0; j < BNH / 64; ++j) {
+        if (t.shared) tma_load_2d_pair(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
+        else tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
       }
     } else {
       // A = dO rows (routed) or dy (shared), B = H rows of the group
 #pragma unroll
       for (int j = 0; j < BM / 64; ++j) {
-        if (t.shared) tma_load_2d(sA + j * 8192, &P.a_alt, bar, m0 + 64 * j, k0);
-        else tma_load_2d(sA + j * 8192, &P.a_main, bar, m0 + 64 * j, t.a_row + k0);
+        if (t.shared) tma_load_2d_pair(sA + j * 8192, &P.a_alt, bar, t.mrow + 64 * j, k0);
+        else tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.a_row + k0);
       }
 #pragma unroll
-      for (int j = 0; j < BN / 64; ++j)
-        tma_load_2d(sB + j * 8192, &P.b_main, bar, n0 + 64 * j, t.o_row + k0);
+      for (int j = 0; j < BNH / 64; ++j)
+        tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
     }
   }
 }
@@ -302,10 +326,14 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
 }
 
 // Returns false if the wait for the accumulator timed out.
+// Warp (q, half) covers rows 32q..32q+31 and the half-th of SPLIT column ranges of the
+// accumulator.  Returns false if the wait for the accumulator timed out.
 template <int KIND>
 __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
-                                              int q, int lane, Ring& ring, uint64_t* tfull,
-                                              uint32_t parity, volatile int* abort_flag) {
+                                              int q, int half, int lane, Ring& ring,
+                                              uint64_t* tfull, uint32_t parity,
+                                              volatile int* abort_flag) {
+  constexpr int SPLIT = Cfg<KIND>::SPLIT;
   const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
   const bool swiglu = P.act == MOE_ACT_SWIGLU;
   float a[64];
@@ -313,9 +341,10 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
-    const int m_row0 = t.m * BM + q * 32;
+    if (!t.live) return true;  // this CTA's half of the pair tile lies past the weight rows
+    const int m_row0 = t.mrow + q * 32;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = half * (BN / 32 / SPLIT); c < (half + 1) * (BN / 32 / SPLIT); ++c) {
       const int n = t.n * BN + c * 32;
       if (n >= P.N) break;
       if (nk > 0) {
@@ -334,7 +363,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     }
     return true;
   }
-  const int row0 = t.o_row + t.m * BM + q * 32;  // first output row of this warp's slab
+  const int row0 = t.o_row + t.mrow + q * 32;  // first output row of this warp's slab
   if (KIND == DGRAD_H) {
     // 32-column steps; U (and V) of the next step are loaded while this step computes, and the
     // first step's are in flight before the wait for the accumulator.
@@ -343,18 +372,21 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     const uint4* U = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux0) + rowoff);
     const uint4* V = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux1) + rowoff);
     uint4 pu[4], pv[4];
-    int n = t.n * BN;
+    int n = t.n * BN + half * (BN / SPLIT);
+    if (t.live) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) pu[i] = U[n / 8 + i];
-    if (swiglu) {
+      for (int i = 0; i < 4; ++i) pu[i] = U[n / 8 + i];
+      if (swiglu) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = V[n / 8 + i];
+        for (int i = 0; i < 4; ++i) pv[i] = V[n / 8 + i];
+      }
     }
     if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
+    if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
 #pragma unroll 1
-    for (int ch = 0; ch < BN / 64; ++ch) {
+    for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
       n = t.n * BN + ch * 64;
       if (n >= F) break;
       uint8_t* su = ring_take(ring, lane);
@@ -370,7 +402,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
           for (int i = 0; i < 4; ++i) unpack_bf16x8(pv[i], v + 8 * i);
         }
         const int nn = ns + 32;
-        if (nn < F && nn < t.n * BN + BN) {
+        if (nn < F && nn < t.n * BN + (half + 1) * (BN / SPLIT)) {
 #pragma unroll
           for (int i = 0; i < 4; ++i) pu[i] = U[nn / 8 + i];
           if (swiglu) {
@@ -383,12 +415,12 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
         tmem_wait_ld();
         if (!swiglu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * gelu_grad_f(u[i]);
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * fast::gelu_grad(u[i]);
           slot_put_bf16_half(su, lane, h, a);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float s = sigmoid_f(u[i]);
+            const float s = fast::sigmoid(u[i]);
             const float dh = __uint_as_float(r[i]);
             a[i] = dh * v[i] * s * (1.f + u[i] * (1.f - s));  // dU
             v[i] = dh * u[i] * s;                             // dV
@@ -405,41 +437,79 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
   __syncwarp();
   tc_fence_after();
+  if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
   if (KIND == UP) {
     const int F = P.N;
     if (!swiglu) {
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 64; ++ch) {
+      for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
         const int n = t.n * BN + ch * 64;
         if (n >= F) break;
-        tmem_ld64(tl + ch * 64, a);
-        uint8_t* slot = ring_take(ring, lane);
-        slot_put_bf16(slot, lane, a);
-        ring_store_2d(ring, &P.o0, slot, n, row0, lane);       // U
+        // U, then H = gelu(U), each staged in 32-column halves (TMEM is read twice)
+        for (int o = 0; o < 2; ++o) {
+          uint8_t* slot = ring_take(ring, lane);
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld32_async(tl + ch * 64 + 32 * h, r);
+            tmem_wait_ld();
+            if (o == 0) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) a[i] = gelu_f(a[i]);
-        slot = ring_take(ring, lane);
-        slot_put_bf16(slot, lane, a);
-        ring_store_2d(ring, &P.o2, slot, n, row0, lane);       // H
+              for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) a[i] = fast::gelu(__uint_as_float(r[i]));
+            }
+            slot_put_bf16_half(slot, lane, h, a);
+          }
+          ring_store_2d(ring, o == 0 ? &P.o0 : &P.o2, slot, n, row0, lane);   // U, H
+        }
       }
     } else {
-      float v[64];
+      // U (accumulator columns [0, 128)) and V (columns [128, 256)) of one 64-column chunk, then
+      // H = silu(U) * V; each output is staged in 32-column halves, re-reading TMEM instead of
+      // keeping 128 values live (10 warps leave each thread at most 168 registers).
 #pragma unroll 1
-      for (int ch = 0; ch < BN / 128; ++ch) {
+      for (int ch = half * (2 / SPLIT); ch < (half + 1) * (2 / SPLIT); ++ch) {
         const int n = t.n * (BN / 2) + ch * 64;
         if (n >= F) break;
-        tmem_ld64(tl + ch * 64, a);                   // U columns
-        tmem_ld64(tl + BN / 2 + ch * 64, v);          // V columns
+        const uint32_t tu = tl + ch * 64, tv = tl + BN / 2 + ch * 64;
         uint8_t* slot = ring_take(ring, lane);
-        slot_put_bf16(slot, lane, a);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld32_async(tu + 32 * h, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
+          slot_put_bf16_half(slot, lane, h, a);
+        }
         ring_store_2d(ring, &P.o0, slot, n, row0, lane);       // U
         slot = ring_take(ring, lane);
-        slot_put_bf16(slot, lane, v);
-        ring_store_2d(ring, &P.o1, slot, n, row0, lane);       // V
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld32_async(tv + 32 * h, r);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 64; ++i) a[i] = a[i] * sigmoid_f(a[i]) * v[i];
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
+          slot_put_bf16_half(slot, lane, h, a);
+        }
+        ring_store_2d(ring, &P.o1, slot, n, row0, lane);       // V
         slot = ring_take(ring, lane);
-        slot_put_bf16(slot, lane, a);
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t ru[32], rv[32];
+          tmem_ld32_async(tu + 32 * h, ru);
+          tmem_ld32_async(tv + 32 * h, rv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float u = __uint_as_float(ru[i]);
+            a[i] = u * fast::sigmoid(u) * __uint_as_float(rv[i]);
+          }
+          slot_put_bf16_half(slot, lane, h, a);
+        }
         ring_store_2d(ring, &P.o2, slot, n, row0, lane);       // H
       }
     }
@@ -447,7 +517,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   }
   // DOWN, DGRAD_X: plain bf16 output
 #pragma unroll 1
-  for (int ch = 0; ch < BN / 64; ++ch) {
+  for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
     const int n = t.n * BN + ch * 64;
     if (n >= P.N) break;
     tmem_ld64(tl + ch * 64, a);
@@ -461,22 +531,29 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
 // ----------------------------------------------------------------------------- kernel
 
 template <int KIND>
-__global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __grid_constant__ Params P) {
+__global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ Params P) {
+  constexpr int STAGES = Cfg<KIND>::STAGES;
+  constexpr int NUM_THREADS = Cfg<KIND>::THREADS;
+  constexpr int NUM_EPI_WARPS = Cfg<KIND>::EPI_WARPS;
+  constexpr uint32_t RING_BYTES = Cfg<KIND>::RING_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* tiles = smem;
   uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // 4 warps x NSLOT slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring_base + RING_BYTES);
-  uint64_t* full = bars;                 // [STAGES]
+  uint64_t* full = bars;                 // [STAGES]  (the leader's are the ones used)
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
-  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* tempty = tfull + 2;          // [2]       (the leader's are the ones used)
   uint64_t* drain = tempty + 2;          // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tile_start = reinterpret_cast<int*>(tmem_slot + 4);   // [MAX_GROUPS + 1]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)cluster_ctarank();   // 0 = leader of the pair
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int n_groups = P.E + P.S;
 
   // per-group tile counts, then an exclusive prefix (warp 0)
@@ -495,12 +572,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 128);
+      mbar_init(&tempty[i], 2 * NUM_EPI_WARPS);   // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+  if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
   __syncthreads();
   if (warp == 0) {
     int carry = 0;
@@ -517,7 +594,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     }
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int n_tiles = tile_start[n_groups];
@@ -527,37 +604,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   constexpr uint32_t IDESC = make_idesc(A_MN, B_MN);
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer (both CTAs)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t outstanding = 0;          // stages with a load in flight not yet seen consumed
     uint32_t out_phase = 0;            // bit s: phase parity of stage s's last issued load
-    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
-      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) { ok = false; break; }
         outstanding &= ~(1u << stage);
-        mbar_expect_tx(&full[stage], STAGE_BYTES);
+        if (rank == 0) mbar_expect_tx(&full[stage], 2 * STAGE_BYTES);
         uint8_t* sA = tiles + stage * STAGE_BYTES;
-        issue_loads<KIND>(P, tl, kb, sA, sA + A_BYTES, &full[stage]);
+        issue_loads<KIND>(P, tl, kb, rank, sA, sA + A_BYTES, mapa_shared(smem_u32(&full[stage]), 0));
         outstanding |= 1u << stage;
         out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
     }
-    if (*abort_flag) {
-      // let our own copies land before the CTA exits
+    if (*abort_flag && rank == 0) {
+      // let the pair's copies into stages we armed land before the CTAs exit
       for (int s = 0; s < STAGES; ++s)
         if (outstanding & (1u << s)) {
           volatile int never = 0;
           wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
         }
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------- MMA issuer
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------- MMA issuer (leader CTA only)
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -566,10 +643,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
     const uint32_t b_step = B_MN ? 2048u : 32u;
     const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
     bool issued_any = false;
-    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
-      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
-      if (!wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, budget)) break;
+      if (!wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, budget)) break;
       tc_fence_after();
       const uint32_t dtm = tmem_base + (uint32_t)(acc * BN);
       bool ok = true;
@@ -582,35 +659,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
         for (int k = 0; k < BK / 16; ++k) {
           const uint64_t ad = sw128_desc(sa + k * a_step, a_lbo, 1024);
           const uint64_t bd = sw128_desc(sb + k * b_step, b_lbo, 1024);
-          umma_bf16(dtm, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_pair(dtm, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
         }
         issued_any = true;
-        umma_commit(&empty[stage]);
+        umma_commit_pair(&empty[stage], 0x3);   // frees this stage in both CTAs
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) break;
-      umma_commit(&tfull[acc]);
+      umma_commit_pair(&tfull[acc], 0x3);       // accumulator ready in both CTAs
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     if (*abort_flag && issued_any) {
-      umma_commit(drain);
+      umma_commit_pair_local(drain);
       volatile int never = 0;
       wait_bounded(drain, 0, &never, 20000000ull);
     }
   } else if (warp >= 2) {
-    // ---------------- epilogue
+    // ---------------- epilogue (both CTAs)
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
     Ring ring{ring_base + (warp - 2) * NSLOT * SLOT_BYTES, 0};
+    const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
+                                       mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
-      const Tile tl = decode<KIND>(P, tile_start, n_groups, t);
+    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+      const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
-      if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, lane, ring,
-                               &tfull[acc], acc_phase, abort_flag))
+      if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, half, lane,
+                               ring, &tfull[acc], acc_phase, abort_flag))
         break;
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     if (lane == 0) bulk_wait<0>();  // this warp's stores have completed
@@ -618,28 +699,51 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grouped_gemm_kernel(const __gr
   }
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // the pair's MMAs, copies and TMEM reads are over before either CTA moves on
   if (*abort_flag && threadIdx.x == 0) atomicOr(P.status, MOE_STATUS_TIMEOUT);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
 // ----------------------------------------------------------------------------- host side
 
 
+// Persistent launch: one CTA pair (cluster of 2) per two SMs, at most one pair per tile.
 template <int KIND>
 static moe_status launch(const Params& P, int max_tiles, cudaStream_t st) {
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES) != cudaSuccess)
+    const cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<KIND>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)Cfg<KIND>::SMEM_BYTES);
+    if (e != cudaSuccess) {
+      note_cuda_error(e);
       return MOE_ERR_CUDA;
+    }
     attr_done = true;
   }
-  const int grid = max_tiles < num_sms() ? (max_tiles > 0 ? max_tiles : 1) : num_sms();
-  grouped_gemm_kernel<KIND><<<grid, NUM_THREADS, SMEM_BYTES, st>>>(P);
+  const int max_pairs = num_sms() / 2;
+  const int pairs = max_tiles < max_pairs ? (max_tiles > 0 ? max_tiles : 1) : max_pairs;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Cfg<KIND>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg<KIND>::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, P);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    note_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
   return launch_status();
 }
 
@@ -657,7 +761,8 @@ static Params base_params(const Dims& D, const int32_t* offsets, uint32_t* statu
   return P;
 }
 
-// Upper bound on the tiles of a row GEMM (every group at its largest).
+// Upper bound on the pair tiles of a row GEMM: a group of r rows (a multiple of 128) has
+// ceil(r / 256) <= r / 128 m tiles.
 static int row_tiles_bound(const Dims& D, int n_tiles_n) {
   return (int)((D.R / BM) * n_tiles_n);
 }
@@ -677,24 +782,23 @@ moe_status launch_expert_up_tc(const Dims& D, const void* Xd, const void* x, con
                                uint32_t* status, cudaStream_t st) {
   Params P = base_params(D, offsets, status);
   const bool sw = D.act == MOE_ACT_SWIGLU;
-  const uint32_t bbox = sw ? BN / 2 : BN;
   bool ok = map2(&P.a_main, Xd, D.d, D.R, 64, BM) && map2(&P.a_alt, x, D.d, D.T, 64, BM) &&
-            map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, bbox);
-  if (sw) ok = ok && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, bbox);
+            map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, BNH);
+  if (sw) ok = ok && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, BNH);
   if (!ok) return MOE_ERR_CUDA;
   ok = map2(&P.o0, U, D.F, D.R, 64, 32) && map2(&P.o2, H, D.F, D.R, 64, 32);
   if (sw) ok = ok && map2(&P.o1, V, D.F, D.R, 64, 32);
   if (!ok) return MOE_ERR_CUDA;
   P.N = D.F;
   P.K = D.d;
-  const int nt = (D.F + bbox - 1) / bbox;
-  return launch<UP>(P, row_tiles_bound(D, nt), st);
+  const int tn = sw ? BN / 2 : BN;
+  return launch<UP>(P, row_tiles_bound(D, (D.F + tn - 1) / tn), st);
 }
 
 moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* offsets,
                                  const void* W2, void* O, uint32_t* status, cudaStream_t st) {
   Params P = base_params(D, offsets, status);
-  if (!(map2(&P.a_main, H, D.F, D.R, 64, BM) && map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, BN)))
+  if (!(map2(&P.a_main, H, D.F, D.R, 64, BM) && map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, BNH)))
     return MOE_ERR_CUDA;
   if (!map2(&P.o0, O, D.d, D.R, 64, 32)) return MOE_ERR_CUDA;
   P.N = D.d;
@@ -745,7 +849,7 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
     P.Mw = D.F;
     P.N = D.d;
     P.which = 0;
-    const int tiles = D.E_tot * ((D.F + BM - 1) / BM) * ((D.d + BN - 1) / BN);
+    const int tiles = D.E_tot * ((D.F + BMP - 1) / BMP) * ((D.d + BN - 1) / BN);
     const moe_status s = launch<WGRAD>(P, tiles, st);
     if (s != MOE_OK) return s;
   }
@@ -764,7 +868,7 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
   P.Mw = D.d;
   P.N = D.F;
   P.which = 2;
-  const int tiles = D.E_tot * ((D.d + BM - 1) / BM) * ((D.F + BN - 1) / BN);
+  const int tiles = D.E_tot * ((D.d + BMP - 1) / BMP) * ((D.F + BN - 1) / BN);
   return launch<WGRAD>(P, tiles, st);
 }
 

@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_logits",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_bwd",
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
-           "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc")
+           "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
+           "moe_last_cuda_error")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -33,8 +34,10 @@ BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wg
 class MoEError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} "
-                         f"({_lib.moe_status_string(status).decode()})")
+        detail = _lib.moe_status_string(status).decode()
+        if status == 5:
+            detail += "; " + _lib.moe_last_cuda_error().decode()
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 class Config(ctypes.Structure):
@@ -78,6 +81,7 @@ def _load():
         "moe_gemm_engine": [CP],
         "moe_kernel_launches": [],
         "moe_set_profile_events": [P, P],
+        "moe_last_cuda_error": [],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -85,6 +89,7 @@ def _load():
         fn.restype = I32
     lib.moe_status_string.restype = ctypes.c_char_p
     lib.moe_kernel_launches.restype = ctypes.c_int64
+    lib.moe_last_cuda_error.restype = ctypes.c_char_p
     return lib
 
 
