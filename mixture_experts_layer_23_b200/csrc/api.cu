@@ -73,7 +73,16 @@ moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
   if (D.S > 0 && D.T_pad > mg) mg = D.T_pad;
   D.max_group_rows = mg < MOE_ROW_ALIGN ? MOE_ROW_ALIGN : mg;
   D.n_blk = (D.T + kDispatchTokensPerBlock - 1) / kDispatchTokensPerBlock;
-  D.n_tchunk = (D.T + kRouterBwdTokensPerChunk - 1) / kRouterBwdTokensPerChunk;
+  // token chunks of the router-weight gradient: enough CTAs (chunks x 256-column slices) to fill
+  // the GPU twice, chunks of at least 64 tokens
+  {
+    const int slices = (D.d + 255) / 256;
+    int chunks = (2 * 148 + slices - 1) / slices;
+    const int max_chunks = (D.T + 63) / 64;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    D.n_tchunk = chunks;
+  }
   *out = D;
   return MOE_OK;
 }

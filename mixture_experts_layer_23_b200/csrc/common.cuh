@@ -37,11 +37,10 @@ struct Dims {
   int64_t T_pad, R, routed_row0, max_group_rows;
   int elem;             // bytes per activation element
   int n_blk;            // dispatch blocks
-  int n_tchunk;         // token chunks of the router-weight gradient
+  int n_tchunk;         // token chunks of the router-weight gradient (two-level reduction)
 };
 
 constexpr int kDispatchTokensPerBlock = 256;
-constexpr int kRouterBwdTokensPerChunk = 512;
 
 __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 

@@ -7,15 +7,15 @@
 //
 // Ranking rule: within one expert, assignments are ordered by token index; the first C are kept
 // ("drop by token order").  The rank must be bit-exact and deterministic, so it is computed as a
-// stable counting sort in three launches, none of which waits on another CTA:
+// stable counting sort in two launches, neither of which waits on another CTA:
 //   1. rank:    each CTA takes 256 tokens; per warp, a shared-memory bitmask per expert marks the
 //               lanes (tokens) that chose it, so a popcount of the lower lanes gives each
 //               assignment's rank inside the warp; warp bases make it a rank inside the CTA.
 //               The CTA's per-expert histogram goes to scratch.
-//   2. scan:    one CTA turns the histograms into per-CTA bases (exclusive scan over CTAs, token
-//               order), counts, kept = min(counts, C) and the 128-row aligned segment offsets.
-//   3. scatter: one warp per token finalises its slots and copies its x row (16-byte vectors,
-//               read once, written to each kept slot); extra CTAs zero the padding rows.
+//   2. scatter: every CTA scans the histograms (exclusive over rank CTAs in token order, per
+//               expert) for its bases, kept = min(counts, C) and the 128-row aligned offsets;
+//               then one warp per token finalises its slots and copies its x row (16-byte
+//               vectors, read once, written to each kept slot); extra CTAs zero padding rows.
 #include <mutex>
 
 #include "common.cuh"
@@ -63,55 +63,77 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
   }
 }
 
-__global__ void __launch_bounds__(256)
-dispatch_scan_kernel(int32_t* __restrict__ blk_counts, int n_blk, int E, int64_t C,
-                     int routed_row0, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
-                     int32_t* __restrict__ offsets) {
-  __shared__ int32_t seg[257];
-  const int e = threadIdx.x;
-  if (e < E) {
-    int run = 0;
-    for (int b = 0; b < n_blk; ++b) {
-      const int c = blk_counts[(int64_t)b * E + e];
-      blk_counts[(int64_t)b * E + e] = run;  // becomes the CTA's base for this expert
-      run += c;
-    }
-    counts[e] = run;
-    const int kp = (int64_t)run < C ? run : (int)C;
-    kept[e] = kp;
-    seg[e] = (int)round_up(kp, MOE_ROW_ALIGN);
-  }
-  __syncthreads();
-  if (e == 0) {
-    int run = routed_row0;
-    for (int i = 0; i < E; ++i) {
-      offsets[i] = run;
-      run += seg[i];
-    }
-    offsets[E] = run;
-  }
-}
+// Scan + scatter.  Every CTA first turns the per-rank-CTA histograms into what it needs: the
+// exclusive token-order base of its own tokens' rank-CTA for each expert, the per-expert totals
+// (counts), kept = min(counts, C) and the 128-row aligned segment offsets (CTA 0 also writes
+// counts, kept and offsets out).  This is E x n_blk integer adds per CTA, cheaper than a
+// separate one-CTA launch.  Then one warp per token finalises its slots and copies its x row
+// (16-byte vectors, read once, written to each kept slot); the last E + 1 CTAs zero the padding
+// rows and mark shared rows in row_token.
+constexpr int SC_TOK = 8;   // tokens per scatter CTA (one per warp)
+static_assert(DT % SC_TOK == 0, "a scatter CTA must not straddle two rank CTAs");
 
 template <typename T>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
-                        const int32_t* __restrict__ blk_base, const int32_t* __restrict__ kept,
-                        const int32_t* __restrict__ offsets, int T_, int d, int E, int k,
-                        int64_t C, int n_tok_blocks, int shared_rows,
+                        const int32_t* __restrict__ blk_counts, int n_blk, int T_, int d, int E,
+                        int k, int64_t C, int routed_row0, int n_tok_blocks, int shared_rows,
+                        int32_t* __restrict__ counts_out, int32_t* __restrict__ kept_out,
+                        int32_t* __restrict__ offsets_out,
                         int32_t* __restrict__ slot /* in: local rank, out: slot */,
                         int32_t* __restrict__ row_token, T* __restrict__ Xd) {
+  __shared__ int32_t s_base[256];   // base of this CTA's rank block, per expert
+  __shared__ int32_t s_kept[256];
+  __shared__ int32_t s_off[257];
   constexpr int VN = Vec16<T>::N;
   const int nv = d / VN;
-  const int lane = threadIdx.x & 31;
-  if ((int)blockIdx.x >= n_tok_blocks) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool tok_cta = (int)blockIdx.x < n_tok_blocks;
+  const int my_blk = tok_cta ? (int)(blockIdx.x * SC_TOK / DT) : 0;
+  for (int e = threadIdx.x; e < E; e += 256) {
+    int run = 0, base = 0;
+    for (int b = 0; b < n_blk; ++b) {
+      if (b == my_blk) base = run;
+      run += blk_counts[(int64_t)b * E + e];
+    }
+    const int kp = (int64_t)run < C ? run : (int)C;
+    s_base[e] = base;
+    s_kept[e] = kp;
+    s_off[e + 1] = (int)round_up(kp, MOE_ROW_ALIGN);
+    if (blockIdx.x == 0) {
+      counts_out[e] = run;
+      kept_out[e] = kp;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive prefix of the segment sizes
+    int carry = routed_row0;
+    for (int base = 0; base < E; base += 32) {
+      const int i = base + lane;
+      int v = (i < E) ? s_off[i + 1] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (i < E) s_off[i + 1] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) s_off[0] = routed_row0;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= E; e += 256) offsets_out[e] = s_off[e];
+
+  if (!tok_cta) {
     // padding rows of routed expert e (or, for the last CTA, the shared rows' row_token)
     const int e = blockIdx.x - n_tok_blocks;
     if (e < E) {
-      const int r0 = offsets[e] + kept[e], r1 = offsets[e + 1];
-      for (int r = r0 + (threadIdx.x >> 5); r < r1; r += 8) {
+      const int r0 = s_off[e] + s_kept[e], r1 = s_off[e + 1];
+      Vec16<T> z;
+      z.raw = make_uint4(0, 0, 0, 0);
+      for (int r = r0 + warp; r < r1; r += 8) {
         if (lane == 0) row_token[r] = -1;
-        Vec16<T> z;
-        z.raw = make_uint4(0, 0, 0, 0);
         for (int v = lane; v < nv; v += 32) st_vec(Xd + (int64_t)r * d + (int64_t)v * VN, z);
       }
     } else {
@@ -119,28 +141,31 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
     }
     return;
   }
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T_) return;
-  int my_slot = -1;
-  if (lane < k) {
-    const int e = topk_idx[(int64_t)t * k + lane];
-    const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
-    const int pos = valid ? blk_base[(int64_t)(t / DT) * E + e] + slot[(int64_t)t * k + lane] : 0;
-    if (valid && (int64_t)pos < C) {
-      my_slot = offsets[e] + pos;
-      row_token[my_slot] = t;
+  for (int tt = warp; tt < SC_TOK; tt += 8) {
+    const int t = blockIdx.x * SC_TOK + tt;
+    if (t >= T_) break;
+    int my_slot = -1;
+    if (lane < k) {
+      const int e = topk_idx[(int64_t)t * k + lane];
+      const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
+      const int pos = valid ? s_base[e] + slot[(int64_t)t * k + lane] : 0;
+      if (valid && (int64_t)pos < C) {
+        my_slot = s_off[e] + pos;
+        row_token[my_slot] = t;
+      }
+      slot[(int64_t)t * k + lane] = my_slot;
     }
-    slot[(int64_t)t * k + lane] = my_slot;
-  }
-  int s[8];
+    int sl[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) s[j] = __shfl_sync(0xffffffffu, my_slot, j);
-  const T* src = x + (int64_t)t * d;
-  for (int v = lane; v < nv; v += 32) {
-    const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
+    for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    const T* src = x + (int64_t)t * d;
+#pragma unroll 4
+    for (int v = lane; v < nv; v += 32) {
+      const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < k && s[j] >= 0) st_vec(Xd + (int64_t)s[j] * d + (int64_t)v * VN, val);
+      for (int j = 0; j < 8; ++j)
+        if (j < k && sl[j] >= 0) st_vec(Xd + (int64_t)sl[j] * d + (int64_t)v * VN, val);
+    }
   }
 }
 
@@ -151,19 +176,18 @@ moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx
                            void* Xd, int32_t* blk_counts, cudaStream_t st) {
   dispatch_rank_kernel<<<D.n_blk, 256, 0, st>>>(topk_idx, D.T, D.E, D.k, blk_counts, slot);
   MOE_LAUNCH_CHECK();
-  dispatch_scan_kernel<<<1, 256, 0, st>>>(blk_counts, D.n_blk, D.E, D.C, (int)D.routed_row0,
-                                          counts, kept, offsets);
-  MOE_LAUNCH_CHECK();
-  const int n_tok_blocks = (D.T + 7) / 8;
+  const int n_tok_blocks = (D.T + SC_TOK - 1) / SC_TOK;
   const int grid = n_tok_blocks + D.E + 1;
   if (D.dtype == MOE_DTYPE_BF16)
     dispatch_scatter_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)x, topk_idx, blk_counts, kept, offsets, D.T, D.d, D.E, D.k, D.C,
-        n_tok_blocks, (int)D.routed_row0, slot, row_token, (__nv_bfloat16*)Xd);
+        (const __nv_bfloat16*)x, topk_idx, blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
+        (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets, slot,
+        row_token, (__nv_bfloat16*)Xd);
   else
     dispatch_scatter_kernel<float><<<grid, 256, 0, st>>>(
-        (const float*)x, topk_idx, blk_counts, kept, offsets, D.T, D.d, D.E, D.k, D.C,
-        n_tok_blocks, (int)D.routed_row0, slot, row_token, (float*)Xd);
+        (const float*)x, topk_idx, blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
+        (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets, slot,
+        row_token, (float*)Xd);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }

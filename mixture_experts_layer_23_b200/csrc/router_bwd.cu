@@ -13,48 +13,67 @@
 namespace moe {
 namespace {
 
-// Partial dWg over one chunk of tokens and 64 columns of d: part[c][e][i] = sum_t dl[t,e] x[t,i].
+// Partial dWg over one chunk of tokens: part[c][e][i] = sum_{t in chunk c} dl[t,e] x[t,i].
+// A CTA of 128 threads covers 256 columns (two per thread) and 16 experts at a time (32
+// accumulators per thread).  For every 64 tokens (32 for fp32) it stages the x tile in shared memory
+// with 16-byte loads that are all in flight together, and the matching dl values; the products
+// are then read from shared memory (x as each thread's two columns, dl as broadcasts).
+constexpr int WG_COLS = 256, WG_EC = 16;
+
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 router_wgrad_partial_kernel(const float* __restrict__ dl, const T* __restrict__ x, int T_, int d,
-                            int E, float* __restrict__ part) {
-  __shared__ float ds[32][68];
-  __shared__ float xs[32][68];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int c = blockIdx.x, i0 = blockIdx.y * 64;
-  const int t_begin = c * kRouterBwdTokensPerChunk;
-  const int t_end = min(T_, t_begin + kRouterBwdTokensPerChunk);
-  for (int e0 = 0; e0 < E; e0 += 64) {
-    float acc[4][4] = {};
-    for (int tb = t_begin; tb < t_end; tb += 32) {
-      for (int q = tid; q < 32 * 64; q += 256) {
-        const int r = q / 64, col = q % 64;
+                            int E, int chunk, float* __restrict__ part) {
+  constexpr int VN = Vec16<T>::N;
+  constexpr int WG_TS = 128 / (int)sizeof(T);  // 64 bf16 or 32 fp32 token rows: a 32 KB tile
+  __shared__ __align__(16) T xs[WG_TS][WG_COLS];
+  __shared__ float ds[WG_TS][WG_EC];
+  const int c = blockIdx.x;
+  const int c0 = blockIdx.y * WG_COLS;
+  const int i = 2 * threadIdx.x;           // column inside the slice
+  const int t_begin = c * chunk;
+  const int t_end = min(T_, t_begin + chunk);
+  const bool col_ok = c0 + i < d;
+  for (int e0 = 0; e0 < E; e0 += WG_EC) {
+    float acc0[WG_EC], acc1[WG_EC];
+#pragma unroll
+    for (int e = 0; e < WG_EC; ++e) acc0[e] = acc1[e] = 0.f;
+    for (int tb = t_begin; tb < t_end; tb += WG_TS) {
+      __syncthreads();
+      constexpr int VPR = WG_COLS / VN;   // 16-byte vectors per tile row
+#pragma unroll 4
+      for (int q = threadIdx.x; q < WG_TS * VPR; q += 128) {
+        const int r = q / VPR, v = q % VPR;
+        const int t = tb + r, col = c0 + v * VN;
+        Vec16<T> val;
+        val.raw = make_uint4(0, 0, 0, 0);
+        if (t < t_end && col < d) val = ld_vec(x + (int64_t)t * d + col);
+        st_vec(&xs[r][v * VN], val);
+      }
+      for (int q = threadIdx.x; q < WG_TS * WG_EC; q += 128) {
+        const int r = q / WG_EC, e = q % WG_EC;
         const int t = tb + r;
-        ds[r][col] = (t < t_end && e0 + col < E) ? dl[(int64_t)t * E + e0 + col] : 0.f;
-        xs[r][col] = (t < t_end && i0 + col < d) ? to_f(x[(int64_t)t * d + i0 + col]) : 0.f;
+        ds[r][e] = (t < t_end && e0 + e < E) ? dl[(int64_t)t * E + e0 + e] : 0.f;
       }
       __syncthreads();
-#pragma unroll 8
-      for (int r = 0; r < 32; ++r) {
-        float a[4], b[4];
+      const int nt = min(WG_TS, t_end - tb);
+#pragma unroll 4
+      for (int r = 0; r < nt; ++r) {
+        const float x0 = to_f(xs[r][i]), x1 = to_f(xs[r][i + 1]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) a[q] = ds[r][ty * 4 + q];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) b[q] = xs[r][tx * 4 + q];
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
+        for (int e = 0; e < WG_EC; ++e) {
+          acc0[e] = fmaf(ds[r][e], x0, acc0[e]);
+          acc1[e] = fmaf(ds[r][e], x1, acc1[e]);
+        }
       }
-      __syncthreads();
     }
+    if (col_ok) {
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int e = e0 + ty * 4 + p, i = i0 + tx * 4 + q;
-        if (e < E && i < d) part[((int64_t)c * E + e) * d + i] = acc[p][q];
-      }
+      for (int e = 0; e < WG_EC; ++e)
+        if (e0 + e < E)
+          *reinterpret_cast<float2*>(part + ((int64_t)c * E + e0 + e) * d + c0 + i) =
+              make_float2(acc0[e], acc1[e]);
+    }
   }
 }
 
@@ -67,59 +86,105 @@ __global__ void router_wgrad_reduce_kernel(const float* __restrict__ part, int n
   dWg[i] = s;
 }
 
-// dx for a tile of 64 tokens x 64 columns: dl Wg (K = E on CUDA cores) plus the gathered rows.
+// dx for 32 tokens x (32 * VN) columns: warp w takes tokens w, w+8, w+16, w+24, two at a time;
+// lane l owns the VN columns at 16-byte vector l.  dx = dl Wg (K = E from shared memory) + the
+// token's gathered dXd rows (routed slots in order, then shared experts), a fixed-order sum.  The
+// four tokens' slots are fetched together, and each pair's gathers are issued before the K = E
+// contraction so that their latency overlaps it.
 template <typename T>
 __global__ void __launch_bounds__(256)
 undispatch_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
                   const T* __restrict__ dXd, const int32_t* __restrict__ slot, int T_, int d,
                   int E, int k, int S, int64_t T_pad, T* __restrict__ dx) {
-  __shared__ float ds[64][33];
-  __shared__ float ws[32][68];
-  __shared__ int32_t ss[64][8];
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-  const int t0 = blockIdx.x * 64, i0 = blockIdx.y * 64;
-  for (int q = tid; q < 64 * 8; q += 256) {
-    const int r = q / 8, j = q % 8;
-    ss[r][j] = (t0 + r < T_ && j < k) ? slot[(int64_t)(t0 + r) * k + j] : -1;
+  constexpr int VN = Vec16<T>::N;
+  constexpr int COLS = 32 * VN;
+  extern __shared__ uint4 ud_smem[];
+  T* ws = reinterpret_cast<T*>(ud_smem);                       // [E][COLS]
+  float* dls = reinterpret_cast<float*>(ws + (size_t)E * COLS); // [32][E]
+  const int t0 = blockIdx.x * 32, c0 = blockIdx.y * COLS;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nvec_row = COLS / VN;  // 32
+  for (int q = threadIdx.x; q < E * nvec_row; q += 256) {
+    const int e = q / nvec_row, v = q % nvec_row;
+    const int col = c0 + v * VN;
+    Vec16<T> w;
+    w.raw = make_uint4(0, 0, 0, 0);
+    if (col < d) w = ld_vec(Wg + (int64_t)e * d + col);
+    st_vec(ws + (size_t)e * COLS + v * VN, w);
   }
-  float acc[4][4] = {};
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    for (int q = tid; q < 64 * 32; q += 256) {
-      const int r = q / 32, e = q % 32;
-      ds[r][e] = (t0 + r < T_ && e0 + e < E) ? dl[(int64_t)(t0 + r) * E + e0 + e] : 0.f;
-      const int er = q / 64, col = q % 64;
-      ws[er][col] = (e0 + er < E && i0 + col < d) ? to_f(Wg[(int64_t)(e0 + er) * d + i0 + col]) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int e = 0; e < 32; ++e) {
-      float a[4], b[4];
-#pragma unroll
-      for (int p = 0; p < 4; ++p) a[p] = ds[ty * 4 + p][e];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) b[q] = ws[e][tx * 4 + q];
-#pragma unroll
-      for (int p = 0; p < 4; ++p)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[p][q] = fmaf(a[p], b[q], acc[p][q]);
-    }
-    __syncthreads();
+  for (int q = threadIdx.x; q < 32 * E; q += 256) {
+    const int r = q / E, e = q % E;
+    dls[q] = (t0 + r < T_) ? dl[(int64_t)(t0 + r) * E + e] : 0.f;
   }
+  // slots of this warp's four tokens: lane q < 4k holds slot (token q / k, choice q % k)
+  int my_slot = -1;
+  if (lane < 4 * k) {
+    const int t = t0 + warp + 8 * (lane / k);
+    if (t < T_) my_slot = slot[(int64_t)t * k + (lane % k)];
+  }
+  __syncthreads();
+  const int col = c0 + lane * VN;
+  const bool col_ok = col < d;  // lanes past d stay in the warp: they source slot shuffles
+#pragma unroll 1
+  for (int p = 0; p < 2; ++p) {
+    const int ra = warp + 16 * p, rb = ra + 8;    // the pair's two tokens
+    const int ta = t0 + ra, tb = t0 + rb;
+    if (ta >= T_) break;
+    const bool hb = tb < T_;
+    Vec16<T> ga[8], gb[8];
+    int sa[8], sb[8];
 #pragma unroll
-  for (int p = 0; p < 4; ++p) {
-    const int r = ty * 4 + p, t = t0 + r;
-    if (t >= T_) continue;
+    for (int j = 0; j < 8; ++j) {
+      sa[j] = __shfl_sync(0xffffffffu, my_slot, (2 * p) * k + j);
+      sb[j] = __shfl_sync(0xffffffffu, my_slot, (2 * p + 1) * k + j);
+      if (j >= k || !col_ok) sa[j] = sb[j] = -1;
+      if (!hb) sb[j] = -1;
+      if (sa[j] >= 0) ga[j] = ld_vec_stream(dXd + (int64_t)sa[j] * d + col);
+      if (sb[j] >= 0) gb[j] = ld_vec_stream(dXd + (int64_t)sb[j] * d + col);
+    }
+    float acc_a[VN], acc_b[VN];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = i0 + tx * 4 + q;
-      if (i >= d) continue;
-      float v = acc[p][q];
-      for (int j = 0; j < k; ++j) {
-        const int s = ss[r][j];
-        if (s >= 0) v += to_f(dXd[(int64_t)s * d + i]);
+    for (int i = 0; i < VN; ++i) acc_a[i] = acc_b[i] = 0.f;
+    for (int sj = 0; sj < (col_ok ? S : 0); ++sj) {
+      const Vec16<T> ha = ld_vec_stream(dXd + ((int64_t)sj * T_pad + ta) * d + col);
+#pragma unroll
+      for (int i = 0; i < VN; ++i) acc_a[i] += ha.get(i);
+      if (hb) {
+        const Vec16<T> hbv = ld_vec_stream(dXd + ((int64_t)sj * T_pad + tb) * d + col);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc_b[i] += hbv.get(i);
       }
-      for (int sh = 0; sh < S; ++sh) v += to_f(dXd[((int64_t)sh * T_pad + t) * d + i]);
-      dx[(int64_t)t * d + i] = from_f<T>(v);
+    }
+    float ca[VN], cb[VN];
+#pragma unroll
+    for (int i = 0; i < VN; ++i) ca[i] = cb[i] = 0.f;
+    const float* dla = dls + ra * E;
+    const float* dlb = dls + rb * E;
+    for (int e = 0; e < E; ++e) {
+      const Vec16<T> wv = *reinterpret_cast<const Vec16<T>*>(ws + (size_t)e * COLS + lane * VN);
+      const float wa = dla[e], wb = dlb[e];
+#pragma unroll
+      for (int i = 0; i < VN; ++i) {
+        ca[i] = fmaf(wa, wv.get(i), ca[i]);
+        cb[i] = fmaf(wb, wv.get(i), cb[i]);
+      }
+    }
+    // fixed order: dl Wg, routed rows j = 0..k-1, shared rows
+    Vec16<T> oa, ob;
+#pragma unroll
+    for (int i = 0; i < VN; ++i) {
+      float va = ca[i], vb = cb[i];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (sa[j] >= 0) va += ga[j].get(i);
+        if (sb[j] >= 0) vb += gb[j].get(i);
+      }
+      oa.set(i, va + acc_a[i]);
+      ob.set(i, vb + acc_b[i]);
+    }
+    if (col_ok) {
+      st_vec(dx + (int64_t)ta * d + col, oa);
+      if (hb) st_vec(dx + (int64_t)tb * d + col, ob);
     }
   }
 }
@@ -128,13 +193,14 @@ undispatch_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
 
 moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
                                float* dWg, cudaStream_t st) {
-  dim3 grid(D.n_tchunk, (D.d + 63) / 64);
+  const int chunk = (D.T + D.n_tchunk - 1) / D.n_tchunk;
+  dim3 grid(D.n_tchunk, (D.d + WG_COLS - 1) / WG_COLS);
   if (D.dtype == MOE_DTYPE_BF16)
-    router_wgrad_partial_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        dlogits, (const __nv_bfloat16*)x, D.T, D.d, D.E, part);
+    router_wgrad_partial_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
+        dlogits, (const __nv_bfloat16*)x, D.T, D.d, D.E, chunk, part);
   else
-    router_wgrad_partial_kernel<float><<<grid, 256, 0, st>>>(dlogits, (const float*)x, D.T, D.d,
-                                                             D.E, part);
+    router_wgrad_partial_kernel<float><<<grid, 128, 0, st>>>(dlogits, (const float*)x, D.T, D.d,
+                                                             D.E, chunk, part);
   MOE_LAUNCH_CHECK();
   const int64_t n = (int64_t)D.E * D.d;
   router_wgrad_reduce_kernel<<<(int)((n + 255) / 256), 256, 0, st>>>(part, D.n_tchunk, n, dWg);
@@ -142,17 +208,28 @@ moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* 
   return MOE_OK;
 }
 
+template <typename T>
+static moe_status undispatch_t(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
+                               const int32_t* slot, void* dx, cudaStream_t st) {
+  constexpr int COLS = 32 * Vec16<T>::N;
+  const size_t smem = (size_t)D.E * COLS * sizeof(T) + 32 * (size_t)D.E * sizeof(float);
+  auto kern = undispatch_kernel<T>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  dim3 grid((D.T + 31) / 32, (D.d + COLS - 1) / COLS);
+  kern<<<grid, 256, smem, st>>>(dlogits, (const T*)Wg, (const T*)dXd, slot, D.T, D.d, D.E, D.k,
+                                D.S, D.T_pad, (T*)dx);
+  MOE_LAUNCH_CHECK();
+  return MOE_OK;
+}
+
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
                              const int32_t* slot, void* dx, cudaStream_t st) {
-  dim3 grid((D.T + 63) / 64, (D.d + 63) / 64);
   if (D.dtype == MOE_DTYPE_BF16)
-    undispatch_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        dlogits, (const __nv_bfloat16*)Wg, (const __nv_bfloat16*)dXd, slot, D.T, D.d, D.E, D.k,
-        D.S, D.T_pad, (__nv_bfloat16*)dx);
-  else
-    undispatch_kernel<float><<<grid, 256, 0, st>>>(dlogits, (const float*)Wg, (const float*)dXd,
-                                                   slot, D.T, D.d, D.E, D.k, D.S, D.T_pad,
-                                                   (float*)dx);
+    return undispatch_t<__nv_bfloat16>(D, dlogits, Wg, dXd, slot, dx, st);
+  return undispatch_t<float>(D, dlogits, Wg, dXd, slot, dx, st);
   MOE_LAUNCH_CHECK();
   return MOE_OK;
 }
