@@ -31,7 +31,7 @@
  *  - Dispatched rows: one row space of R rows (see moe_layout_t).  Rows [s*T_pad, s*T_pad + T)
  *    belong to shared expert s (T_pad = T rounded up to 128); routed expert e owns rows
  *    [offsets[e], offsets[e+1]), its kept assignments first (in token order), then zero rows
- *    up to a multiple of 128.  Buffers indexed by this row space: Xd, O [R, d]; U, V, H [R, F].
+ *    up to a multiple of 128.  Buffers indexed by this row space: Xd, O [R, d]; Gu, Gv, H [R, F].
  *  - Grad outputs are overwritten, never accumulated.
  *  - Calls are stream-ordered; concurrent calls on different streams need different scratch.
  */
@@ -86,7 +86,7 @@ typedef struct {
   int64_t routed_row0;    /* first routed row = S * T_pad */
   int64_t max_group_rows; /* largest row count any one expert can own (multiple of 128) */
   size_t ctx_logits, ctx_topk_idx, ctx_topk_w, ctx_counts, ctx_kept, ctx_offsets, ctx_slot,
-      ctx_row_token, ctx_Xd, ctx_U, ctx_V, ctx_H, ctx_O;
+      ctx_row_token, ctx_Xd, ctx_Gu, ctx_Gv, ctx_H, ctx_O;
   size_t ctx_bytes;       /* total ctx size */
   size_t scratch_bytes;   /* total scratch size (forward and backward) */
 } moe_layout_t;
@@ -137,13 +137,17 @@ moe_status moe_dispatch_noalloc(const moe_config_t* cfg, const void* x, const in
                                 int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
                                 int32_t* row_token, void* Xd, moe_stream_t stream);
 
-/* Step 3, the expert FFNs as grouped GEMMs over the row space.
- * GELU: U = Xd W1_e^T, H = gelu(U);  SwiGLU: U = Xd W1_e^T, V = Xd W3_e^T, H = silu(U) * V;
- * O = H W2_e^T.  Shared experts read x directly (all T tokens).  U, V (SwiGLU only, else may
- * be NULL), H are kept for the backward pass.  W3 may be NULL for GELU. */
+/* Step 3, the expert FFNs as grouped GEMMs over the row space, with u = Xd W1_e^T, v = Xd W3_e^T:
+ *   GELU:   H = gelu(u);            Gu = gelu'(u)
+ *   SwiGLU: H = silu(u) * v;        Gu = v s (1 + u (1 - s)),  Gv = silu(u),  s = sigmoid(u)
+ *   O = H W2_e^T.
+ * Gu and Gv are the factors the backward pass needs (dU = dH * Gu, dV = dH * Gv): they are stored
+ * instead of u and v.  Shared experts read x directly (all T tokens).  Gv may be NULL and W3 may
+ * be NULL for GELU. */
 moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x,
                           const int32_t* offsets, const void* W1, const void* W3, const void* W2,
-                          void* U, void* V, void* H, void* O, void* scratch, moe_stream_t stream);
+                          void* Gu, void* Gv, void* H, void* O, void* scratch,
+                          moe_stream_t stream);
 
 /* Step 4, combine: y_t = sum over kept j of topk_w[t,j] * O[slot[t,j]] + sum_s O[s*T_pad + t].
  * A gather in a fixed order: deterministic, no atomics. */

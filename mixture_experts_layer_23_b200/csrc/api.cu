@@ -126,8 +126,8 @@ moe_status ctx_layout(const Dims& D, moe_layout_t* L) {
   L->ctx_slot = take(T * D.k * 4);
   L->ctx_row_token = take(R * 4);
   L->ctx_Xd = take(R * D.d * D.elem);
-  L->ctx_U = take(R * D.F * D.elem);
-  L->ctx_V = (D.act == MOE_ACT_SWIGLU) ? take(R * D.F * D.elem) : 0;
+  L->ctx_Gu = take(R * D.F * D.elem);
+  L->ctx_Gv = (D.act == MOE_ACT_SWIGLU) ? take(R * D.F * D.elem) : 0;
   L->ctx_H = take(R * D.F * D.elem);
   L->ctx_O = take(R * D.d * D.elem);
   L->ctx_bytes = off;
@@ -310,8 +310,8 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   int32_t* slot = (int32_t*)(c + L.ctx_slot);
   int32_t* row_token = (int32_t*)(c + L.ctx_row_token);
   void* Xd = c + L.ctx_Xd;
-  void* U = c + L.ctx_U;
-  void* V = L.ctx_V ? c + L.ctx_V : nullptr;
+  void* U = c + L.ctx_Gu;
+  void* V = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
   void* H = c + L.ctx_H;
   void* O = c + L.ctx_O;
   MOE_TRY(mark_fwd(0, st));
@@ -352,8 +352,8 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   const int32_t* offsets = (const int32_t*)(c + L.ctx_offsets);
   const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
   const void* Xd = c + L.ctx_Xd;
-  const void* U = c + L.ctx_U;
-  const void* V = L.ctx_V ? c + L.ctx_V : nullptr;
+  const void* U = c + L.ctx_Gu;
+  const void* V = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
   const void* H = c + L.ctx_H;
   const void* O = c + L.ctx_O;
   void* dO = s + S.dO;

@@ -85,7 +85,9 @@ __device__ __forceinline__ void mainloop(const View<TA>& A, const View<TB>& B, i
   }
 }
 
-// U = A W1^T (and V = A W3^T); H = gelu(U) or silu(U) * V.
+// u = A W1^T (and v = A W3^T); H = gelu(u) or silu(u) * v.  Instead of u and v, the factors the
+// backward needs are stored: U <- Gu = gelu'(u), or Gu = v s (1 + u (1 - s)) and V <- Gv = silu(u)
+// with s = sigmoid(u).
 template <typename T>
 __global__ void __launch_bounds__(256)
 up_kernel(const T* __restrict__ Xd, const T* __restrict__ x, const int32_t* __restrict__ offsets,
@@ -114,13 +116,15 @@ up_kernel(const T* __restrict__ Xd, const T* __restrict__ x, const int32_t* __re
       if (n >= F) continue;
       const int64_t o = (G.o_row + m) * F + n;
       const float u = au[i][j];
-      U[o] = from_f<T>(u);
       if (act == MOE_ACT_GELU) {
+        U[o] = from_f<T>(gelu_grad_f(u));                  // Gu = GELU'(u)
         H[o] = from_f<T>(gelu_f(u));
       } else {
         const float v = av[i][j];
-        V[o] = from_f<T>(v);
-        H[o] = from_f<T>(u * sigmoid_f(u) * v);
+        const float s = sigmoid_f(u);
+        U[o] = from_f<T>(v * s * (1.f + u * (1.f - s)));   // Gu
+        V[o] = from_f<T>(u * s);                           // Gv = silu(u)
+        H[o] = from_f<T>(u * s * v);
       }
     }
   }
@@ -152,7 +156,7 @@ down_kernel(const T* __restrict__ H, const int32_t* __restrict__ offsets,
   }
 }
 
-// dH = dO W2 (B = W2_e read N-contiguous), then dU = dH * act'(U) (and dV).
+// dH = dO W2 (B = W2_e read N-contiguous), then dU = dH * Gu (and dV = dH * Gv).
 template <typename T>
 __global__ void __launch_bounds__(256)
 dgrad_h_kernel(const T* __restrict__ dO, const T* __restrict__ dy,
@@ -178,15 +182,8 @@ dgrad_h_kernel(const T* __restrict__ dO, const T* __restrict__ dy,
       if (n >= F) continue;
       const int64_t o = (G.o_row + m) * F + n;
       const float dh = acc[i][j];
-      const float u = to_f(U[o]);
-      if (act == MOE_ACT_GELU) {
-        dU[o] = from_f<T>(dh * gelu_grad_f(u));
-      } else {
-        const float v = to_f(V[o]);
-        const float s = sigmoid_f(u);
-        dU[o] = from_f<T>(dh * v * s * (1.f + u * (1.f - s)));
-        dV[o] = from_f<T>(dh * u * s);
-      }
+      dU[o] = from_f<T>(dh * to_f(U[o]));                  // dU = dH * Gu
+      if (act == MOE_ACT_SWIGLU) dV[o] = from_f<T>(dh * to_f(V[o]));   // dV = dH * Gv
     }
   }
 }

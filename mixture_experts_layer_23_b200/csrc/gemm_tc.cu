@@ -8,9 +8,11 @@
 // launch, so a thin expert only costs its own tiles.
 //
 // One kernel, five kinds of grouped GEMM over the dispatched row space (bf16 in, fp32 accumulate):
-//   UP      : [U|V] = A W1^T (W3^T), epilogue H = gelu(U) or silu(U) * V      A = Xd (or x)
+//   UP      : u (and v) = A W1^T (W3^T); epilogue H = gelu(u) or silu(u) * v, plus the factors
+//             the backward needs: Gu = gelu'(u), or Gu = v s (1 + u (1 - s)) and Gv = silu(u)
+//             with s = sigmoid(u)                                             A = Xd (or x)
 //   DOWN    : O = H W2^T
-//   DGRAD_H : dH = A W2, epilogue dU = dH * gelu'(U)  or  dU, dV for SwiGLU   A = dO (or dy)
+//   DGRAD_H : dH = A W2, epilogue dU = dH * Gu (and dV = dH * Gv)             A = dO (or dy)
 //   DGRAD_X : dXd = dU W1 (+ dV W3)
 //   WGRAD   : dW1 = dU^T Xd, dW3 = dV^T Xd (which 0)  or  dW2 = dO^T H (which 2), fp32 out
 // Tiles are 256 x 256 (M x N) computed by a pair of CTAs on two SMs with tcgen05.mma.cta_group::2:
@@ -415,15 +417,14 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
         tmem_wait_ld();
         if (!swiglu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * fast::gelu_grad(u[i]);
+          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * u[i];   // dH * GELU'(u)
           slot_put_bf16_half(su, lane, h, a);
         } else {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float s = fast::sigmoid(u[i]);
             const float dh = __uint_as_float(r[i]);
-            a[i] = dh * v[i] * s * (1.f + u[i] * (1.f - s));  // dU
-            v[i] = dh * u[i] * s;                             // dV
+            a[i] = dh * u[i];   // dU = dH * Gu
+            v[i] = dh * v[i];   // dV = dH * Gv
           }
           slot_put_bf16_half(su, lane, h, a);
           slot_put_bf16_half(sv, lane, h, v);
@@ -445,58 +446,61 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
       for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
         const int n = t.n * BN + ch * 64;
         if (n >= F) break;
-        // U, then H = gelu(U), each staged in 32-column halves (TMEM is read twice)
-        for (int o = 0; o < 2; ++o) {
-          uint8_t* slot = ring_take(ring, lane);
+        // Gu = GELU'(u) (what the backward needs) and H = GELU(u) from one erf evaluation,
+        // staged in 32-column halves into two slots
+        uint8_t* sg = ring_take(ring, lane);
+        uint8_t* sh = ring_take<1>(ring, lane);
 #pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            uint32_t r[32];
-            tmem_ld32_async(tl + ch * 64 + 32 * h, r);
-            tmem_wait_ld();
-            if (o == 0) {
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[32];
+          tmem_ld32_async(tl + ch * 64 + 32 * h, r);
+          tmem_wait_ld();
+          float hv[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) a[i] = fast::gelu(__uint_as_float(r[i]));
-            }
-            slot_put_bf16_half(slot, lane, h, a);
+          for (int i = 0; i < 32; ++i) {
+            const float u = __uint_as_float(r[i]);
+            const fast::ErfParts q = fast::erf_parts(u);
+            const float phi_cdf = fmaf(0.5f, copysignf(q.erf_abs, u), 0.5f);   // Phi(u)
+            a[i] = fmaf(u, 0.39894228040143268f * q.e, phi_cdf);              // GELU'(u)
+            hv[i] = u * phi_cdf;                                               // GELU(u)
           }
-          ring_store_2d(ring, o == 0 ? &P.o0 : &P.o2, slot, n, row0, lane);   // U, H
+          slot_put_bf16_half(sg, lane, h, a);
+          slot_put_bf16_half(sh, lane, h, hv);
         }
+        ring_store_2d(ring, &P.o0, sg, n, row0, lane);   // Gu
+        ring_store_2d(ring, &P.o2, sh, n, row0, lane);   // H
       }
     } else {
-      // U (accumulator columns [0, 128)) and V (columns [128, 256)) of one 64-column chunk, then
-      // H = silu(U) * V; each output is staged in 32-column halves, re-reading TMEM instead of
-      // keeping 128 values live (10 warps leave each thread at most 168 registers).
+      // u (accumulator columns [0, 128)) and v (columns [128, 256)) of one 64-column chunk.
+      // Outputs: Gu = v s (1 + u (1 - s)) and Gv = u s (the backward's factors, s = sigmoid(u)),
+      // then H = u s v.  Two passes over TMEM keep two staging slots enough.
 #pragma unroll 1
       for (int ch = half * (2 / SPLIT); ch < (half + 1) * (2 / SPLIT); ++ch) {
         const int n = t.n * (BN / 2) + ch * 64;
         if (n >= F) break;
         const uint32_t tu = tl + ch * 64, tv = tl + BN / 2 + ch * 64;
-        uint8_t* slot = ring_take(ring, lane);
+        uint8_t* sa = ring_take(ring, lane);
+        uint8_t* sb = ring_take<1>(ring, lane);
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld32_async(tu + 32 * h, r);
+          uint32_t ru[32], rv[32];
+          tmem_ld32_async(tu + 32 * h, ru);
+          tmem_ld32_async(tv + 32 * h, rv);
           tmem_wait_ld();
+          float gv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
-          slot_put_bf16_half(slot, lane, h, a);
+          for (int i = 0; i < 32; ++i) {
+            const float u = __uint_as_float(ru[i]), v = __uint_as_float(rv[i]);
+            const float sg = fast::sigmoid(u);
+            a[i] = v * sg * fmaf(u, 1.f - sg, 1.f);   // Gu
+            gv[i] = u * sg;                            // Gv
+          }
+          slot_put_bf16_half(sa, lane, h, a);
+          slot_put_bf16_half(sb, lane, h, gv);
         }
-        ring_store_2d(ring, &P.o0, slot, n, row0, lane);       // U
-        slot = ring_take(ring, lane);
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld32_async(tv + 32 * h, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]);
-          slot_put_bf16_half(slot, lane, h, a);
-        }
-        ring_store_2d(ring, &P.o1, slot, n, row0, lane);       // V
-        slot = ring_take(ring, lane);
+        ring_store_2d(ring, &P.o0, sa, n, row0, lane);   // Gu
+        ring_store_2d(ring, &P.o1, sb, n, row0, lane);   // Gv
+        uint8_t* sh = ring_take(ring, lane);
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t ru[32], rv[32];
@@ -508,9 +512,9 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
             const float u = __uint_as_float(ru[i]);
             a[i] = u * fast::sigmoid(u) * __uint_as_float(rv[i]);
           }
-          slot_put_bf16_half(slot, lane, h, a);
+          slot_put_bf16_half(sh, lane, h, a);
         }
-        ring_store_2d(ring, &P.o2, slot, n, row0, lane);       // H
+        ring_store_2d(ring, &P.o2, sh, n, row0, lane);   // H
       }
     }
     return true;

@@ -68,8 +68,8 @@ class MoELayer:
             "slot": (L.ctx_slot, INT32, (s.T, s.k)),
             "row_token": (L.ctx_row_token, INT32, (R,)),
             "Xd": (L.ctx_Xd, self.dt, (R, s.d)),
-            "U": (L.ctx_U, self.dt, (R, s.d_ff)),
-            "V": (L.ctx_V, self.dt, (R, s.d_ff)),
+            "Gu": (L.ctx_Gu, self.dt, (R, s.d_ff)),
+            "Gv": (L.ctx_Gv, self.dt, (R, s.d_ff)),
             "H": (L.ctx_H, self.dt, (R, s.d_ff)),
             "O": (L.ctx_O, self.dt, (R, s.d)),
         }

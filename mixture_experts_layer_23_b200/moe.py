@@ -53,7 +53,7 @@ class Layout(ctypes.Structure):
                 ("routed_row0", ctypes.c_int64), ("max_group_rows", ctypes.c_int64)] + [
         (n, ctypes.c_size_t) for n in (
             "ctx_logits", "ctx_topk_idx", "ctx_topk_w", "ctx_counts", "ctx_kept", "ctx_offsets",
-            "ctx_slot", "ctx_row_token", "ctx_Xd", "ctx_U", "ctx_V", "ctx_H", "ctx_O",
+            "ctx_slot", "ctx_row_token", "ctx_Xd", "ctx_Gu", "ctx_Gv", "ctx_H", "ctx_O",
             "ctx_bytes", "scratch_bytes")]
 
 

@@ -53,7 +53,7 @@ def test_layout_capacity_matches_the_capacity_rule(moe):
         worst = min(s.T * s.k, s.E * kmax)
         assert L.rows - L.routed_row0 >= worst
         assert L.ctx_bytes > 0 and L.scratch_bytes > 0
-        for f in ("ctx_logits", "ctx_topk_idx", "ctx_Xd", "ctx_U", "ctx_H", "ctx_O"):
+        for f in ("ctx_logits", "ctx_topk_idx", "ctx_Xd", "ctx_Gu", "ctx_H", "ctx_O"):
             assert getattr(L, f) % 256 == 0
 
 
