@@ -195,7 +195,9 @@ int64_t moe_kernel_launches(void);
  * NULL, or MOE_BWD_PHASES + 1.  While set, moe_layer_fwd records events[0] on its stream before
  * its first launch and events[i] after the launches of phase i (1-based, order below), and
  * moe_layer_bwd does the same with bwd_events.  The caller owns the events and must keep them
- * alive while set.  Process-wide setting; not for concurrent use from several threads.
+ * alive while set.  A NULL entry is not recorded (so a caller can time one phase only: events
+ * between kernels keep consecutive launches from overlapping).  Process-wide setting; not for
+ * concurrent use from several threads.
  *   forward phases:  router, dispatch, expert_up, expert_down, combine
  *   backward phases: combine_bwd, router_bwd, dgrad_h, dgrad_x, wgrad_w1 (and w3), wgrad_w2,
  *                    undispatch */

@@ -1,6 +1,7 @@
 // The C ABI of the MoE layer: argument checks, workspace layout and the call sequences of the
 // forward and backward passes.  Declarations and the contract are in include/moe.h.
 #include <math.h>
+#include <stdlib.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -11,6 +12,14 @@ namespace moe {
 unsigned long long g_kernel_launches = 0;
 
 static char g_last_cuda_error[256] = "";
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_DISABLE_PDL");
+    return !(v && v[0] == '1');
+  }();
+  return on;
+}
 void note_cuda_error(cudaError_t e) {
   snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(e),
            cudaGetErrorString(e));
@@ -22,11 +31,13 @@ static cudaEvent_t g_bwd_events[MOE_BWD_PHASES + 1];
 static bool g_fwd_prof = false, g_bwd_prof = false;
 
 static inline moe_status mark_fwd(int i, cudaStream_t st) {
-  if (g_fwd_prof && cudaEventRecord(g_fwd_events[i], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (g_fwd_prof && g_fwd_events[i] && cudaEventRecord(g_fwd_events[i], st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 static inline moe_status mark_bwd(int i, cudaStream_t st) {
-  if (g_bwd_prof && cudaEventRecord(g_bwd_events[i], st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (g_bwd_prof && g_bwd_events[i] && cudaEventRecord(g_bwd_events[i], st) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return MOE_OK;
 }
 
@@ -383,14 +394,10 @@ int64_t moe_kernel_launches(void) {
 moe_status moe_set_profile_events(void* const* fwd_events, void* const* bwd_events) {
   g_fwd_prof = fwd_events != nullptr;
   g_bwd_prof = bwd_events != nullptr;
-  for (int i = 0; g_fwd_prof && i <= MOE_FWD_PHASES; ++i) {
-    if (!fwd_events[i]) { g_fwd_prof = g_bwd_prof = false; return MOE_ERR_INVALID_ARG; }
-    g_fwd_events[i] = (cudaEvent_t)fwd_events[i];
-  }
-  for (int i = 0; g_bwd_prof && i <= MOE_BWD_PHASES; ++i) {
-    if (!bwd_events[i]) { g_fwd_prof = g_bwd_prof = false; return MOE_ERR_INVALID_ARG; }
+  for (int i = 0; g_fwd_prof && i <= MOE_FWD_PHASES; ++i)
+    g_fwd_events[i] = (cudaEvent_t)fwd_events[i];   // NULL entries are skipped
+  for (int i = 0; g_bwd_prof && i <= MOE_BWD_PHASES; ++i)
     g_bwd_events[i] = (cudaEvent_t)bwd_events[i];
-  }
   return MOE_OK;
 }
 

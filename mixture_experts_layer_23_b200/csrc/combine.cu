@@ -13,50 +13,66 @@
 namespace moe {
 namespace {
 
-template <typename T>
+// y_t = sum_j w_j O[slot_j] + sum_s O[s * T_pad + t].  KS >= k + S (a power of two): the
+// token's rows are gathered U = max(1, 8 / KS) vectors per lane at a time, all loads in flight
+// before the sums.
+template <typename T, int KS>
 __global__ void __launch_bounds__(256)
 combine_fwd_kernel(const T* __restrict__ O, const int32_t* __restrict__ slot,
                    const float* __restrict__ topk_w, int T_, int d, int k, int S, int64_t T_pad,
                    T* __restrict__ y) {
+  pdl_prologue();
   constexpr int VN = Vec16<T>::N;
+  constexpr int U = KS >= 8 ? 1 : 8 / KS;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T_) return;
+  // row list: k routed slots (weight topk_w, -1 if dropped) then S shared rows (weight 1)
   int my_s = -1;
   float my_w = 0.f;
   if (lane < k) {
     my_s = slot[(int64_t)t * k + lane];
     my_w = topk_w[(int64_t)t * k + lane];
+  } else if (lane < k + S) {
+    my_s = (int)((int64_t)(lane - k) * T_pad + t);
+    my_w = 1.f;
   }
-  int s[8];
-  float w[8];
+  int s[KS];
+  float w[KS];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < KS; ++j) {
     s[j] = __shfl_sync(0xffffffffu, my_s, j);
     w[j] = __shfl_sync(0xffffffffu, my_w, j);
+    if (j >= k + S) s[j] = -1;
   }
   const int nv = d / VN;
-  for (int v = lane; v < nv; v += 32) {
-    float acc[VN];
+  for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+    Vec16<T> o[U][KS];
 #pragma unroll
-    for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+    for (int u = 0; u < U; ++u)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k && s[j] >= 0) {
-        const Vec16<T> o = ld_vec_stream(O + (int64_t)s[j] * d + (int64_t)v * VN);
-#pragma unroll
-        for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[j], o.get(i), acc[i]);
+      for (int j = 0; j < KS; ++j) {
+        const int v = v0 + 32 * u;
+        if (v < nv && s[j] >= 0) o[u][j] = ld_vec_stream(O + (int64_t)s[j] * d + (int64_t)v * VN);
       }
-    }
-    for (int sh = 0; sh < S; ++sh) {
-      const Vec16<T> o = ld_vec_stream(O + ((int64_t)sh * T_pad + t) * d + (int64_t)v * VN);
 #pragma unroll
-      for (int i = 0; i < VN; ++i) acc[i] += o.get(i);
-    }
-    Vec16<T> out;
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v >= nv) break;
+      float acc[VN];
 #pragma unroll
-    for (int i = 0; i < VN; ++i) out.set(i, acc[i]);
-    st_vec(y + (int64_t)t * d + (int64_t)v * VN, out);
+      for (int i = 0; i < VN; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < KS; ++j)
+        if (s[j] >= 0) {
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[i] = fmaf(w[j], o[u][j].get(i), acc[i]);
+        }
+      Vec16<T> out;
+#pragma unroll
+      for (int i = 0; i < VN; ++i) out.set(i, acc[i]);
+      st_vec(y + (int64_t)t * d + (int64_t)v * VN, out);
+    }
   }
 }
 
@@ -126,7 +142,7 @@ __device__ __forceinline__ void dlogits_row(const float* __restrict__ lrow, cons
   }
 }
 
-template <typename T>
+template <typename T, int KS>
 __global__ void __launch_bounds__(256)
 combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                    const int32_t* __restrict__ slot, const float* __restrict__ topk_w,
@@ -134,7 +150,9 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                    const int32_t* __restrict__ kept, const int32_t* __restrict__ offsets, int T_,
                    int d, int E, int k, int gate_norm, int n_tok_blocks, float* __restrict__ dg,
                    float* __restrict__ dlogits, T* __restrict__ dO) {
+  pdl_prologue();
   constexpr int VN = Vec16<T>::N;
+  constexpr int U = KS >= 8 ? 1 : 8 / KS;
   const int lane = threadIdx.x & 31;
   const int nv = d / VN;
   if ((int)blockIdx.x >= n_tok_blocks) {  // zero the padding rows of expert e in dO
@@ -162,21 +180,36 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
     s[j] = __shfl_sync(0xffffffffu, my_s, j);
     w[j] = __shfl_sync(0xffffffffu, my_w, j);
     ej[j] = __shfl_sync(0xffffffffu, my_e, j);
+    if (j >= k) s[j] = -1;
     part[j] = 0.f;
   }
-  for (int v = lane; v < nv; v += 32) {
-    const Vec16<T> g = ld_vec_stream(dy + (int64_t)t * d + (int64_t)v * VN);
+  for (int v0 = lane; v0 < nv; v0 += 32 * U) {
+    Vec16<T> g[U], o[U][KS];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k && s[j] >= 0) {
-        const Vec16<T> o = ld_vec_stream(O + (int64_t)s[j] * d + (int64_t)v * VN);
-        Vec16<T> out;
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v < nv) {
+        g[u] = ld_vec_stream(dy + (int64_t)t * d + (int64_t)v * VN);
 #pragma unroll
-        for (int i = 0; i < VN; ++i) {
-          part[j] = fmaf(g.get(i), o.get(i), part[j]);
-          out.set(i, w[j] * g.get(i));
+        for (int j = 0; j < KS; ++j)
+          if (s[j] >= 0) o[u][j] = ld_vec_stream(O + (int64_t)s[j] * d + (int64_t)v * VN);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int v = v0 + 32 * u;
+      if (v >= nv) break;
+#pragma unroll
+      for (int j = 0; j < KS; ++j) {
+        if (s[j] >= 0) {
+          Vec16<T> out;
+#pragma unroll
+          for (int i = 0; i < VN; ++i) {
+            part[j] = fmaf(g[u].get(i), o[u][j].get(i), part[j]);
+            out.set(i, w[j] * g[u].get(i));
+          }
+          st_vec(dO + (int64_t)s[j] * d + (int64_t)v * VN, out);
         }
-        st_vec(dO + (int64_t)s[j] * d + (int64_t)v * VN, out);
       }
     }
   }
@@ -194,35 +227,74 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
 
 }  // namespace
 
+// smallest power of two >= n (n <= 16)
+static inline int pow2_at_least(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+template <typename T, int KS>
+static moe_status combine_t(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
+                            void* y, cudaStream_t st) {
+  return launch_k(combine_fwd_kernel<T, KS>, (D.T + 7) / 8, 256, 0, st, 1, (const T*)O, slot,
+                  topk_w, D.T, D.d, D.k, D.S, D.T_pad, (T*)y);
+}
+template <typename T>
+static moe_status combine_ks(const Dims& D, const void* O, const int32_t* slot,
+                             const float* topk_w, void* y, cudaStream_t st) {
+  switch (pow2_at_least(D.k + D.S)) {
+    case 1: case 2: return combine_t<T, 2>(D, O, slot, topk_w, y, st);
+    case 4: return combine_t<T, 4>(D, O, slot, topk_w, y, st);
+    case 8: return combine_t<T, 8>(D, O, slot, topk_w, y, st);
+    default: return combine_t<T, 16>(D, O, slot, topk_w, y, st);
+  }
+}
+
 moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
                           void* y, cudaStream_t st) {
-  const int grid = (D.T + 7) / 8;
-  if (D.dtype == MOE_DTYPE_BF16)
-    combine_fwd_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)O, slot, topk_w, D.T, D.d, D.k, D.S, D.T_pad, (__nv_bfloat16*)y);
-  else
-    combine_fwd_kernel<float><<<grid, 256, 0, st>>>((const float*)O, slot, topk_w, D.T, D.d, D.k,
-                                                    D.S, D.T_pad, (float*)y);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  if (D.dtype == MOE_DTYPE_BF16) return combine_ks<__nv_bfloat16>(D, O, slot, topk_w, y, st);
+  return combine_ks<float>(D, O, slot, topk_w, y, st);
+}
+
+template <typename T, int KS>
+static moe_status combine_bwd_t(const Dims& D, const void* dy, const void* O, const int32_t* slot,
+                                const float* topk_w, const int32_t* topk_idx,
+                                const float* logits, const int32_t* kept, const int32_t* offsets,
+                                float* dg, float* dlogits, void* dO, cudaStream_t st) {
+  const int n_tok_blocks = (D.T + 7) / 8;
+  return launch_k(combine_bwd_kernel<T, KS>, n_tok_blocks + D.E, 256, 0, st, 1, (const T*)dy,
+                  (const T*)O, slot, topk_w, topk_idx, logits, kept, offsets, D.T, D.d, D.E, D.k,
+                  D.gate_norm, n_tok_blocks, dg, dlogits, (T*)dO);
+}
+template <typename T>
+static moe_status combine_bwd_ks(const Dims& D, const void* dy, const void* O, const int32_t* slot,
+                                 const float* topk_w, const int32_t* topk_idx,
+                                 const float* logits, const int32_t* kept,
+                                 const int32_t* offsets, float* dg, float* dlogits, void* dO,
+                                 cudaStream_t st) {
+  switch (pow2_at_least(D.k)) {
+    case 1: case 2:
+      return combine_bwd_t<T, 2>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
+                                 dlogits, dO, st);
+    case 4:
+      return combine_bwd_t<T, 4>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
+                                 dlogits, dO, st);
+    default:
+      return combine_bwd_t<T, 8>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
+                                 dlogits, dO, st);
+  }
 }
 
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
                               const int32_t* kept, const int32_t* offsets, float* dg,
                               float* dlogits, void* dO, cudaStream_t st) {
-  const int n_tok_blocks = (D.T + 7) / 8;
-  const int grid = n_tok_blocks + D.E;
   if (D.dtype == MOE_DTYPE_BF16)
-    combine_bwd_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)dy, (const __nv_bfloat16*)O, slot, topk_w, topk_idx, logits, kept,
-        offsets, D.T, D.d, D.E, D.k, D.gate_norm, n_tok_blocks, dg, dlogits, (__nv_bfloat16*)dO);
-  else
-    combine_bwd_kernel<float><<<grid, 256, 0, st>>>(
-        (const float*)dy, (const float*)O, slot, topk_w, topk_idx, logits, kept, offsets, D.T,
-        D.d, D.E, D.k, D.gate_norm, n_tok_blocks, dg, dlogits, (float*)dO);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+    return combine_bwd_ks<__nv_bfloat16>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
+                                         dg, dlogits, dO, st);
+  return combine_bwd_ks<float>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
+                               dlogits, dO, st);
 }
 
 }  // namespace moe

@@ -105,6 +105,15 @@ __device__ __forceinline__ void st_vec(T* p, const Vec16<T>& v) {
   *reinterpret_cast<uint4*>(p) = v.raw;
 }
 
+// Programmatic dependent launch: every kernel of this library is launched so that it may start
+// while its predecessor on the stream drains.  It first waits until the predecessor grid has
+// completed and its writes are visible (a no-op without the launch attribute), then lets its own
+// successor start launching.  Nothing global is touched before the wait.
+__device__ __forceinline__ void pdl_prologue() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ float gelu_f(float u) {
   return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
 }
@@ -148,6 +157,48 @@ inline moe_status launch_status() {
   if (e == cudaSuccess) return MOE_OK;
   note_cuda_error(e);
   return MOE_ERR_CUDA;
+}
+}  // namespace moe
+
+namespace moe {
+// Whether launches carry the programmatic-dependent-launch attribute (default on; the environment
+// variable MOE_DISABLE_PDL=1 turns it off).
+bool pdl_enabled();
+
+// Launch `kern` on `st` with the programmatic-dependent-launch attribute (and, when cluster_x > 1,
+// a cluster dimension); counts the launch and records a failure like launch_status().
+template <typename... KArgs, typename... Args>
+inline moe_status launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t st, int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  __atomic_fetch_add(&g_kernel_launches, 1ull, __ATOMIC_RELAXED);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    note_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 }  // namespace moe
 

@@ -29,6 +29,7 @@ static_assert(DT == 256, "rank kernel assumes 8 warps of 32 tokens");
 __global__ void __launch_bounds__(256)
 dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
                      int32_t* __restrict__ blk_counts, int32_t* __restrict__ local_rank) {
+  pdl_prologue();
   __shared__ uint32_t mask[8][256];
   __shared__ int32_t wbase[8][256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -82,6 +83,7 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
                         int32_t* __restrict__ offsets_out,
                         int32_t* __restrict__ slot /* in: local rank, out: slot */,
                         int32_t* __restrict__ row_token, T* __restrict__ Xd) {
+  pdl_prologue();
   __shared__ int32_t s_base[256];   // base of this CTA's rank block, per expert
   __shared__ int32_t s_kept[256];
   __shared__ int32_t s_off[257];
@@ -174,22 +176,19 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
 moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
                            int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
                            void* Xd, int32_t* blk_counts, cudaStream_t st) {
-  dispatch_rank_kernel<<<D.n_blk, 256, 0, st>>>(topk_idx, D.T, D.E, D.k, blk_counts, slot);
-  MOE_LAUNCH_CHECK();
+  MOE_TRY_S(launch_k(dispatch_rank_kernel, D.n_blk, 256, 0, st, 1, topk_idx, D.T, D.E, D.k,
+                     blk_counts, slot));
   const int n_tok_blocks = (D.T + SC_TOK - 1) / SC_TOK;
   const int grid = n_tok_blocks + D.E + 1;
   if (D.dtype == MOE_DTYPE_BF16)
-    dispatch_scatter_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        (const __nv_bfloat16*)x, topk_idx, blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
-        (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets, slot,
-        row_token, (__nv_bfloat16*)Xd);
-  else
-    dispatch_scatter_kernel<float><<<grid, 256, 0, st>>>(
-        (const float*)x, topk_idx, blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
-        (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets, slot,
-        row_token, (float*)Xd);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+    return launch_k(dispatch_scatter_kernel<__nv_bfloat16>, grid, 256, 0, st, 1,
+                    (const __nv_bfloat16*)x, topk_idx, (const int32_t*)blk_counts, D.n_blk, D.T,
+                    D.d, D.E, D.k, D.C, (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0,
+                    counts, kept, offsets, slot, row_token, (__nv_bfloat16*)Xd);
+  return launch_k(dispatch_scatter_kernel<float>, grid, 256, 0, st, 1, (const float*)x, topk_idx,
+                  (const int32_t*)blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
+                  (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets,
+                  slot, row_token, (float*)Xd);
 }
 
 // ----------------------------------------------------------------------------- no-allocation form

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(256)
 up_kernel(const T* __restrict__ Xd, const T* __restrict__ x, const int32_t* __restrict__ offsets,
           const T* __restrict__ W1, const T* __restrict__ W3, int T_, int d, int F, int E,
           int64_t T_pad, int act, T* __restrict__ U, T* __restrict__ V, T* __restrict__ H) {
+  pdl_prologue();
   __shared__ float As[BK][BM + 4], Bs[BK][BN + 4];
   const Group G = group_of(blockIdx.z, E, offsets, T_pad);
   const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
@@ -135,6 +136,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 down_kernel(const T* __restrict__ H, const int32_t* __restrict__ offsets,
             const T* __restrict__ W2, int d, int F, int E, int64_t T_pad, T* __restrict__ O) {
+  pdl_prologue();
   __shared__ float As[BK][BM + 4], Bs[BK][BN + 4];
   const Group G = group_of(blockIdx.z, E, offsets, T_pad);
   const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
@@ -163,6 +165,7 @@ dgrad_h_kernel(const T* __restrict__ dO, const T* __restrict__ dy,
                const int32_t* __restrict__ offsets, const T* __restrict__ W2,
                const T* __restrict__ U, const T* __restrict__ V, int T_, int d, int F, int E,
                int64_t T_pad, int act, T* __restrict__ dU, T* __restrict__ dV) {
+  pdl_prologue();
   __shared__ float As[BK][BM + 4], Bs[BK][BN + 4];
   const Group G = group_of(blockIdx.z, E, offsets, T_pad);
   const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
@@ -195,6 +198,7 @@ dgrad_x_kernel(const T* __restrict__ dU, const T* __restrict__ dV,
                const int32_t* __restrict__ offsets, const T* __restrict__ W1,
                const T* __restrict__ W3, int d, int F, int E, int64_t T_pad, int act,
                T* __restrict__ dXd) {
+  pdl_prologue();
   __shared__ float As[BK][BM + 4], Bs[BK][BN + 4];
   const Group G = group_of(blockIdx.z, E, offsets, T_pad);
   const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
@@ -227,6 +231,7 @@ __global__ void __launch_bounds__(256)
 wgrad_kernel(int which, const T* __restrict__ Gf /* dU, dV or H */, const T* __restrict__ Xd_or_dO,
              const T* __restrict__ tok /* x or dy */, const int32_t* __restrict__ offsets, int T_,
              int d, int F, int E, int64_t T_pad, float* __restrict__ dW) {
+  pdl_prologue();
   __shared__ float As[BK][BM + 4], Bs[BK][BN + 4];
   const Group G = group_of(blockIdx.z, E, offsets, T_pad);
   const int64_t m0 = (int64_t)blockIdx.x * BM, n0 = (int64_t)blockIdx.y * BN;
@@ -258,23 +263,24 @@ wgrad_kernel(int which, const T* __restrict__ Gf /* dU, dV or H */, const T* __r
 #define MOE_SIMT_DISPATCH(D, CALL)                                   \
   ((D).dtype == MOE_DTYPE_BF16 ? [&] { using T = __nv_bfloat16; return CALL; }() \
                                : [&] { using T = float; return CALL; }())
+#define SIMT_LAUNCH(KERN, GRID, ...) launch_k(KERN, GRID, 256, 0, st, 1, __VA_ARGS__)
 
 moe_status launch_expert_up_simt(const Dims& D, const void* Xd, const void* x,
                                  const int32_t* offsets, const void* W1, const void* W3, void* U,
                                  void* V, void* H, cudaStream_t st) {
   const int mt = (int)((D.max_group_rows + BM - 1) / BM);
   const dim3 grid(mt, (D.F + BN - 1) / BN, D.E_tot);
-  return MOE_SIMT_DISPATCH(D, (up_kernel<T><<<grid, 256, 0, st>>>(
+  return MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(up_kernel<T>, grid,
       (const T*)Xd, (const T*)x, offsets, (const T*)W1, (const T*)W3, D.T, D.d, D.F, D.E,
-      D.T_pad, D.act, (T*)U, (T*)V, (T*)H), launch_status()));
+      D.T_pad, D.act, (T*)U, (T*)V, (T*)H));
 }
 
 moe_status launch_expert_down_simt(const Dims& D, const void* H, const int32_t* offsets,
                                    const void* W2, void* O, cudaStream_t st) {
   const int mt = (int)((D.max_group_rows + BM - 1) / BM);
   const dim3 grid(mt, (D.d + BN - 1) / BN, D.E_tot);
-  return MOE_SIMT_DISPATCH(D, (down_kernel<T><<<grid, 256, 0, st>>>(
-      (const T*)H, offsets, (const T*)W2, D.d, D.F, D.E, D.T_pad, (T*)O), launch_status()));
+  return MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(down_kernel<T>, grid,
+      (const T*)H, offsets, (const T*)W2, D.d, D.F, D.E, D.T_pad, (T*)O));
 }
 
 moe_status launch_dgrad_h_simt(const Dims& D, const void* dO, const void* dy,
@@ -282,9 +288,9 @@ moe_status launch_dgrad_h_simt(const Dims& D, const void* dO, const void* dy,
                                const void* V, void* dU, void* dV, cudaStream_t st) {
   const int mt = (int)((D.max_group_rows + BM - 1) / BM);
   const dim3 grid(mt, (D.F + BN - 1) / BN, D.E_tot);
-  return MOE_SIMT_DISPATCH(D, (dgrad_h_kernel<T><<<grid, 256, 0, st>>>(
+  return MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(dgrad_h_kernel<T>, grid,
       (const T*)dO, (const T*)dy, offsets, (const T*)W2, (const T*)U, (const T*)V, D.T, D.d, D.F,
-      D.E, D.T_pad, D.act, (T*)dU, (T*)dV), launch_status()));
+      D.E, D.T_pad, D.act, (T*)dU, (T*)dV));
 }
 
 moe_status launch_dgrad_x_simt(const Dims& D, const void* dU, const void* dV,
@@ -292,31 +298,28 @@ moe_status launch_dgrad_x_simt(const Dims& D, const void* dU, const void* dV,
                                cudaStream_t st) {
   const int mt = (int)((D.max_group_rows + BM - 1) / BM);
   const dim3 grid(mt, (D.d + BN - 1) / BN, D.E_tot);
-  return MOE_SIMT_DISPATCH(D, (dgrad_x_kernel<T><<<grid, 256, 0, st>>>(
+  return MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(dgrad_x_kernel<T>, grid,
       (const T*)dU, (const T*)dV, offsets, (const T*)W1, (const T*)W3, D.d, D.F, D.E, D.T_pad,
-      D.act, (T*)dXd), launch_status()));
+      D.act, (T*)dXd));
 }
 
 moe_status launch_wgrad_w13_simt(const Dims& D, const void* dU, const void* dV, const void* Xd,
                                  const void* x, const int32_t* offsets, float* dW1, float* dW3,
                                  cudaStream_t st) {
   const dim3 g1((D.F + BM - 1) / BM, (D.d + BN - 1) / BN, D.E_tot);
-  MOE_TRY_S(MOE_SIMT_DISPATCH(D, (wgrad_kernel<T><<<g1, 256, 0, st>>>(
-      0, (const T*)dU, (const T*)Xd, (const T*)x, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW1),
-      launch_status())));
+  MOE_TRY_S(MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(wgrad_kernel<T>, g1,
+      0, (const T*)dU, (const T*)Xd, (const T*)x, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW1)));
   if (D.act == MOE_ACT_SWIGLU)
-    MOE_TRY_S(MOE_SIMT_DISPATCH(D, (wgrad_kernel<T><<<g1, 256, 0, st>>>(
-        1, (const T*)dV, (const T*)Xd, (const T*)x, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW3),
-        launch_status())));
+    MOE_TRY_S(MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(wgrad_kernel<T>, g1,
+        1, (const T*)dV, (const T*)Xd, (const T*)x, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW3)));
   return MOE_OK;
 }
 
 moe_status launch_wgrad_w2_simt(const Dims& D, const void* H, const void* dO, const void* dy,
                                 const int32_t* offsets, float* dW2, cudaStream_t st) {
   const dim3 g2((D.d + BM - 1) / BM, (D.F + BN - 1) / BN, D.E_tot);
-  return MOE_SIMT_DISPATCH(D, (wgrad_kernel<T><<<g2, 256, 0, st>>>(
-      2, (const T*)H, (const T*)dO, (const T*)dy, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW2),
-      launch_status()));
+  return MOE_SIMT_DISPATCH(D, SIMT_LAUNCH(wgrad_kernel<T>, g2,
+      2, (const T*)H, (const T*)dO, (const T*)dy, offsets, D.T, D.d, D.F, D.E, D.T_pad, dW2));
 }
 
 }  // namespace moe

@@ -537,6 +537,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
 template <int KIND>
 __global__ void __launch_bounds__(Cfg<KIND>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ Params P) {
+  pdl_prologue();
   constexpr int STAGES = Cfg<KIND>::STAGES;
   constexpr int NUM_THREADS = Cfg<KIND>::THREADS;
   constexpr int NUM_EPI_WARPS = Cfg<KIND>::EPI_WARPS;
@@ -730,25 +731,8 @@ static moe_status launch(const Params& P, int max_tiles, cudaStream_t st) {
   }
   const int max_pairs = num_sms() / 2;
   const int pairs = max_tiles < max_pairs ? (max_tiles > 0 ? max_tiles : 1) : max_pairs;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(Cfg<KIND>::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = Cfg<KIND>::SMEM_BYTES;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<KIND>, P);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    note_cuda_error(e);
-    return MOE_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_k(grouped_gemm_kernel<KIND>, dim3(2 * pairs, 1, 1), dim3(Cfg<KIND>::THREADS, 1, 1),
+                  Cfg<KIND>::SMEM_BYTES, st, 2, P);
 }
 
 static Params base_params(const Dims& D, const int32_t* offsets, uint32_t* status) {

@@ -25,6 +25,7 @@ router_fwd_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
                   const float* __restrict__ bias, int T_, int d, int E, int k, int gate_norm,
                   float* __restrict__ logits, int32_t* __restrict__ topk_idx,
                   float* __restrict__ topk_w) {
+  pdl_prologue();
   extern __shared__ float smem[];
   float* xs = smem;                                // [RT_BK][RT_TOK + 4] (k-major)
   float* ws = xs + RT_BK * (RT_TOK + 4);           // [RT_BK][RT_EC + 4]
@@ -86,6 +87,7 @@ router_fwd_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
 __global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T_, int E, int k,
                                         int gate_norm, int32_t* __restrict__ topk_idx,
                                         float* __restrict__ topk_w) {
+  pdl_prologue();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T_) return;
   const float* row = logits + (int64_t)t * E;
@@ -109,29 +111,25 @@ moe_status launch_router(const Dims& D, const void* x, const void* Wg, const flo
     auto kern = router_fwd_kernel<__nv_bfloat16>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
       return MOE_ERR_CUDA;
-    kern<<<grid, RT_THREADS, sm, st>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)Wg,
-                                       D.has_bias ? bias : nullptr, D.T, D.d, D.E, D.k,
-                                       D.gate_norm, logits, topk_idx, topk_w);
+    return launch_k(kern, grid, RT_THREADS, sm, st, 1, (const __nv_bfloat16*)x,
+                    (const __nv_bfloat16*)Wg, D.has_bias ? bias : nullptr, D.T, D.d, D.E, D.k,
+                    D.gate_norm, logits, topk_idx, topk_w);
   } else {
     auto kern = router_fwd_kernel<float>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
       return MOE_ERR_CUDA;
-    kern<<<grid, RT_THREADS, sm, st>>>((const float*)x, (const float*)Wg,
-                                       D.has_bias ? bias : nullptr, D.T, D.d, D.E, D.k,
-                                       D.gate_norm, logits, topk_idx, topk_w);
+    return launch_k(kern, grid, RT_THREADS, sm, st, 1, (const float*)x, (const float*)Wg,
+                    D.has_bias ? bias : nullptr, D.T, D.d, D.E, D.k, D.gate_norm, logits,
+                    topk_idx, topk_w);
   }
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
 }
 
 moe_status launch_topk_from_logits(const Dims& D, const float* logits, int32_t* topk_idx,
                                    float* topk_w, cudaStream_t st) {
   const int threads = 128;
   const int grid = (D.T + threads - 1) / threads;
-  topk_from_logits_kernel<<<grid, threads, 0, st>>>(logits, D.T, D.E, D.k, D.gate_norm, topk_idx,
-                                                    topk_w);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  return launch_k(topk_from_logits_kernel, grid, threads, 0, st, 1, logits, D.T, D.E, D.k,
+                  D.gate_norm, topk_idx, topk_w);
 }
 
 }  // namespace moe

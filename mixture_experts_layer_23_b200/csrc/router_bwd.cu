@@ -24,6 +24,7 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 router_wgrad_partial_kernel(const float* __restrict__ dl, const T* __restrict__ x, int T_, int d,
                             int E, int chunk, float* __restrict__ part) {
+  pdl_prologue();
   constexpr int VN = Vec16<T>::N;
   constexpr int WG_TS = 128 / (int)sizeof(T);  // 64 bf16 or 32 fp32 token rows: a 32 KB tile
   __shared__ __align__(16) T xs[WG_TS][WG_COLS];
@@ -79,6 +80,7 @@ router_wgrad_partial_kernel(const float* __restrict__ dl, const T* __restrict__ 
 
 __global__ void router_wgrad_reduce_kernel(const float* __restrict__ part, int n_chunk,
                                            int64_t n, float* __restrict__ dWg) {
+  pdl_prologue();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float s = 0.f;
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(256)
 undispatch_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
                   const T* __restrict__ dXd, const int32_t* __restrict__ slot, int T_, int d,
                   int E, int k, int S, int64_t T_pad, T* __restrict__ dx) {
+  pdl_prologue();
   constexpr int VN = Vec16<T>::N;
   constexpr int COLS = 32 * VN;
   extern __shared__ uint4 ud_smem[];
@@ -196,16 +199,14 @@ moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* 
   const int chunk = (D.T + D.n_tchunk - 1) / D.n_tchunk;
   dim3 grid(D.n_tchunk, (D.d + WG_COLS - 1) / WG_COLS);
   if (D.dtype == MOE_DTYPE_BF16)
-    router_wgrad_partial_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(
-        dlogits, (const __nv_bfloat16*)x, D.T, D.d, D.E, chunk, part);
+    MOE_TRY_S(launch_k(router_wgrad_partial_kernel<__nv_bfloat16>, grid, 128, 0, st, 1, dlogits,
+                       (const __nv_bfloat16*)x, D.T, D.d, D.E, chunk, part));
   else
-    router_wgrad_partial_kernel<float><<<grid, 128, 0, st>>>(dlogits, (const float*)x, D.T, D.d,
-                                                             D.E, chunk, part);
-  MOE_LAUNCH_CHECK();
+    MOE_TRY_S(launch_k(router_wgrad_partial_kernel<float>, grid, 128, 0, st, 1, dlogits,
+                       (const float*)x, D.T, D.d, D.E, chunk, part));
   const int64_t n = (int64_t)D.E * D.d;
-  router_wgrad_reduce_kernel<<<(int)((n + 255) / 256), 256, 0, st>>>(part, D.n_tchunk, n, dWg);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  return launch_k(router_wgrad_reduce_kernel, (int)((n + 255) / 256), 256, 0, st, 1,
+                  (const float*)part, D.n_tchunk, n, dWg);
 }
 
 template <typename T>
@@ -219,10 +220,8 @@ static moe_status undispatch_t(const Dims& D, const float* dlogits, const void* 
           cudaSuccess)
     return MOE_ERR_CUDA;
   dim3 grid((D.T + 31) / 32, (D.d + COLS - 1) / COLS);
-  kern<<<grid, 256, smem, st>>>(dlogits, (const T*)Wg, (const T*)dXd, slot, D.T, D.d, D.E, D.k,
-                                D.S, D.T_pad, (T*)dx);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
+  return launch_k(kern, grid, 256, smem, st, 1, dlogits, (const T*)Wg, (const T*)dXd, slot, D.T,
+                  D.d, D.E, D.k, D.S, D.T_pad, (T*)dx);
 }
 
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,

@@ -40,6 +40,7 @@ struct alignas(64) RouterParams {
 };
 
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
+  pdl_prologue();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -189,8 +190,7 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  router_tc_kernel<<<(D.T + 127) / 128, 192, smem, st>>>(P);
-  return launch_status();
+  return launch_k(router_tc_kernel, (D.T + 127) / 128, 192, smem, st, 1, P);
 }
 
 }  // namespace moe

@@ -220,8 +220,8 @@ def kernel_launches() -> int:
 
 def set_profile_events(fwd_events=None, bwd_events=None):
     """Install (or clear, with None) per-phase CUDA events for moe_layer_fwd / moe_layer_bwd.
-    Each is a list of torch.cuda.Event (timing enabled), len(phases) + 1 long; the arrays are
-    kept alive on this module until cleared."""
+    Each is a list of torch.cuda.Event (timing enabled) or None (boundary not recorded),
+    len(phases) + 1 long; the arrays are kept alive on this module until cleared."""
     global _prof_keep
 
     def arr(evs, n):
@@ -229,9 +229,9 @@ def set_profile_events(fwd_events=None, bwd_events=None):
             return None
         assert len(evs) == n + 1
         for e in evs:
-            if not e.cuda_event:      # torch creates the CUDA event on its first record
+            if e is not None and not e.cuda_event:  # torch creates the event on first record
                 e.record()
-        return (ctypes.c_void_p * (n + 1))(*[e.cuda_event for e in evs])
+        return (ctypes.c_void_p * (n + 1))(*[None if e is None else e.cuda_event for e in evs])
     a, b = arr(fwd_events, len(FWD_PHASES)), arr(bwd_events, len(BWD_PHASES))
     _prof_keep = (a, b, fwd_events, bwd_events)
     _check(_lib.moe_set_profile_events(a, b), "moe_set_profile_events")
