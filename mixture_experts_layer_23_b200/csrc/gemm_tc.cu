@@ -58,33 +58,38 @@ constexpr int MAX_GROUPS = 264;
 // in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
 constexpr int NSLOT = 2;
 constexpr uint32_t SLOT_BYTES = 32 * 128;
-constexpr size_t MISC_BYTES = 1280;   // barriers, TMEM slot, abort flag, tile prefix
+constexpr size_t MISC_BYTES = 1536;   // barriers, TMEM slot, abort flag, tile prefix
 
 enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
 
 // Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
 // up-projection's activation epilogue is the heaviest per output, so it gets 8 epilogue warps (two
 // per TMEM lane quarter, each taking half the columns) and 5 stages; the others keep 4 epilogue
-// warps and 6 stages of loads in flight.  10 warps cap each thread at 168 registers (each SM
-// sub-partition's register file holds 3 of the 10 warps).
+// warps and 6 stages of loads in flight, except the activation-gradient GEMM, whose epilogue
+// reads the saved factors Gu (Gv) through TMA into NIN input slots per warp and keeps 4 stages to
+// make room.  10 warps cap each thread at 168 registers (each SM sub-partition's register file
+// holds 3 of the 10 warps).
 template <int KIND>
 struct Cfg {
   static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
   static constexpr int SPLIT = EPI_WARPS / 4;
-  static constexpr int STAGES = (KIND == UP) ? 5 : 6;
+  static constexpr int STAGES = (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4 : 6;
+  static constexpr int NIN = (KIND == DGRAD_H) ? 4 : 0;   // epilogue input slots per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr uint32_t RING_BYTES = EPI_WARPS * NSLOT * SLOT_BYTES;
-  static constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RING_BYTES + MISC_BYTES;
+  static constexpr uint32_t IN_BYTES = EPI_WARPS * NIN * SLOT_BYTES;
+  static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN;
+  static constexpr size_t SMEM_BYTES =
+      1024 + STAGES * STAGE_BYTES + RING_BYTES + IN_BYTES + MISC_BYTES;
   static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
-  static_assert(8 * (2 * STAGES + 5) + 16 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc too small");
+  static_assert(8 * NBARS + 16 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc too small");
 };
 
 struct alignas(64) Params {
   CUtensorMap a_main, a_alt, b_main, b_alt;
   CUtensorMap o0, o1, o2;  // output tensor maps (TMA stores), see the epilogue of each kind
+  CUtensorMap i0, i1;      // DGRAD_H epilogue inputs Gu, Gv (TMA loads, 64 x 32 boxes)
   const int32_t* offsets;
-  const void* aux0;      // U (DGRAD_H epilogue)
-  const void* aux1;      // V (DGRAD_H epilogue, SwiGLU)
   uint32_t* status;
   unsigned long long timeout_ns;
   long long T_pad;
@@ -275,6 +280,50 @@ __device__ __forceinline__ void ring_store_3d(Ring& r, const CUtensorMap* map, u
   }
 }
 
+// Epilogue input slots (DGRAD_H): 32 x 64 bf16 boxes of Gu / Gv loaded by TMA in the same
+// swizzled layout the output slots use, one mbarrier per slot.  Loads are consumed in issue order,
+// so load j uses slot j % NIN with parity (j / NIN) & 1; a slot is refilled only after the chunk
+// that read it has been computed.
+struct InRing {
+  uint8_t* base;
+  uint64_t* bars;
+  int issued, consumed;
+};
+template <int NIN>
+__device__ __forceinline__ void in_issue(InRing& r, const CUtensorMap* map, int c0, int c1,
+                                         int lane) {
+  const int s = r.issued % NIN;
+  if (lane == 0) {
+    fence_async_smem();   // earlier generic reads of this slot before the async-proxy write
+    mbar_expect_tx(&r.bars[s], SLOT_BYTES);
+    tma_load_2d(r.base + s * SLOT_BYTES, map, &r.bars[s], c0, c1);
+  }
+  ++r.issued;
+}
+template <int NIN>
+__device__ __forceinline__ const uint8_t* in_wait(InRing& r, volatile int* abort_flag,
+                                                  unsigned long long budget) {
+  const int j = r.consumed;
+  if (!wait_bounded(&r.bars[j % NIN], (uint32_t)(j / NIN) & 1u, abort_flag, budget))
+    return nullptr;   // still counted as in flight: the exit path waits for it
+  ++r.consumed;
+  return r.base + (j % NIN) * SLOT_BYTES;
+}
+// 32 columns (half h) of row r of an input slot -> fp32
+__device__ __forceinline__ void slot_get_bf16_half(const uint8_t* slot, int r, int h, float* v) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const int cc = 4 * h + c;
+    const uint4 w = *reinterpret_cast<const uint4*>(slot + r * 128 + ((cc ^ (r & 7)) << 4));
+    const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[8 * c + 2 * i] = __uint_as_float(q[i] << 16);
+      v[8 * c + 2 * i + 1] = __uint_as_float(q[i] & 0xFFFF0000u);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -333,7 +382,7 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
 template <int KIND>
 __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
                                               int q, int half, int lane, Ring& ring,
-                                              uint64_t* tfull, uint32_t parity,
+                                              InRing& inr, uint64_t* tfull, uint32_t parity,
                                               volatile int* abort_flag) {
   constexpr int SPLIT = Cfg<KIND>::SPLIT;
   const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
@@ -366,70 +415,60 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     return true;
   }
   const int row0 = t.o_row + t.mrow + q * 32;  // first output row of this warp's slab
-  if (KIND == DGRAD_H) {
-    // 32-column steps; U (and V) of the next step are loaded while this step computes, and the
-    // first step's are in flight before the wait for the accumulator.
+  if constexpr (KIND == DGRAD_H) {
+    // 64-column chunks; each chunk's Gu (and Gv) box is loaded by TMA into an input slot, the
+    // first chunks' loads issued before the wait for the accumulator.
+    constexpr int NIN = Cfg<KIND>::NIN;
     const int F = P.N;
-    const size_t rowoff = (size_t)(row0 + lane) * F;
-    const uint4* U = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux0) + rowoff);
-    const uint4* V = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.aux1) + rowoff);
-    uint4 pu[4], pv[4];
-    int n = t.n * BN + half * (BN / SPLIT);
-    if (t.live) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) pu[i] = U[n / 8 + i];
-      if (swiglu) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) pv[i] = V[n / 8 + i];
-      }
-    }
+    const int per = swiglu ? 2 : 1;              // input slots per chunk
+    const int depth = NIN / per;                 // chunks in flight
+    const int ch0 = half * (BN / 64 / SPLIT), ch1 = (half + 1) * (BN / 64 / SPLIT);
+    int nch = 0;                                 // chunks of this warp inside [0, F)
+    for (int ch = ch0; ch < ch1 && t.n * BN + ch * 64 < F; ++ch) ++nch;
+    if (!t.live) nch = 0;
+    auto issue_chunk = [&](int i) {
+      const int n = t.n * BN + (ch0 + i) * 64;
+      in_issue<NIN>(inr, &P.i0, n, row0, lane);
+      if (swiglu) in_issue<NIN>(inr, &P.i1, n, row0, lane);
+    };
+    for (int i = 0; i < nch && i < depth; ++i) issue_chunk(i);
     if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
-    if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
 #pragma unroll 1
-    for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
-      n = t.n * BN + ch * 64;
-      if (n >= F) break;
+    for (int i = 0; i < nch; ++i) {
+      const int n = t.n * BN + (ch0 + i) * 64;
+      const uint8_t* gu = in_wait<NIN>(inr, abort_flag, P.timeout_ns);
+      const uint8_t* gv = swiglu ? in_wait<NIN>(inr, abort_flag, P.timeout_ns) : nullptr;
+      if (gu == nullptr || (swiglu && gv == nullptr)) return false;
       uint8_t* su = ring_take(ring, lane);
       uint8_t* sv = swiglu ? ring_take<1>(ring, lane) : nullptr;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        const int ns = n + 32 * h;
-        float u[32], v[32];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) unpack_bf16x8(pu[i], u + 8 * i);
-        if (swiglu) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) unpack_bf16x8(pv[i], v + 8 * i);
-        }
-        const int nn = ns + 32;
-        if (nn < F && nn < t.n * BN + (half + 1) * (BN / SPLIT)) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) pu[i] = U[nn / 8 + i];
-          if (swiglu) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) pv[i] = V[nn / 8 + i];
-          }
-        }
         uint32_t r[32];
-        tmem_ld32_async(tl + ch * 64 + h * 32, r);
+        tmem_ld32_async(tl + (ch0 + i) * 64 + h * 32, r);
+        float u[32];
+        slot_get_bf16_half(gu, lane, h, u);
         tmem_wait_ld();
         if (!swiglu) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(r[i]) * u[i];   // dH * GELU'(u)
+          for (int j = 0; j < 32; ++j) a[j] = __uint_as_float(r[j]) * u[j];   // dU = dH * Gu
           slot_put_bf16_half(su, lane, h, a);
         } else {
+          float v[32];
+          slot_get_bf16_half(gv, lane, h, v);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float dh = __uint_as_float(r[i]);
-            a[i] = dh * u[i];   // dU = dH * Gu
-            v[i] = dh * v[i];   // dV = dH * Gv
+          for (int j = 0; j < 32; ++j) {
+            const float dh = __uint_as_float(r[j]);
+            a[j] = dh * u[j];   // dU = dH * Gu
+            v[j] = dh * v[j];   // dV = dH * Gv
           }
           slot_put_bf16_half(su, lane, h, a);
           slot_put_bf16_half(sv, lane, h, v);
         }
       }
+      __syncwarp();   // every lane has read this chunk's input slots
+      if (i + depth < nch) issue_chunk(i + depth);
       ring_store_2d(ring, &P.o0, su, n, row0, lane);
       if (swiglu) ring_store_2d(ring, &P.o1, sv, n, row0, lane);
     }
@@ -546,13 +585,16 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* tiles = smem;
   uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // 4 warps x NSLOT slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring_base + RING_BYTES);
+  constexpr int NIN = Cfg<KIND>::NIN;
+  uint8_t* in_base = ring_base + RING_BYTES;                     // epilogue warps x NIN slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(in_base + Cfg<KIND>::IN_BYTES);
   uint64_t* full = bars;                 // [STAGES]  (the leader's are the ones used)
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
   uint64_t* tempty = tfull + 2;          // [2]       (the leader's are the ones used)
   uint64_t* drain = tempty + 2;          // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* in_bars = drain + 1;         // [EPI_WARPS * NIN]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(in_bars + NUM_EPI_WARPS * NIN);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tile_start = reinterpret_cast<int*>(tmem_slot + 4);   // [MAX_GROUPS + 1]
 
@@ -580,6 +622,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       mbar_init(&tempty[i], 2 * NUM_EPI_WARPS);   // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -684,6 +727,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     Ring ring{ring_base + (warp - 2) * NSLOT * SLOT_BYTES, 0};
+    InRing inr{in_base + (warp - 2) * NIN * SLOT_BYTES, in_bars + (warp - 2) * NIN, 0, 0};
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0;
@@ -692,7 +736,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, half, lane,
-                               ring, &tfull[acc], acc_phase, abort_flag))
+                               ring, inr, &tfull[acc], acc_phase, abort_flag))
         break;
       tc_fence_before();
       __syncwarp();
@@ -700,6 +744,12 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
     if (lane == 0) bulk_wait<0>();  // this warp's stores have completed
+    // on abort, let input loads still in flight land before the CTA exits
+    for (int j = inr.consumed; j < inr.issued; ++j) {
+      volatile int never = 0;
+      wait_bounded(&inr.bars[j % (NIN > 0 ? NIN : 1)], (uint32_t)(j / (NIN > 0 ? NIN : 1)) & 1u,
+                   &never, 20000000ull);
+    }
     __syncwarp();
   }
   __syncwarp();
@@ -801,8 +851,8 @@ moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, cons
   if (!(map2(&P.a_main, dO, D.d, D.R, 64, BM) && map2(&P.a_alt, dy, D.d, D.T, 64, BM) &&
         map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, 64)))
     return MOE_ERR_CUDA;
-  P.aux0 = U;
-  P.aux1 = V;
+  if (!map2(&P.i0, U, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
+  if (D.act == MOE_ACT_SWIGLU && !map2(&P.i1, V, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
   if (!map2(&P.o0, dU, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
   if (D.act == MOE_ACT_SWIGLU && !map2(&P.o1, dV, D.F, D.R, 64, 32)) return MOE_ERR_CUDA;
   P.N = D.F;

@@ -229,8 +229,6 @@ moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg
   if (D.dtype == MOE_DTYPE_BF16)
     return undispatch_t<__nv_bfloat16>(D, dlogits, Wg, dXd, slot, dx, st);
   return undispatch_t<float>(D, dlogits, Wg, dXd, slot, dx, st);
-  MOE_LAUNCH_CHECK();
-  return MOE_OK;
 }
 
 }  // namespace moe
