@@ -245,16 +245,25 @@ int32_t moe_gemm_engine(const moe_config_t* cfg) {
   return tc_supported(D) ? 1 : 0;
 }
 
+// Router choice: bf16 with d a multiple of 64 takes the tcgen05 kernel (measured faster than the
+// warp-per-token kernel from 16 experts up); other shapes with up to 32 experts whose gate matrix
+// fits in shared memory take the warp-per-token kernel; the rest the CUDA-core tile kernel.  All
+// three end in the same serial softmax + top-k.
+static moe_status launch_route(const Dims& D, const void* x, const void* Wg, const float* bias,
+                               float* logits, int32_t* idx, float* w, uint32_t* status,
+                               cudaStream_t st) {
+  if (router_tc_supported(D)) return launch_router_tc(D, x, Wg, bias, logits, idx, w, status, st);
+  if (router_warp_supported(D)) return launch_router_warp(D, x, Wg, bias, logits, idx, w, st);
+  return launch_router(D, x, Wg, bias, logits, idx, w, st);
+}
+
 moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, const float* bias,
                      float* logits, int32_t* topk_idx, float* topk_w, moe_stream_t stream) {
   Dims D;
   MOE_TRY(resolve_dims(cfg, &D));
   MOE_TRY(check_ptrs({x, Wg, logits, topk_idx, topk_w}));
   if (D.has_bias) MOE_TRY(check_ptrs({bias}));
-  if (router_tc_supported(D))
-    return launch_router_tc(D, x, Wg, bias, logits, topk_idx, topk_w, nullptr,
-                            (cudaStream_t)stream);
-  return launch_router(D, x, Wg, bias, logits, topk_idx, topk_w, (cudaStream_t)stream);
+  return launch_route(D, x, Wg, bias, logits, topk_idx, topk_w, nullptr, (cudaStream_t)stream);
 }
 
 moe_status moe_route_from_logits(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
@@ -326,10 +335,7 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   void* H = c + L.ctx_H;
   void* O = c + L.ctx_O;
   MOE_TRY(mark_fwd(0, st));
-  if (router_tc_supported(D))
-    MOE_TRY(launch_router_tc(D, x, Wg, bias, logits, idx, w, (uint32_t*)(s + S.status), st));
-  else
-    MOE_TRY(launch_router(D, x, Wg, bias, logits, idx, w, st));
+  MOE_TRY(launch_route(D, x, Wg, bias, logits, idx, w, (uint32_t*)(s + S.status), st));
   MOE_TRY(mark_fwd(1, st));
   MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
                           (int32_t*)(s + S.blk_counts), st));

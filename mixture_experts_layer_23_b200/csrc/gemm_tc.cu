@@ -22,13 +22,14 @@
 //
 // CTA organisation (one CTA per SM, clusters of 2, persistent over tiles; see Cfg for the per-kind
 // numbers of epilogue warps and stages):
-//   warp 0      TMA producer: loads this CTA's A and B halves into a 5- or 6-stage ring;
+//   warp 0      TMA producer: loads this CTA's A and B halves into a 4- to 6-stage ring;
 //               completion is counted on the leader CTA's barrier (cta_group::2 loads)
 //   warp 1      owns 512 TMEM columns (two 128x256 fp32 accumulators, allocated pair-wide); on the
 //               leader, one lane issues the MMAs and commits each stage back to both producers
 //   warps 2..    epilogue: tcgen05.ld the finished accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31 = tile rows; with 8 epilogue warps, warps 2..5 take the first half
-//               of the columns and 6..9 the second), apply the fused activation, store via TMA
+//               32*(w%4)..+31 = tile rows; with 8 epilogue warps, the two warps of a lane
+//               quarter take its 64-column chunks in turn), apply the fused activation, store
+//               via TMA
 // The two accumulators let the epilogue of one tile overlap the main loop of the next.
 // Every mbarrier wait is bounded: on timeout the kernel records MOE_STATUS_TIMEOUT in the status
 // word, drains its own copies and MMAs (with a bound), frees TMEM and returns.
@@ -54,9 +55,8 @@ constexpr uint32_t B_BYTES = BNH * BK * 2;          // 16 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES; // per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
-// Epilogue staging: each epilogue warp owns a ring of NSLOT 4 KB slots (32 rows x 128 B, laid out
+// Epilogue staging: each epilogue warp owns a ring of Cfg::NSLOT 4 KB slots (32 rows x 128 B, laid out
 // in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
-constexpr int NSLOT = 2;
 constexpr uint32_t SLOT_BYTES = 32 * 128;
 constexpr size_t MISC_BYTES = 1536;   // barriers, TMEM slot, abort flag, tile prefix
 
@@ -64,18 +64,21 @@ enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
 
 // Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
 // up-projection's activation epilogue is the heaviest per output, so it gets 8 epilogue warps (two
-// per TMEM lane quarter, each taking half the columns) and 5 stages; the others keep 4 epilogue
-// warps and 6 stages of loads in flight, except the activation-gradient GEMM, whose epilogue
-// reads the saved factors Gu (Gv) through TMA into NIN input slots per warp and keeps 4 stages to
-// make room.  10 warps cap each thread at 168 registers (each SM sub-partition's register file
-// holds 3 of the 10 warps).
+// per TMEM lane quarter, taking the tile's 64-column chunks in turn) and 5 stages (12 warps with
+// 4 stages measured slower); the others keep 4 epilogue warps and 6 stages of loads in flight, except the
+// activation-gradient GEMM, whose epilogue reads the saved factors Gu (Gv) through TMA into NIN
+// input slots per warp and keeps 4 stages to make room.  Warps are spread over the SM's four
+// sub-partitions by warp index and each sub-partition has a quarter of the register file
+// (16384 registers): 10 warps put 3 on one sub-partition, capping threads at 168 registers;
+// 6 warps allow 255.
 template <int KIND>
 struct Cfg {
   static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
-  static constexpr int SPLIT = EPI_WARPS / 4;
+  static constexpr int SPLIT = EPI_WARPS / 4;   // epilogue warps per TMEM lane quarter
   static constexpr int STAGES = (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4 : 6;
   static constexpr int NIN = (KIND == DGRAD_H) ? 4 : 0;   // epilogue input slots per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int NSLOT = 2;                          // output staging slots per warp
   static constexpr uint32_t RING_BYTES = EPI_WARPS * NSLOT * SLOT_BYTES;
   static constexpr uint32_t IN_BYTES = EPI_WARPS * NIN * SLOT_BYTES;
   static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN;
@@ -244,6 +247,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 // writes into the async proxy, and lane 0 hands the 32 x 128 B box to a TMA store.  Stores that
 // fall outside the tensor (a partial last N tile) are clipped by TMA.
 
+template <int NSLOT>
 struct Ring {
   uint8_t* base;
   int next;  // slots taken so far; slot = next % NSLOT.  Stores are issued in take order.
@@ -252,8 +256,8 @@ struct Ring {
 // Take the next slot.  AHEAD = slots taken earlier whose stores are not issued yet.  Take j
 // reuses the slot of take j - NSLOT, whose store must have finished reading shared memory; at
 // this point j - AHEAD stores have been issued, so at most NSLOT - 1 - AHEAD may still be pending.
-template <int AHEAD = 0>
-__device__ __forceinline__ uint8_t* ring_take(Ring& r, int lane) {
+template <int AHEAD = 0, int NSLOT>
+__device__ __forceinline__ uint8_t* ring_take(Ring<NSLOT>& r, int lane) {
   static_assert(AHEAD < NSLOT, "more slots held than the ring has");
   if (r.next >= NSLOT && lane == 0) bulk_wait_read<NSLOT - 1 - AHEAD>();
   __syncwarp();
@@ -261,8 +265,8 @@ __device__ __forceinline__ uint8_t* ring_take(Ring& r, int lane) {
   ++r.next;
   return p;
 }
-__device__ __forceinline__ void ring_store_2d(Ring& r, const CUtensorMap* map, uint8_t* slot,
-                                              int c0, int c1, int lane) {
+__device__ __forceinline__ void ring_store_2d(const CUtensorMap* map, uint8_t* slot, int c0,
+                                              int c1, int lane) {
   fence_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -270,8 +274,21 @@ __device__ __forceinline__ void ring_store_2d(Ring& r, const CUtensorMap* map, u
     bulk_commit();
   }
 }
-__device__ __forceinline__ void ring_store_3d(Ring& r, const CUtensorMap* map, uint8_t* slot,
-                                              int c0, int c1, int c2, int lane) {
+// two slots written at the same coordinates of two tensors, behind one proxy fence
+__device__ __forceinline__ void ring_store_2d_two(const CUtensorMap* m0, uint8_t* s0,
+                                                  const CUtensorMap* m1, uint8_t* s1, int c0,
+                                                  int c1, int lane) {
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(m0, s0, c0, c1);
+    bulk_commit();
+    tma_store_2d(m1, s1, c0, c1);
+    bulk_commit();
+  }
+}
+__device__ __forceinline__ void ring_store_3d(const CUtensorMap* map, uint8_t* slot, int c0,
+                                              int c1, int c2, int lane) {
   fence_async_smem();
   __syncwarp();
   if (lane == 0) {
@@ -328,6 +345,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+// 16-byte unit cc of row r of a slot <- 8 values as bf16
+__device__ __forceinline__ void slot_put8(uint8_t* slot, int r, int cc, const float* v) {
+  *reinterpret_cast<uint4*>(slot + r * 128 + ((cc ^ (r & 7)) << 4)) =
+      make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                 pack_bf16(v[6], v[7]));
+}
 // row r of a slot <- 64 values as bf16
 __device__ __forceinline__ void slot_put_bf16(uint8_t* slot, int r, const float* v) {
 #pragma unroll
@@ -376,14 +399,21 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
   }
 }
 
-// Returns false if the wait for the accumulator timed out.
-// Warp (q, half) covers rows 32q..32q+31 and the half-th of SPLIT column ranges of the
-// accumulator.  Returns false if the wait for the accumulator timed out.
+// First chunk of warp `sub` (of `split` warps sharing a TMEM lane quarter) when `before` chunks
+// of the quarter were dealt before this tile: chunk c goes to warp (before + c) % split.
+__device__ __forceinline__ int q_sub_first(int sub, int before, int split) {
+  return ((sub - before) % split + split) % split;
+}
+
+// Warp (q, sub) covers rows 32q..32q+31 of the tile; with SPLIT > 1 warps per quarter (UP) it
+// takes the 64-column chunks q_sub_first deals to it.  Returns false if the wait for the
+// accumulator timed out.
 template <int KIND>
 __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
-                                              int q, int half, int lane, Ring& ring,
-                                              InRing& inr, uint64_t* tfull, uint32_t parity,
-                                              volatile int* abort_flag) {
+                                              int q, int sub, int lane,
+                                              Ring<Cfg<KIND>::NSLOT>& ring,
+                                              InRing& inr, int tcount, uint64_t* tfull,
+                                              uint32_t parity, volatile int* abort_flag) {
   constexpr int SPLIT = Cfg<KIND>::SPLIT;
   const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
   const bool swiglu = P.act == MOE_ACT_SWIGLU;
@@ -392,10 +422,10 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
-    if (!t.live) return true;  // this CTA's half of the pair tile lies past the weight rows
+    if (!t.live) return true;  // this CTA's sub of the pair tile lies past the weight rows
     const int m_row0 = t.mrow + q * 32;
 #pragma unroll 1
-    for (int c = half * (BN / 32 / SPLIT); c < (half + 1) * (BN / 32 / SPLIT); ++c) {
+    for (int c = sub * (BN / 32 / SPLIT); c < (sub + 1) * (BN / 32 / SPLIT); ++c) {
       const int n = t.n * BN + c * 32;
       if (n >= P.N) break;
       if (nk > 0) {
@@ -410,7 +440,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
       }
       uint8_t* slot = ring_take(ring, lane);
       slot_put_f32(slot, lane, a);
-      ring_store_3d(ring, &P.o0, slot, n, m_row0, t.g, lane);
+      ring_store_3d(&P.o0, slot, n, m_row0, t.g, lane);
     }
     return true;
   }
@@ -422,7 +452,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     const int F = P.N;
     const int per = swiglu ? 2 : 1;              // input slots per chunk
     const int depth = NIN / per;                 // chunks in flight
-    const int ch0 = half * (BN / 64 / SPLIT), ch1 = (half + 1) * (BN / 64 / SPLIT);
+    const int ch0 = sub * (BN / 64 / SPLIT), ch1 = (sub + 1) * (BN / 64 / SPLIT);
     int nch = 0;                                 // chunks of this warp inside [0, F)
     for (int ch = ch0; ch < ch1 && t.n * BN + ch * 64 < F; ++ch) ++nch;
     if (!t.live) nch = 0;
@@ -469,24 +499,30 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
       }
       __syncwarp();   // every lane has read this chunk's input slots
       if (i + depth < nch) issue_chunk(i + depth);
-      ring_store_2d(ring, &P.o0, su, n, row0, lane);
-      if (swiglu) ring_store_2d(ring, &P.o1, sv, n, row0, lane);
+      if (swiglu)
+        ring_store_2d_two(&P.o0, su, &P.o1, sv, n, row0, lane);
+      else
+        ring_store_2d(&P.o0, su, n, row0, lane);
     }
     return true;
   }
   if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
   __syncwarp();
   tc_fence_after();
-  if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
+  if (!t.live) return true;  // this CTA's sub of the pair tile lies past the group's rows
   if (KIND == UP) {
     const int F = P.N;
+    // this warp's chunks: the quarter's chunks are dealt round robin over its SPLIT warps,
+    // continuing from the previous tile (tcount tiles of nch chunks each came before)
+    const int nch = swiglu ? 2 : BN / 64;
+    const int first = (q_sub_first(sub, tcount * nch, SPLIT));
     if (!swiglu) {
 #pragma unroll 1
-      for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
+      for (int ch = first; ch < nch; ch += SPLIT) {
         const int n = t.n * BN + ch * 64;
         if (n >= F) break;
         // Gu = GELU'(u) (what the backward needs) and H = GELU(u) from one erf evaluation,
-        // staged in 32-column halves into two slots
+        // 8 columns at a time into two slots
         uint8_t* sg = ring_take(ring, lane);
         uint8_t* sh = ring_take<1>(ring, lane);
 #pragma unroll 1
@@ -494,27 +530,29 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
           uint32_t r[32];
           tmem_ld32_async(tl + ch * 64 + 32 * h, r);
           tmem_wait_ld();
-          float hv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float u = __uint_as_float(r[i]);
-            const fast::ErfParts q = fast::erf_parts(u);
-            const float phi_cdf = fmaf(0.5f, copysignf(q.erf_abs, u), 0.5f);   // Phi(u)
-            a[i] = fmaf(u, 0.39894228040143268f * q.e, phi_cdf);              // GELU'(u)
-            hv[i] = u * phi_cdf;                                               // GELU(u)
+          for (int c = 0; c < 4; ++c) {
+            float g8[8], h8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float u = __uint_as_float(r[8 * c + i]);
+              const fast::ErfParts e = fast::erf_parts(u);
+              const float phi_cdf = fmaf(0.5f, copysignf(e.erf_abs, u), 0.5f);   // Phi(u)
+              g8[i] = fmaf(u, 0.39894228040143268f * e.e, phi_cdf);              // GELU'(u)
+              h8[i] = u * phi_cdf;                                               // GELU(u)
+            }
+            slot_put8(sg, lane, 4 * h + c, g8);
+            slot_put8(sh, lane, 4 * h + c, h8);
           }
-          slot_put_bf16_half(sg, lane, h, a);
-          slot_put_bf16_half(sh, lane, h, hv);
         }
-        ring_store_2d(ring, &P.o0, sg, n, row0, lane);   // Gu
-        ring_store_2d(ring, &P.o2, sh, n, row0, lane);   // H
+        ring_store_2d_two(&P.o0, sg, &P.o2, sh, n, row0, lane);   // Gu, H
       }
     } else {
       // u (accumulator columns [0, 128)) and v (columns [128, 256)) of one 64-column chunk.
       // Outputs: Gu = v s (1 + u (1 - s)) and Gv = u s (the backward's factors, s = sigmoid(u)),
-      // then H = u s v.  Two passes over TMEM keep two staging slots enough.
+      // then H = u s v in a second pass over TMEM, so that two staging slots are enough.
 #pragma unroll 1
-      for (int ch = half * (2 / SPLIT); ch < (half + 1) * (2 / SPLIT); ++ch) {
+      for (int ch = first; ch < nch; ch += SPLIT) {
         const int n = t.n * (BN / 2) + ch * 64;
         if (n >= F) break;
         const uint32_t tu = tl + ch * 64, tv = tl + BN / 2 + ch * 64;
@@ -526,19 +564,21 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
           tmem_ld32_async(tu + 32 * h, ru);
           tmem_ld32_async(tv + 32 * h, rv);
           tmem_wait_ld();
-          float gv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float u = __uint_as_float(ru[i]), v = __uint_as_float(rv[i]);
-            const float sg = fast::sigmoid(u);
-            a[i] = v * sg * fmaf(u, 1.f - sg, 1.f);   // Gu
-            gv[i] = u * sg;                            // Gv
+          for (int c = 0; c < 4; ++c) {
+            float gu8[8], gv8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float u = __uint_as_float(ru[8 * c + i]), v = __uint_as_float(rv[8 * c + i]);
+              const float sg = fast::sigmoid(u);
+              gu8[i] = v * sg * fmaf(u, 1.f - sg, 1.f);   // Gu
+              gv8[i] = u * sg;                            // Gv
+            }
+            slot_put8(sa, lane, 4 * h + c, gu8);
+            slot_put8(sb, lane, 4 * h + c, gv8);
           }
-          slot_put_bf16_half(sa, lane, h, a);
-          slot_put_bf16_half(sb, lane, h, gv);
         }
-        ring_store_2d(ring, &P.o0, sa, n, row0, lane);   // Gu
-        ring_store_2d(ring, &P.o1, sb, n, row0, lane);   // Gv
+        ring_store_2d_two(&P.o0, sa, &P.o1, sb, n, row0, lane);   // Gu, Gv
         uint8_t* sh = ring_take(ring, lane);
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
@@ -547,26 +587,30 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
           tmem_ld32_async(tv + 32 * h, rv);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float u = __uint_as_float(ru[i]);
-            a[i] = u * fast::sigmoid(u) * __uint_as_float(rv[i]);
+          for (int c = 0; c < 4; ++c) {
+            float h8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float u = __uint_as_float(ru[8 * c + i]);
+              h8[i] = u * fast::sigmoid(u) * __uint_as_float(rv[8 * c + i]);   // H
+            }
+            slot_put8(sh, lane, 4 * h + c, h8);
           }
-          slot_put_bf16_half(sh, lane, h, a);
         }
-        ring_store_2d(ring, &P.o2, sh, n, row0, lane);   // H
+        ring_store_2d(&P.o2, sh, n, row0, lane);   // H
       }
     }
     return true;
   }
   // DOWN, DGRAD_X: plain bf16 output
 #pragma unroll 1
-  for (int ch = half * (BN / 64 / SPLIT); ch < (half + 1) * (BN / 64 / SPLIT); ++ch) {
+  for (int ch = sub * (BN / 64 / SPLIT); ch < (sub + 1) * (BN / 64 / SPLIT); ++ch) {
     const int n = t.n * BN + ch * 64;
     if (n >= P.N) break;
     tmem_ld64(tl + ch * 64, a);
     uint8_t* slot = ring_take(ring, lane);
     slot_put_bf16(slot, lane, a);
-    ring_store_2d(ring, &P.o0, slot, n, row0, lane);
+    ring_store_2d(&P.o0, slot, n, row0, lane);
   }
   return true;
 }
@@ -584,7 +628,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* tiles = smem;
-  uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // 4 warps x NSLOT slots
+  uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // epilogue warps x NSLOT slots
   constexpr int NIN = Cfg<KIND>::NIN;
   uint8_t* in_base = ring_base + RING_BYTES;                     // epilogue warps x NIN slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(in_base + Cfg<KIND>::IN_BYTES);
@@ -725,18 +769,18 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   } else if (warp >= 2) {
     // ---------------- epilogue (both CTAs)
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
-    Ring ring{ring_base + (warp - 2) * NSLOT * SLOT_BYTES, 0};
+    const int sub = (warp - 2) >> 2;   // which of the quarter's SPLIT warps
+    Ring<Cfg<KIND>::NSLOT> ring{ring_base + (warp - 2) * Cfg<KIND>::NSLOT * SLOT_BYTES, 0};
     InRing inr{in_base + (warp - 2) * NIN * SLOT_BYTES, in_bars + (warp - 2) * NIN, 0, 0};
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
-    int acc = 0;
+    int acc = 0, tcount = 0;
     uint32_t acc_phase = 0;
-    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs, ++tcount) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
-      if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, half, lane,
-                               ring, inr, &tfull[acc], acc_phase, abort_flag))
+      if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, sub, lane,
+                               ring, inr, tcount, &tfull[acc], acc_phase, abort_flag))
         break;
       tc_fence_before();
       __syncwarp();

@@ -8,6 +8,9 @@ namespace moe {
 size_t router_smem_bytes(int E);
 moe_status launch_router(const Dims& D, const void* x, const void* Wg, const float* bias,
                          float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
+bool router_warp_supported(const Dims& D);
+moe_status launch_router_warp(const Dims& D, const void* x, const void* Wg, const float* bias,
+                              float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
 moe_status launch_topk_from_logits(const Dims& D, const float* logits, int32_t* topk_idx,
                                    float* topk_w, cudaStream_t st);
 moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,

@@ -8,6 +8,8 @@
 // CTA owns 64 tokens, computes their [64 x E] logit tile with fp32 FMA (x and Wg staged through
 // shared memory), adds the constant bias and writes the logits; then one thread per token runs
 // the serial softmax + top-k of route_serial.cuh over its row in shared memory.
+#include <algorithm>
+
 #include "common.cuh"
 #include "route_serial.cuh"
 
@@ -97,7 +99,123 @@ __global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T_
   topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
 }
 
+// Few experts: one warp per token.  The CTA stages the whole gate matrix Wg [E, d] in shared
+// memory; a warp reads its token's row once (16-byte vectors, lane-strided), keeps EP partial
+// dot products per lane, and folds them across the warp with a transposing butterfly (each
+// exchange halves the values a lane keeps), after which lane l holds the logit of expert
+// l >> (5 - log2 EP).  Lane 0 then runs the serial softmax + top-k of route_serial.cuh.
+constexpr int RW_THREADS = 512;
+
+template <int EP>
+__device__ __forceinline__ float transpose_reduce(float (&acc)[EP], int lane) {
+  int n = EP;
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int off = 16 >> s;
+    if (n > 1) {
+      const int h = n >> 1;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < EP / 2; ++i)
+        if (i < h) {
+          const float send = up ? acc[i] : acc[i + h];
+          const float keep = up ? acc[i + h] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      n = h;
+    } else {
+      acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+    }
+  }
+  return acc[0];
+}
+
+template <typename T, int EP>
+__global__ void __launch_bounds__(RW_THREADS)
+router_warp_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
+                   const float* __restrict__ bias, int T_, int d, int E, int k, int gate_norm,
+                   float* __restrict__ logits, int32_t* __restrict__ topk_idx,
+                   float* __restrict__ topk_w) {
+  pdl_prologue();
+  constexpr int VN = Vec16<T>::N;
+  constexpr int SH = (EP >= 32) ? 0 : (EP >= 16) ? 1 : (EP >= 8) ? 2 : (EP >= 4) ? 3 : (EP >= 2) ? 4 : 5;
+  extern __shared__ uint4 rw_smem[];
+  const int nv = d / VN;
+  const uint4* wsrc = reinterpret_cast<const uint4*>(Wg);
+  for (int q = threadIdx.x; q < E * nv; q += RW_THREADS) rw_smem[q] = __ldg(wsrc + q);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warps = RW_THREADS / 32;
+  const int e_l = lane >> SH;   // expert whose logit this lane ends up with
+  const float b_l = (bias != nullptr && e_l < E) ? bias[e_l] : 0.f;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T_; t += gridDim.x * warps) {
+    float acc[EP];
+#pragma unroll
+    for (int e = 0; e < EP; ++e) acc[e] = 0.f;
+    const T* xr = x + (int64_t)t * d;
+    for (int v = lane; v < nv; v += 32) {
+      const Vec16<T> xv = ld_vec_stream(xr + (int64_t)v * VN);
+      float xf[VN];
+#pragma unroll
+      for (int i = 0; i < VN; ++i) xf[i] = xv.get(i);
+#pragma unroll
+      for (int e = 0; e < EP; ++e)
+        if (e < E) {
+          Vec16<T> w;
+          w.raw = rw_smem[e * nv + v];
+#pragma unroll
+          for (int i = 0; i < VN; ++i) acc[e] = fmaf(xf[i], w.get(i), acc[e]);
+        }
+    }
+    const float lg = transpose_reduce<EP>(acc, lane) + b_l;
+    if ((lane & ((1 << SH) - 1)) == 0 && e_l < E) logits[(int64_t)t * E + e_l] = lg;
+    TopK8 st;
+    topk_init(st);
+    for (int e = 0; e < E; ++e) {
+      const float v = __shfl_sync(0xffffffffu, lg, e << SH);
+      if (lane == 0) topk_push(st, v, e);
+    }
+    if (lane == 0) topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
+  }
+}
+
+template <typename T, int EP>
+static moe_status router_warp_t(const Dims& D, const void* x, const void* Wg, const float* bias,
+                                float* logits, int32_t* topk_idx, float* topk_w,
+                                cudaStream_t st) {
+  const size_t sm = (size_t)D.E * D.d * sizeof(T);
+  auto kern = router_warp_kernel<T, EP>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int grid = (int)std::min<int64_t>((D.T + RW_THREADS / 32 - 1) / (RW_THREADS / 32), 148);
+  return launch_k(kern, grid, RW_THREADS, sm, st, 1, (const T*)x, (const T*)Wg, bias, D.T, D.d,
+                  D.E, D.k, D.gate_norm, logits, topk_idx, topk_w);
+}
+
+template <typename T>
+static moe_status router_warp_e(const Dims& D, const void* x, const void* Wg, const float* bias,
+                                float* logits, int32_t* topk_idx, float* topk_w,
+                                cudaStream_t st) {
+  if (D.E <= 4) return router_warp_t<T, 4>(D, x, Wg, bias, logits, topk_idx, topk_w, st);
+  if (D.E <= 8) return router_warp_t<T, 8>(D, x, Wg, bias, logits, topk_idx, topk_w, st);
+  if (D.E <= 16) return router_warp_t<T, 16>(D, x, Wg, bias, logits, topk_idx, topk_w, st);
+  return router_warp_t<T, 32>(D, x, Wg, bias, logits, topk_idx, topk_w, st);
+}
+
 }  // namespace
+
+bool router_warp_supported(const Dims& D) {
+  const int esz = D.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  return D.E <= 32 && D.d % (16 / esz) == 0 && (size_t)D.E * D.d * esz <= (size_t)96 * 1024;
+}
+
+moe_status launch_router_warp(const Dims& D, const void* x, const void* Wg, const float* bias,
+                              float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  const float* b = D.has_bias ? bias : nullptr;
+  if (D.dtype == MOE_DTYPE_BF16)
+    return router_warp_e<__nv_bfloat16>(D, x, Wg, b, logits, topk_idx, topk_w, st);
+  return router_warp_e<float>(D, x, Wg, b, logits, topk_idx, topk_w, st);
+}
 
 size_t router_smem_bytes(int E) {
   return sizeof(float) * (RT_BK * (RT_TOK + 4) + RT_BK * (RT_EC + 4) + RT_TOK * (E + 1));

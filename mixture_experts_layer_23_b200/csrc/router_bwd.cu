@@ -8,6 +8,8 @@
 //   (the softmax backward, dl from dg, runs inside the combine backward kernel)
 //   dWg = dl^T x (two-level fixed-order reduction, bit-reproducible)
 //   dx  = dl Wg + sum_j dXd[slot_j] + sum_s dXd[shared row of t]   (a gather, no atomics)
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace moe {
@@ -192,7 +194,123 @@ undispatch_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
   }
 }
 
+// Few experts (the gate matrix fits in shared memory): one warp per token, persistent CTAs.  The
+// CTA stages Wg [E, d] once; a warp loads its token's k routed and S shared dXd rows, U = 8 / KR
+// vectors per lane at a time with all loads in flight together, and the dl row (lane e holds
+// dl[t, e], broadcast by shuffles).  Per element: (sum_e dl_e Wg_e) + routed rows j = 0..k-1 +
+// (sum of shared rows), a fixed order.
+constexpr int UW_THREADS = 512;
+
+template <typename T, int KR>
+__global__ void __launch_bounds__(UW_THREADS)
+undispatch_warp_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
+                       const T* __restrict__ dXd, const int32_t* __restrict__ slot, int T_, int d,
+                       int E, int k, int S, int64_t T_pad, T* __restrict__ dx) {
+  pdl_prologue();
+  constexpr int VN = Vec16<T>::N;
+  constexpr int U = KR >= 8 ? 1 : 8 / KR;
+  extern __shared__ uint4 uw_smem[];
+  const int nv = d / VN;
+  const uint4* wsrc = reinterpret_cast<const uint4*>(Wg);
+  for (int q = threadIdx.x; q < E * nv; q += UW_THREADS) uw_smem[q] = __ldg(wsrc + q);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warps = UW_THREADS / 32;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T_; t += gridDim.x * warps) {
+    int my_s = -1;
+    if (lane < k)
+      my_s = slot[(int64_t)t * k + lane];
+    else if (lane < k + S)
+      my_s = (int)((int64_t)(lane - k) * T_pad + t);
+    const float my_dl = lane < E ? dl[(int64_t)t * E + lane] : 0.f;
+    int s[KR];
+#pragma unroll
+    for (int j = 0; j < KR; ++j) {
+      s[j] = __shfl_sync(0xffffffffu, my_s, j);
+      if (j >= k + S) s[j] = -1;
+    }
+    // the loop bounds are the same for every lane (the dl shuffles need the whole warp)
+    for (int base = 0; base < nv; base += 32 * U) {
+      const int v0 = base + lane;
+      Vec16<T> g[U][KR];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int j = 0; j < KR; ++j) {
+          const int v = v0 + 32 * u;
+          if (v < nv && s[j] >= 0) g[u][j] = ld_vec_stream(dXd + (int64_t)s[j] * d + (int64_t)v * VN);
+        }
+      float acc[U][VN];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int i = 0; i < VN; ++i) acc[u][i] = 0.f;
+      for (int e = 0; e < E; ++e) {
+        const float w = __shfl_sync(0xffffffffu, my_dl, e);
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nv) {
+            Vec16<T> wv;
+            wv.raw = uw_smem[e * nv + v];
+#pragma unroll
+            for (int i = 0; i < VN; ++i) acc[u][i] = fmaf(w, wv.get(i), acc[u][i]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int v = v0 + 32 * u;
+        if (v >= nv) break;
+        Vec16<T> out;
+#pragma unroll
+        for (int i = 0; i < VN; ++i) {
+          float r = acc[u][i], sh = 0.f;
+#pragma unroll
+          for (int j = 0; j < KR; ++j)
+            if (s[j] >= 0) {
+              if (j < k) r += g[u][j].get(i);
+              else sh += g[u][j].get(i);
+            }
+          out.set(i, r + sh);
+        }
+        st_vec(dx + (int64_t)t * d + (int64_t)v * VN, out);
+      }
+    }
+  }
+}
+
 }  // namespace
+
+bool undispatch_warp_supported(const Dims& D) {
+  const int esz = D.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  return D.E <= 32 && D.k + D.S <= 16 && (size_t)D.E * D.d * esz <= (size_t)96 * 1024;
+}
+
+template <typename T, int KR>
+static moe_status undispatch_warp_t(const Dims& D, const float* dlogits, const void* Wg,
+                                    const void* dXd, const int32_t* slot, void* dx,
+                                    cudaStream_t st) {
+  const size_t sm = (size_t)D.E * D.d * sizeof(T);
+  auto kern = undispatch_warp_kernel<T, KR>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int wpc = UW_THREADS / 32;
+  const int grid = (int)std::min<int64_t>((D.T + wpc - 1) / wpc, 148);
+  return launch_k(kern, grid, UW_THREADS, sm, st, 1, dlogits, (const T*)Wg, (const T*)dXd, slot,
+                  D.T, D.d, D.E, D.k, D.S, D.T_pad, (T*)dx);
+}
+
+template <typename T>
+static moe_status undispatch_warp_kr(const Dims& D, const float* dlogits, const void* Wg,
+                                     const void* dXd, const int32_t* slot, void* dx,
+                                     cudaStream_t st) {
+  const int r = D.k + D.S;
+  if (r <= 2) return undispatch_warp_t<T, 2>(D, dlogits, Wg, dXd, slot, dx, st);
+  if (r <= 4) return undispatch_warp_t<T, 4>(D, dlogits, Wg, dXd, slot, dx, st);
+  if (r <= 8) return undispatch_warp_t<T, 8>(D, dlogits, Wg, dXd, slot, dx, st);
+  return undispatch_warp_t<T, 16>(D, dlogits, Wg, dXd, slot, dx, st);
+}
 
 moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
                                float* dWg, cudaStream_t st) {
@@ -226,6 +344,11 @@ static moe_status undispatch_t(const Dims& D, const float* dlogits, const void* 
 
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
                              const int32_t* slot, void* dx, cudaStream_t st) {
+  if (undispatch_warp_supported(D)) {
+    if (D.dtype == MOE_DTYPE_BF16)
+      return undispatch_warp_kr<__nv_bfloat16>(D, dlogits, Wg, dXd, slot, dx, st);
+    return undispatch_warp_kr<float>(D, dlogits, Wg, dXd, slot, dx, st);
+  }
   if (D.dtype == MOE_DTYPE_BF16)
     return undispatch_t<__nv_bfloat16>(D, dlogits, Wg, dXd, slot, dx, st);
   return undispatch_t<float>(D, dlogits, Wg, dXd, slot, dx, st);

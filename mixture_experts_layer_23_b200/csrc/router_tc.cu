@@ -8,10 +8,13 @@
 //
 // One CTA per 128 tokens (192 threads): warp 0 streams x tiles [128 x 64] and the whole gate
 // matrix slice [E_pad x 64] (E rounded up to 16, zero rows from TMA's out-of-bounds fill) through
-// a 4-stage ring; one lane of warp 1 issues tcgen05.mma (M = 128, N = E_pad) into a TMEM
+// a ring of up to 16 stages (as many as shared memory holds: with d <= 1024 and few experts the
+// whole token tile is in flight at once, since a CTA has only one tile to load); one lane of warp 1 issues tcgen05.mma (M = 128, N = E_pad) into a TMEM
 // accumulator; warps 2..5 read it back with tcgen05.ld, so each thread holds the E logits of one
 // token, adds the bias, writes the logits and runs the serial softmax + top-k of route_serial.cuh.
 #include <string.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "launch.h"
@@ -23,7 +26,8 @@ namespace moe {
 namespace tc {
 namespace {
 
-constexpr int RSTAGES = 4;
+constexpr int MAX_RSTAGES = 16;
+constexpr size_t RSMEM_BUDGET = 200 * 1024;   // stage ring bytes
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
 
 struct alignas(64) RouterParams {
@@ -37,6 +41,7 @@ struct alignas(64) RouterParams {
   unsigned long long timeout_ns;
   int T, d, E, E_pad, k, gate_norm;
   uint32_t idesc, tmem_cols, stage_bytes;
+  int nstages;
 };
 
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
@@ -44,6 +49,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
+  const int RSTAGES = P.nstages;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RSTAGES * P.stage_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + RSTAGES;
@@ -186,7 +192,9 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   while ((int)cols < E_pad) cols <<= 1;
   P.tmem_cols = cols;
   P.stage_bytes = RA_BYTES + (uint32_t)E_pad * 128u;
-  const size_t smem = 1024 + RSTAGES * (size_t)P.stage_bytes + 256;
+  P.nstages = (int)std::min<size_t>(std::min<size_t>(MAX_RSTAGES, RSMEM_BUDGET / P.stage_bytes),
+                                    (size_t)(D.d / 64));
+  const size_t smem = 1024 + (size_t)P.nstages * P.stage_bytes + 512;
   if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;

@@ -74,9 +74,17 @@ EDGE = [
     # tensor-core router at its widest (E = 256 experts, N = 256 accumulator columns), k = 8
     LayerShape("wide_router_tc", T=300, d=64, E=256, k=8, d_ff=64, capacity_factor=2.0,
                dtype=BF16, bias="normal"),
-    # tensor-core router with E not a multiple of 16 and a ragged last token tile
-    LayerShape("odd_experts_tc", T=517, d=128, E=13, k=3, d_ff=128, capacity_factor=1.1,
+    # tensor-core router (more than 32 experts) with E not a multiple of 16 and a ragged last
+    # token tile
+    LayerShape("odd_experts_tc", T=517, d=128, E=45, k=3, d_ff=128, capacity_factor=1.1,
                dtype=BF16, bias="zipf"),
+    # warp-per-token router and un-dispatch at their widest (32 experts, every lane holds a
+    # logit), d not a multiple of 64 (so not the tensor-core router) nor of the warp's 256-column
+    # stride, k = 8
+    LayerShape("warp_router_e32", T=333, d=136, E=32, k=8, d_ff=64, capacity_factor=1.5,
+               dtype=BF16, bias="normal"),
+    LayerShape("warp_router_fp32", T=301, d=100, E=24, k=3, d_ff=36, n_shared=1,
+               capacity_factor=1.2, dtype=FP32, bias="zipf"),
 ]
 
 
