@@ -114,6 +114,11 @@ ScratchLayout scratch_layout(const Dims& D) {
   S.dg = take(T * D.k * 4);
   S.dlogits = take(T * D.E * 4);
   S.dWg_part = take((size_t)D.n_tchunk * D.E * D.d * 4);
+  S.dl16 = S.dxg = 0;
+  if (router_bwd_tc_supported(D)) {
+    S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
+    S.dxg = take(T * D.d * 2);
+  }
   S.total = off;
   return S;
 }
@@ -381,14 +386,30 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   float* dl = (float*)(s + S.dlogits);
   float* part = (float*)(s + S.dWg_part);
   MOE_TRY(mark_bwd(0, st));
-  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, dg, dl, dO, st));
+  // many experts (bf16): both router-backward contractions run on the tensor cores from a bf16
+  // copy of dlogits; otherwise CUDA-core kernels read the fp32 dlogits
+  const bool rtc = S.dl16 != 0;
+  __nv_bfloat16* dl16 = rtc ? (__nv_bfloat16*)(s + S.dl16) : nullptr;
+  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, dg, dl, dl16, dO, st));
   MOE_TRY(mark_bwd(1, st));
-  MOE_TRY(launch_router_wgrad(D, dl, x, part, dWg, st));
+  if (rtc) {
+    int n_chunks = 0;
+    MOE_TRY(launch_router_wgrad_tc(D, dl16, x, part, &n_chunks, (uint32_t*)(s + S.status), st));
+    MOE_TRY(launch_router_wgrad_reduce(D, part, n_chunks, dWg, st));
+  } else {
+    MOE_TRY(launch_router_wgrad(D, dl, x, part, dWg, st));
+  }
   MOE_TRY(mark_bwd(2, st));
   MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, U, V, H, dU, dV, dXd, dW1, dW3, dW2,
                      (uint32_t*)(s + S.status), st));
   MOE_TRY(mark_bwd(6, st));
-  MOE_TRY(launch_undispatch(D, dl, Wg, dXd, slot, dx, st));
+  if (rtc) {
+    void* dxg = s + S.dxg;
+    MOE_TRY(launch_router_dx_tc(D, dl16, Wg, dxg, (uint32_t*)(s + S.status), st));
+    MOE_TRY(launch_undispatch_gather(D, dxg, dXd, slot, dx, st));
+  } else {
+    MOE_TRY(launch_undispatch(D, dl, Wg, dXd, slot, dx, st));
+  }
   MOE_TRY(mark_bwd(7, st));
   return MOE_OK;
 }

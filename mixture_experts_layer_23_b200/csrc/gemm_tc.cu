@@ -36,6 +36,8 @@
 #include <cuda.h>  // CUtensorMap and its enums (types only; the encoder is fetched at run time)
 #include <string.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 #include "tc_host.h"
@@ -102,6 +104,8 @@ struct alignas(64) Params {
   int K;                 // row GEMMs: inner dimension (d or F)
   int act;
   int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
+  int chunk;             // > 0: the groups are fixed chunks of this many token rows (router
+                         // backward) instead of the experts' row ranges
 };
 
 // Instruction descriptor of the pair MMA: bf16 x bf16 -> fp32, M = 256 (two CTAs), N = BN.
@@ -140,7 +144,13 @@ __device__ __forceinline__ int group_tiles(const Params& P, int rows) {
 
 __device__ __forceinline__ void group_rows(const Params& P, int g, int& a_row, int& o_row,
                                            int& rows, bool& shared) {
-  if (g < P.E) {
+  if (P.chunk > 0) {   // token chunk g: rows [g * chunk, min((g + 1) * chunk, T)), K-padded to 64
+    a_row = g * P.chunk;
+    o_row = a_row;
+    const int n = P.T - a_row < P.chunk ? P.T - a_row : P.chunk;
+    rows = (int)round_up(n, BK);
+    shared = false;
+  } else if (g < P.E) {
     a_row = P.offsets[g];
     o_row = a_row;
     rows = P.offsets[g + 1] - a_row;
@@ -422,8 +432,9 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
-    if (!t.live) return true;  // this CTA's sub of the pair tile lies past the weight rows
+    if (!t.live) return true;  // this CTA's half of the pair tile lies past the weight rows
     const int m_row0 = t.mrow + q * 32;
+    if (m_row0 >= P.Mw) return true;  // this warp's 32 rows lie past the weight rows
 #pragma unroll 1
     for (int c = sub * (BN / 32 / SPLIT); c < (sub + 1) * (BN / 32 / SPLIT); ++c) {
       const int n = t.n * BN + c * 32;
@@ -509,7 +520,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
   __syncwarp();
   tc_fence_after();
-  if (!t.live) return true;  // this CTA's sub of the pair tile lies past the group's rows
+  if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
   if (KIND == UP) {
     const int F = P.N;
     // this warp's chunks: the quarter's chunks are dealt round robin over its SPLIT warps,
@@ -952,6 +963,63 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
   P.which = 2;
   const int tiles = D.E_tot * ((D.d + BMP - 1) / BMP) * ((D.F + BN - 1) / BN);
   return launch<WGRAD>(P, tiles, st);
+}
+
+// ----------------------------------------------------------------------------- router backward
+//
+// With many experts the router's two backward contractions are GEMMs worth the tensor cores
+// (2 T E d FLOPs each; 4.3 GFLOP for T = 16384, E = 64, d = 2048).  Both read a bf16 copy of
+// dlogits, dl16 [T, E8] (E8 = E rounded up to 8, zero padded), and reuse the grouped kernel with
+// fixed token chunks as its groups:
+//   dWg partials  (WGRAD form): part[c] = dl16[chunk c]^T x[chunk c]  -> [n_chunks, E, d] fp32,
+//                 M = E, N = d, K = the chunk's tokens; summed over c in order afterwards
+//   dl Wg         (DGRAD_X form): dxg = dl16 Wg -> [T, d] bf16, one chunk of all T rows, K = E
+
+bool router_bwd_tc_supported(const Dims& D) {
+  return D.dtype == MOE_DTYPE_BF16 && D.E > 32 && D.d % 64 == 0 && tc::encoder() != nullptr;
+}
+
+moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
+                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st) {
+  using namespace tc;
+  Params P = base_params(D, nullptr, status);
+  const int E8 = (int)round_up(D.E, 8);
+  if (!(map2(&P.a_main, dl16, E8, D.T, 64, 64) && map2(&P.b_main, x, D.d, D.T, 64, 64)))
+    return MOE_ERR_CUDA;
+  const int n_tiles = (int)(((D.E + BMP - 1) / BMP) * ((D.d + BN - 1) / BN));
+  // enough chunks to give every CTA pair a tile, within the partial buffer and the group table
+  int nc = (num_sms() / 2 + n_tiles - 1) / n_tiles;
+  nc = std::min(nc, std::min(D.n_tchunk, MAX_GROUPS));
+  nc = std::max(1, std::min<int>(nc, (int)((D.T + BK - 1) / BK)));
+  const int chunk = (int)round_up((D.T + nc - 1) / nc, BK);
+  nc = (D.T + chunk - 1) / chunk;
+  if (!map3_f32(&P.o0, part, D.d, D.E, nc, 32, 32)) return MOE_ERR_CUDA;
+  P.E = nc;
+  P.S = 0;
+  P.chunk = chunk;
+  P.Mw = D.E;
+  P.N = D.d;
+  P.which = 0;
+  *n_chunks = nc;
+  return launch<WGRAD>(P, nc * n_tiles, st);
+}
+
+moe_status launch_router_dx_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
+                               void* dxg, uint32_t* status, cudaStream_t st) {
+  using namespace tc;
+  Params P = base_params(D, nullptr, status);
+  P.act = MOE_ACT_GELU;   // one operand pair per K block (not the SwiGLU pair of DGRAD_X)
+  const int E8 = (int)round_up(D.E, 8);
+  if (!(map2(&P.a_main, dl16, E8, D.T, 64, BM) && map3(&P.b_main, Wg, D.d, D.E, 1, 64, 64) &&
+        map2(&P.o0, dxg, D.d, D.T, 64, 32)))
+    return MOE_ERR_CUDA;
+  P.E = 1;
+  P.S = 0;
+  P.chunk = (int)round_up(D.T, BK);
+  P.N = D.d;
+  P.K = (int)round_up(D.E, BK);
+  const int tiles = (int)(((D.T + BMP - 1) / BMP) * ((D.d + BN - 1) / BN));
+  return launch<DGRAD_X>(P, tiles, st);
 }
 
 }  // namespace moe

@@ -21,7 +21,18 @@ moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, con
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
                               const int32_t* kept, const int32_t* offsets, float* dg,
-                              float* dlogits, void* dO, cudaStream_t st);
+                              float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st);
+// Router backward on the tensor cores (bf16, more than 32 experts): dWg partials over token
+// chunks, their fixed-order sum, dl Wg, and the un-dispatch gather that adds it.
+bool router_bwd_tc_supported(const Dims& D);
+moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
+                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st);
+moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,
+                                      cudaStream_t st);
+moe_status launch_router_dx_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
+                               void* dxg, uint32_t* status, cudaStream_t st);
+moe_status launch_undispatch_gather(const Dims& D, const void* dxg, const void* dXd,
+                                    const int32_t* slot, void* dx, cudaStream_t st);
 moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
                                float* dWg, cudaStream_t st);
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,
