@@ -23,6 +23,7 @@ timed on a bounded sample (rank 0, one GPU).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -36,6 +37,28 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE-layer tokens/s fwd+bwd on 1 B200; % bf16 TC peak (GEMM), % HBM BW (rest)"
 FLUSH_BYTES = 256 << 20
 GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2"}
+
+
+# DRAM traffic of a kernel from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of
+# one launch), keyed by workload and phase.  It stands only for the kernel sources it was taken on:
+# the SHA-256 of those files is stored with it and the bench reports null once they have changed.
+GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "act_fast.cuh", "common.cuh"]
+NCU_TRAFFIC = {}
+
+
+def sources_sha256(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "mixture_experts_layer_23_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload, phase):
+    e = NCU_TRAFFIC.get((workload, phase))
+    if e is None or sources_sha256(e["sources"]) != e["sha256"]:
+        return None, None
+    return e["bytes"], e["profile"]
 
 
 def parse():
@@ -364,15 +387,19 @@ def run_ours(args):
             ach = amount / (ms * 1e-3) / 1e9
             phases[name] = {"ms": ms, "bound": bound, "achieved_gbs": ach, "frac": ach / hbm_gbs}
     tb, tw = work[top]
+    traffic, traffic_src = measured_traffic(shape.name, top)
     if tb == "tensor":
         ach = tw / (top_ms_live * 1e-3) / 1e12
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16_tf,
-                "unit": "TFLOP/s", "frac": ach / bf16_tf, "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / bf16_tf, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
     else:
         ach = tw / (top_ms_live * 1e-3) / 1e9
         roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
-                "frac": ach / hbm_gbs, "traffic": None, "peak_source": f"{peak_src} HBM copy"}
+                "frac": ach / hbm_gbs, "traffic": traffic, "peak_source": f"{peak_src} HBM copy"}
+    if traffic is not None:
+        roof["traffic_unit"] = "bytes per launch"
+        roof["traffic_source"] = traffic_src
 
     # end to end through the C ABI with host buffers
     x_pin = x.cpu().pin_memory()

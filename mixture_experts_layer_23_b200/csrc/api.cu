@@ -386,8 +386,8 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   float* dl = (float*)(s + S.dlogits);
   float* part = (float*)(s + S.dWg_part);
   MOE_TRY(mark_bwd(0, st));
-  // many experts (bf16): both router-backward contractions run on the tensor cores from a bf16
-  // copy of dlogits; otherwise CUDA-core kernels read the fp32 dlogits
+  // bf16 with d a multiple of 64: both router-backward contractions run on the tensor cores
+  // from a bf16 copy of dlogits; otherwise CUDA-core kernels read the fp32 dlogits
   const bool rtc = S.dl16 != 0;
   __nv_bfloat16* dl16 = rtc ? (__nv_bfloat16*)(s + S.dl16) : nullptr;
   MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, dg, dl, dl16, dO, st));

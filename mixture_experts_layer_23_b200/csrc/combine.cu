@@ -16,8 +16,11 @@ namespace {
 // y_t = sum_j w_j O[slot_j] + sum_s O[s * T_pad + t].  KS >= k + S (a power of two): the
 // token's rows are gathered U = max(1, 8 / KS) vectors per lane at a time, all loads in flight
 // before the sums.
+// Occupancy: 4 CTAs of 256 threads per SM (64 registers) keep a whole T / 8 grid resident in one
+// wave for T up to 4736, where 3 (the register count unconstrained) left a tail wave; the
+// 16-row form stays at 2 CTAs (it would spill).
 template <typename T, int KS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, KS >= 16 ? 2 : 4)
 combine_fwd_kernel(const T* __restrict__ O, const int32_t* __restrict__ slot,
                    const float* __restrict__ topk_w, int T_, int d, int k, int S, int64_t T_pad,
                    T* __restrict__ y) {
@@ -150,7 +153,7 @@ __device__ __forceinline__ void dlogits_row(const float* __restrict__ lrow, cons
 }
 
 template <typename T, int KS>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                    const int32_t* __restrict__ slot, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ topk_idx, const float* __restrict__ logits,

@@ -967,8 +967,9 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
 
 // ----------------------------------------------------------------------------- router backward
 //
-// With many experts the router's two backward contractions are GEMMs worth the tensor cores
-// (2 T E d FLOPs each; 4.3 GFLOP for T = 16384, E = 64, d = 2048).  Both read a bf16 copy of
+// The router's two backward contractions are GEMMs worth the tensor cores (2 T E d FLOPs each;
+// 4.3 GFLOP for T = 16384, E = 64, d = 2048; measured faster than the CUDA-core kernels from
+// E = 16 up, by 2x at E = 32).  Both read a bf16 copy of
 // dlogits, dl16 [T, E8] (E8 = E rounded up to 8, zero padded), and reuse the grouped kernel with
 // fixed token chunks as its groups:
 //   dWg partials  (WGRAD form): part[c] = dl16[chunk c]^T x[chunk c]  -> [n_chunks, E, d] fp32,
@@ -976,7 +977,7 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
 //   dl Wg         (DGRAD_X form): dxg = dl16 Wg -> [T, d] bf16, one chunk of all T rows, K = E
 
 bool router_bwd_tc_supported(const Dims& D) {
-  return D.dtype == MOE_DTYPE_BF16 && D.E > 32 && D.d % 64 == 0 && tc::encoder() != nullptr;
+  return D.dtype == MOE_DTYPE_BF16 && D.d % 64 == 0 && tc::encoder() != nullptr;
 }
 
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,

@@ -22,7 +22,7 @@ moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, cons
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
                               const int32_t* kept, const int32_t* offsets, float* dg,
                               float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st);
-// Router backward on the tensor cores (bf16, more than 32 experts): dWg partials over token
+// Router backward on the tensor cores (bf16, d a multiple of 64): dWg partials over token
 // chunks, their fixed-order sum, dl Wg, and the un-dispatch gather that adds it.
 bool router_bwd_tc_supported(const Dims& D);
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,

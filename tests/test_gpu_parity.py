@@ -85,7 +85,7 @@ EDGE = [
                dtype=BF16, bias="normal"),
     LayerShape("warp_router_fp32", T=301, d=100, E=24, k=3, d_ff=36, n_shared=1,
                capacity_factor=1.2, dtype=FP32, bias="zipf"),
-    # router backward on the tensor cores (more than 32 experts): E = 72 is not a multiple of the
+    # router backward on the tensor cores: E = 72 is not a multiple of the
     # 64-wide K block, T not a multiple of the token chunk, with shared experts and SwiGLU
     LayerShape("router_bwd_tc_shared", T=700, d=192, E=72, k=6, d_ff=128, n_shared=2,
                capacity_factor=1.5, act=SWIGLU, dtype=BF16, bias="normal"),
