@@ -57,6 +57,7 @@ constexpr uint32_t B_BYTES = BNH * BK * 2;          // 16 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES; // per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
+constexpr int TILE_GROUP_M = 16;  // m tiles per band of the tile order (see decode)
 // Epilogue staging: each epilogue warp owns a ring of Cfg::NSLOT 4 KB slots (32 rows x 128 B, laid out
 // in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
 constexpr uint32_t SLOT_BYTES = 32 * 128;
@@ -174,10 +175,20 @@ __device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, i
   Tile T;
   T.g = lo;
   group_rows(P, lo, T.a_row, T.o_row, T.rows, T.shared);
+  // Tile order inside the group: bands of TILE_GROUP_M m tiles, each walked m-fastest across all
+  // n tiles.  The CTA pairs run consecutive tile indices at the same time, so one wave of pairs
+  // touches about TILE_GROUP_M A slices and (pairs / TILE_GROUP_M) B slices, which stay in L2;
+  // walking all m tiles first would stream the whole A operand from DRAM once per wave when it
+  // is larger than L2 (the weight gradients of a 14336-wide expert).
   const int local = t - tile_start[lo];
   const int mt = m_tiles<KIND>(P, T.rows);
-  T.m = local % mt;
-  T.n = local / mt;
+  const int nt = (P.N + tile_n<KIND>(P) - 1) / tile_n<KIND>(P);
+  const int band = local / (TILE_GROUP_M * nt);
+  const int m0 = band * TILE_GROUP_M;
+  const int gm = mt - m0 < TILE_GROUP_M ? mt - m0 : TILE_GROUP_M;
+  const int r = local - band * TILE_GROUP_M * nt;
+  T.m = m0 + r % gm;
+  T.n = r / gm;
   T.mrow = T.m * BMP + rank * BM;
   T.live = T.mrow < (KIND == WGRAD ? P.Mw : T.rows);
   return T;
