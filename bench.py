@@ -43,7 +43,16 @@ GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wg
 # one launch), keyed by workload and phase.  It stands only for the kernel sources it was taken on:
 # the SHA-256 of those files is stored with it and the bench reports null once they have changed.
 GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "act_fast.cuh", "common.cuh"]
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # python bench.py --steps 1 --warmup 1 --no-cpu-baseline under ncu --set full, one launch of
+    # the up-projection GEMM: dram__bytes_read.sum 89.720064 MB + dram__bytes_write.sum 60.959232 MB
+    ("gpt2_gshard", "expert_up"): {
+        "bytes": 150679296,
+        "sources": GEMM_SOURCES,
+        "sha256": "be35e948941c8af985dc6e69584e6d6f598b5d6a7bc4e2d7e29029765e893ecd",
+        "profile": "profiles/expert_up_gpt2_gshard.md",
+    },
+}
 
 
 def sources_sha256(files):
@@ -233,9 +242,16 @@ class ClockSampler:
                 "reasons": sorted(self.reasons)}
 
 
+# fp32 layers run their GEMMs on the CUDA cores: peak = 148 SMs x 128 FP32 lanes x 2 FLOP (FMA)
+# x 1965 MHz (the B200's maximum SM clock)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1965e6 / 1e12
+
+
 def phase_work(shape, n_kept):
-    """Algorithmic work per phase: FLOPs for the GEMMs (kept rows only), bytes for the rest."""
+    """Algorithmic work per phase: FLOPs for the GEMMs (kept rows only), bytes for the rest.  The
+    GEMMs of bf16 layers are tensor-core bound, those of fp32 layers ALU (FMA) bound."""
     b = 2 if shape.dtype == 1 else 4
+    mm = "tensor" if shape.dtype == 1 else "alu"
     T, d, F, S, E, k = shape.T, shape.d, shape.d_ff, shape.n_shared, shape.E, shape.k
     rows = n_kept + S * T
     g = 2 if shape.act == 1 else 1
@@ -243,15 +259,15 @@ def phase_work(shape, n_kept):
     return {
         "router": ("hbm", Td + E * d * b + T * E * 4 + T * k * 8),
         "dispatch": ("hbm", Td + Nd + T * k * 8),
-        "expert_up": ("tensor", 2.0 * rows * d * F * g),
-        "expert_down": ("tensor", 2.0 * rows * F * d),
+        "expert_up": (mm, 2.0 * rows * d * F * g),
+        "expert_down": (mm, 2.0 * rows * F * d),
         "combine": ("hbm", Nd + S * Td + Td),
         "combine_bwd": ("hbm", Td + 2 * Nd),
         "router_bwd": ("hbm", Td + 2 * T * E * 4),
-        "dgrad_h": ("tensor", 2.0 * rows * d * F),
-        "dgrad_x": ("tensor", 2.0 * rows * F * d * g),
-        "wgrad_w1": ("tensor", 2.0 * rows * F * d * g),
-        "wgrad_w2": ("tensor", 2.0 * rows * d * F),
+        "dgrad_h": (mm, 2.0 * rows * d * F),
+        "dgrad_x": (mm, 2.0 * rows * F * d * g),
+        "wgrad_w1": (mm, 2.0 * rows * F * d * g),
+        "wgrad_w2": (mm, 2.0 * rows * d * F),
         "undispatch": ("hbm", Nd + S * Td + Td),
     }
 
@@ -379,10 +395,10 @@ def run_ours(args):
     phases = {}
     for name, ms in phase_ms.items():
         bound, amount = work[name]
-        if bound == "tensor":
+        if bound in ("tensor", "alu"):
             ach = amount / (ms * 1e-3) / 1e12
-            phases[name] = {"ms": ms, "bound": bound, "achieved_tflops": ach,
-                            "frac": ach / bf16_tf}
+            peak = bf16_tf if bound == "tensor" else FP32_FMA_TFLOPS
+            phases[name] = {"ms": ms, "bound": bound, "achieved_tflops": ach, "frac": ach / peak}
         else:
             ach = amount / (ms * 1e-3) / 1e9
             phases[name] = {"ms": ms, "bound": bound, "achieved_gbs": ach, "frac": ach / hbm_gbs}
@@ -393,6 +409,11 @@ def run_ours(args):
         roof = {"kernel": top, "bound": "tensor", "achieved": ach, "peak": bf16_tf,
                 "unit": "TFLOP/s", "frac": ach / bf16_tf, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
+    elif tb == "alu":
+        ach = tw / (top_ms_live * 1e-3) / 1e12
+        roof = {"kernel": top, "bound": "alu", "achieved": ach, "peak": FP32_FMA_TFLOPS,
+                "unit": "TFLOP/s", "frac": ach / FP32_FMA_TFLOPS, "traffic": traffic,
+                "peak_source": "derived: 148 SMs x 128 FP32 FMA lanes x 2 x 1965 MHz"}
     else:
         ach = tw / (top_ms_live * 1e-3) / 1e9
         roof = {"kernel": top, "bound": "hbm", "achieved": ach, "peak": hbm_gbs, "unit": "GB/s",
