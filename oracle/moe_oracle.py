@@ -202,11 +202,42 @@ def expert_backward(X, U, V, H, dO, W1e, W3e, W2e, act: int):
     return dX, dW1, dW3, dW2
 
 
+# ----------------------------------------------------------------------------- load balancing
+
+def aux_loss(logits, counts, k: int, coef: float) -> float:
+    """Auxiliary load-balancing loss.
+
+    Ch.4 "分布式训练": section "框架" (DeepSpeed config: `loss_coef`, the load-balancing loss
+    coefficient), section "实践" part 四 (model config `aux_loss_factor`) and part 七.3 (the
+    auxiliary loss should sit near 0 with experts chosen evenly).  The pages give no formula.
+    Reading: coef * E * sum_e f_e * P_e, with f_e = counts[e] / (T k) the share of the T k
+    assignments routed to expert e (before the capacity drop) and P_e the mean over tokens of
+    the full softmax probability of e.  At a perfectly even routing with uniform probabilities
+    it equals coef, so with the pages' small coefficients it stays near 0; it grows to coef * E
+    when every token goes to one expert with certainty.
+    """
+    T, E = logits.shape
+    f = np.asarray(counts, dtype=np.float64) / (T * k)
+    P = softmax(logits).mean(axis=0)
+    return float(coef * E * np.sum(f * P))
+
+
+def aux_loss_grad(logits, counts, k: int, coef: float) -> np.ndarray:
+    """dL_aux / dlogits.  f is piecewise constant in the logits (no gradient through the
+    selection); dP_e / dl[t, :] = (1/T) p_t * (onehot_e - p_t), so
+    dl[t] = coef * E / T * p_t * (f - <p_t, f>)."""
+    T, E = logits.shape
+    f = np.asarray(counts, dtype=np.float64) / (T * k)
+    p = softmax(logits)
+    return coef * E / T * p * (f[None, :] - (p @ f)[:, None])
+
+
 # ----------------------------------------------------------------------------- whole layer
 
 def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
                   capacity_factor, n_shared: int = 0, identity_experts: bool = False,
-                  idx_override: np.ndarray | None = None, capacity_override=None):
+                  idx_override: np.ndarray | None = None, capacity_override=None,
+                  aux_loss_coef: float = 0.0):
     """Forward of the layer: route, dispatch under capacity, run experts, combine.
 
     Combine (Ch.4 "专家并行" 二 step 4: results return and sequence order is restored):
@@ -218,6 +249,7 @@ def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
     idx_override: route with these expert ids instead of re-selecting (used to compare against a
     device whose logits differ from the oracle's inside a near-tie).
     capacity_override: an explicit capacity C instead of the one the capacity factor gives.
+    aux_loss_coef: weight of the load-balancing loss (aux_loss); 0 leaves it out.
     """
     T, d = x.shape
     E = Wg.shape[0]
@@ -249,9 +281,10 @@ def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
             U, V, H, O = expert_forward(x, W1[e], None if W3 is None else W3[e], W2[e], act)
         y = y + O
         cache[e] = (np.arange(T), None, x, U, V, H, O)
+    aux = aux_loss(logits, counts, k, aux_loss_coef) if aux_loss_coef else 0.0
     return {"logits": logits, "idx": idx, "g": g, "C": C, "counts": counts, "kept": kept,
             "pos": pos, "y": y, "cache": cache, "k": k, "act": act, "gate_norm": gate_norm,
-            "E": E, "n_shared": n_shared}
+            "E": E, "n_shared": n_shared, "aux_loss": aux, "aux_loss_coef": aux_loss_coef}
 
 
 def router_backward(logits, idx, g, dg, gate_norm: int):
@@ -275,7 +308,8 @@ def router_backward(logits, idx, g, dg, gate_norm: int):
 
 
 def layer_backward(fwd: dict, x, Wg, W1, W3, W2, dy):
-    """Backward of the layer for the scalar L = <y, dy>.
+    """Backward of the layer for the scalar L = <y, dy> (+ the load-balancing loss when the
+    forward had a coefficient).
 
     Ch.4 "专家并行与数据并行的结合" 三.3: gradients are routed back to the experts, whose weight
     gradients are computed locally; the router and the token rows receive theirs on the way back.
@@ -303,6 +337,8 @@ def layer_backward(fwd: dict, x, Wg, W1, W3, W2, dy):
         if dW3 is not None:
             dW3[e] = dW3e
     dl = router_backward(fwd["logits"], idx, g, dg, fwd["gate_norm"])
+    if fwd.get("aux_loss_coef"):
+        dl = dl + aux_loss_grad(fwd["logits"], fwd["counts"], k, fwd["aux_loss_coef"])
     dWg = dl.T @ x
     dx = dx + dl @ Wg
     return {"dx": dx, "dWg": dWg, "dW1": dW1, "dW3": dW3, "dW2": dW2, "dg": dg, "dlogits": dl}

@@ -92,7 +92,7 @@ def pin_activation_derivatives():
 
 
 def _tiny_layer(seed, *, T=8, d=4, E=3, k=2, F=5, act=mo.GELU, gate_norm=0, cf=0.75,
-                n_shared=0, bias=True, min_gap=1e-3):
+                n_shared=0, bias=True, min_gap=1e-3, aux=0.0):
     """Random float64 layer whose top-k sets sit at least min_gap from a logit tie."""
     rng = np.random.default_rng(seed)
     for _ in range(1000):
@@ -109,14 +109,15 @@ def _tiny_layer(seed, *, T=8, d=4, E=3, k=2, F=5, act=mo.GELU, gate_norm=0, cf=0
         W2 = rng.standard_normal((Et, d, F)) / math.sqrt(F)
         dy = rng.standard_normal((T, d))
         return dict(x=x, Wg=Wg, bias=b, W1=W1, W3=W3, W2=W2, dy=dy,
-                    kw=dict(k=k, act=act, gate_norm=gate_norm, capacity_factor=cf, n_shared=n_shared))
+                    kw=dict(k=k, act=act, gate_norm=gate_norm, capacity_factor=cf, n_shared=n_shared,
+                            aux_loss_coef=aux))
     raise RuntimeError("no tie-free draw")
 
 
 def _loss(p, **over):
     q = {**p, **over}
     f = mo.layer_forward(q["x"], q["Wg"], q["bias"], q["W1"], q["W3"], q["W2"], **p["kw"])
-    return float(np.sum(f["y"] * p["dy"]))
+    return float(np.sum(f["y"] * p["dy"])) + f["aux_loss"]
 
 
 def pin_backward_fd(p, h=1e-6, tol=1e-6):
@@ -143,6 +144,9 @@ FD_CASES = {
     "swiglu_shared": dict(seed=2, act=mo.SWIGLU, gate_norm=0, cf=1.0, n_shared=1),
     "swiglu_renorm_dropless": dict(seed=3, act=mo.SWIGLU, gate_norm=1, cf=None),
     "gelu_top1": dict(seed=4, act=mo.GELU, gate_norm=0, k=1, cf=1.0),
+    # the load-balancing loss added to <y, dy>: its gradient reaches dx and dWg through dlogits
+    "gelu_aux_drops": dict(seed=5, act=mo.GELU, gate_norm=0, cf=0.75, aux=0.3),
+    "swiglu_renorm_aux": dict(seed=6, act=mo.SWIGLU, gate_norm=1, cf=None, n_shared=1, aux=0.3),
 }
 
 
@@ -266,6 +270,48 @@ def test_backward_matches_finite_differences(case):
     assert pin_backward_fd(p)
 
 
+def pin_aux_loss_closed_forms():
+    """Closed forms of the load-balancing loss: an even routing with uniform probabilities gives
+    coef; every token sent to one expert with (numerically) certain probability gives coef * E;
+    E = 2 reduces to coef * 2 * (f0 * mean sigmoid(l0 - l1) + f1 * mean sigmoid(l1 - l0))."""
+    coef, T, E, k = 0.7, 12, 4, 2
+    ok = math.isclose(mo.aux_loss(np.zeros((T, E)), np.full(E, T * k // E), k, coef), coef,
+                      rel_tol=1e-15)
+    L = np.zeros((T, E)); L[:, 0] = 200.0
+    ok &= math.isclose(mo.aux_loss(L, np.array([T, 0, 0, 0]), 1, coef), coef * E, rel_tol=1e-12)
+    rng = np.random.default_rng(11)
+    L2 = rng.standard_normal((T, 2))
+    cnt = np.array([7, 5])
+    p0 = expit(L2[:, 0] - L2[:, 1])
+    want = coef * 2 * (7 / T * p0.mean() + 5 / T * (1 - p0).mean())
+    ok &= math.isclose(mo.aux_loss(L2, cnt, 1, coef), want, rel_tol=1e-12)
+    return bool(ok)
+
+
+def pin_aux_grad_fd(h=1e-6):
+    """The gradient of the load-balancing loss against central differences of the loss itself
+    (counts held fixed: they do not depend continuously on the logits)."""
+    rng = np.random.default_rng(12)
+    T, E, k, coef = 6, 5, 2, 0.4
+    L = rng.standard_normal((T, E))
+    cnt = rng.integers(0, 5, size=E)
+    g = mo.aux_loss_grad(L, cnt, k, coef)
+    fd = np.zeros_like(L)
+    for i in np.ndindex(L.shape):
+        a = L.copy(); a[i] += h
+        b = L.copy(); b[i] -= h
+        fd[i] = (mo.aux_loss(a, cnt, k, coef) - mo.aux_loss(b, cnt, k, coef)) / (2 * h)
+    return bool(np.max(np.abs(fd - g)) <= 1e-8)
+
+
+def test_aux_loss_closed_forms():
+    assert pin_aux_loss_closed_forms()
+
+
+def test_aux_loss_gradient_matches_finite_differences():
+    assert pin_aux_grad_fd()
+
+
 def test_sampled_forms_equal_full_layer():
     from mixture_experts_layer_23_b200.configs import LayerShape, SWIGLU as SW
     from mixture_experts_layer_23_b200.synth import make_inputs, to_f64
@@ -353,6 +399,31 @@ def test_planted_choice_major_drop_order_is_caught(monkeypatch):
         return counts, kept, pos
     _planted(monkeypatch, "dispatch", wrong)
     assert not pin_dispatch_brute()
+
+
+def test_planted_aux_loss_without_expert_count_is_caught(monkeypatch):
+    def wrong(logits, counts, k, coef):                  # forgets the factor E
+        T, E = logits.shape
+        f = np.asarray(counts, dtype=np.float64) / (T * k)
+        return float(coef * np.sum(f * mo.softmax(logits).mean(axis=0)))
+    _planted(monkeypatch, "aux_loss", wrong)
+    assert not pin_aux_loss_closed_forms()
+
+
+def test_planted_aux_grad_missing_centering_is_caught(monkeypatch):
+    def wrong(logits, counts, k, coef):                  # drops the -<p, f> term
+        T, E = logits.shape
+        f = np.asarray(counts, dtype=np.float64) / (T * k)
+        return coef * E / T * mo.softmax(logits) * f[None, :]
+    _planted(monkeypatch, "aux_loss_grad", wrong)
+    assert not pin_aux_grad_fd()
+
+
+def test_planted_aux_grad_left_out_of_backward_is_caught(monkeypatch):
+    _planted(monkeypatch, "aux_loss_grad", lambda logits, counts, k, coef: np.zeros(logits.shape))
+    c = dict(FD_CASES["gelu_aux_drops"])
+    p = _tiny_layer(c.pop("seed"), **c)
+    assert not pin_backward_fd(p)
 
 
 def test_planted_dropped_term_in_dx_is_caught(monkeypatch):
