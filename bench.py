@@ -78,6 +78,8 @@ def parse():
     ap.add_argument("--workload", default="gpt2_gshard")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--aux-loss-coef", type=float, default=0.0,
+                    help="also compute the load-balancing loss (and its gradient) with this weight")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -258,7 +260,7 @@ def phase_work(shape, n_kept):
     Td, Nd = T * d * b, n_kept * d * b
     return {
         "router": ("hbm", Td + E * d * b + T * E * 4 + T * k * 8),
-        "dispatch": ("hbm", Td + Nd + T * k * 8),
+        "dispatch": ("hbm", Td + Nd + T * k * 8 + (T * E * 4 if shape.aux_loss_coef else 0)),
         "expert_up": (mm, 2.0 * rows * d * F * g),
         "expert_down": (mm, 2.0 * rows * F * d),
         "combine": ("hbm", Nd + S * Td + Td),
@@ -292,6 +294,9 @@ def run_ours(args):
     from mixture_experts_layer_23_b200.synth import make_inputs
 
     shape = BY_NAME[args.workload]
+    if args.aux_loss_coef:
+        from dataclasses import replace
+        shape = replace(shape, aux_loss_coef=args.aux_loss_coef)
     inp = make_inputs(shape, 0)
     w = {n: to_device(inp[n], shape, dev) for n in ("Wg", "W1", "W3", "W2")}
     bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
@@ -458,6 +463,7 @@ def run_ours(args):
         "config": {"workload": WORKLOAD_TEXT[shape.name], "name": shape.name, "T": shape.T,
                    "d": shape.d, "E": shape.E, "k": shape.k, "d_ff": shape.d_ff,
                    "n_shared": shape.n_shared, "kept_assignments": n_kept,
+                   "aux_loss_coef": shape.aux_loss_coef,
                    "gemm_engine": ["cuda_core", "tcgen05"][moe.gemm_engine(layer.cfg)],
                    "l2": "flushed between timed steps (256 MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},

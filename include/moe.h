@@ -75,6 +75,11 @@ typedef struct {
                               MOE_DROPLESS: no limit;  otherwise C itself */
   int32_t dtype;           /* MOE_DTYPE_F32 | MOE_DTYPE_BF16 */
   int32_t has_bias;        /* bias[E] (a constant logit offset, no gradient) is read when 1 */
+  float aux_loss_coef;     /* >= 0, finite: weight of the auxiliary load-balancing loss
+                              coef * E * sum_e (counts[e] / (T k)) * mean_t softmax(logits_t)[e]
+                              (Ch.4 "框架" DeepSpeed loss_coef; "实践" 四 aux_loss_factor; the
+                              pages give no formula, this is the reading taken).  0: the forward
+                              does not compute it and the backward adds no gradient for it. */
 } moe_config_t;
 
 /* Sizes and the layout of the forward context (state saved for the backward pass).
@@ -89,6 +94,8 @@ typedef struct {
       ctx_row_token, ctx_Xd, ctx_Gu, ctx_Gv, ctx_H, ctx_O;
   size_t ctx_bytes;       /* total ctx size */
   size_t scratch_bytes;   /* total scratch size (forward and backward) */
+  size_t ctx_aux_loss;    /* one float: the load-balancing loss of the last forward (written
+                             only when aux_loss_coef > 0) */
 } moe_layout_t;
 
 /* Validate a config and report the workspace sizes / ctx layout.  Host only, no CUDA calls. */
@@ -153,6 +160,16 @@ moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x
  * A gather in a fixed order: deterministic, no atomics. */
 moe_status moe_combine(const moe_config_t* cfg, const void* O, const int32_t* slot,
                        const float* topk_w, void* y, moe_stream_t stream);
+
+/* The auxiliary load-balancing loss from float logits [T,E] and counts [E] (the demand per
+ * expert before the capacity drop, as moe_dispatch reports it): loss[0] = aux_loss_coef * E *
+ * sum_e (counts[e] / (T k)) * P_e, P_e the mean over tokens of softmax(logits_t)[e] over all E
+ * (whatever gate_norm is).  Fixed-order reductions: bitwise reproducible.  Uses the scratch
+ * buffer of moe_get_layout.  moe_layer_fwd computes the same into ctx when aux_loss_coef > 0,
+ * and moe_layer_bwd then adds its gradient, aux_loss_coef * E / T * p_t * (f - <p_t, f>), to
+ * the router's logit gradient. */
+moe_status moe_aux_loss(const moe_config_t* cfg, const float* logits, const int32_t* counts,
+                        float* loss, void* scratch, moe_stream_t stream);
 
 /* Whole forward: steps 1-4.  ctx (moe_layout_t.ctx_bytes) receives the saved state; y [T,d]. */
 moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,

@@ -37,6 +37,7 @@ class LayerShape:
     dtype: int = BF16
     bias: str = "none"        # synthetic per-expert logit offset: "none" | "zipf" | "normal"
     fwd_only: bool = False
+    aux_loss_coef: float = 0.0   # weight of the load-balancing loss (0: not computed)
 
     @property
     def E_tot(self) -> int:

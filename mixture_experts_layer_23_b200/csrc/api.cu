@@ -53,6 +53,7 @@ moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
   if (c.gate_norm != 0 && c.gate_norm != 1) return MOE_ERR_INVALID_ARG;
   if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
   if (c.has_bias != 0 && c.has_bias != 1) return MOE_ERR_INVALID_ARG;
+  if (!(c.aux_loss_coef >= 0.f) || !isfinite(c.aux_loss_coef)) return MOE_ERR_INVALID_ARG;
   if (c.k > 8 || c.E > 256 || c.n_shared > 8 || c.T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
   const int vec = (c.dtype == MOE_DTYPE_BF16) ? 8 : 4;
   if (c.d % vec != 0 || c.d_ff % vec != 0) return MOE_ERR_UNSUPPORTED;
@@ -94,6 +95,9 @@ moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
     if (chunks < 1) chunks = 1;
     D.n_tchunk = chunks;
   }
+  D.aux_coef = c.aux_loss_coef;
+  D.n_aux = (D.T + kAuxTokensPerChunk - 1) / kAuxTokensPerChunk;
+  if (D.n_aux > kAuxMaxChunks) D.n_aux = kAuxMaxChunks;
   *out = D;
   return MOE_OK;
 }
@@ -119,6 +123,7 @@ ScratchLayout scratch_layout(const Dims& D) {
     S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
     S.dxg = take(T * D.d * 2);
   }
+  S.aux_part = take((size_t)D.n_aux * D.E * 4);
   S.total = off;
   return S;
 }
@@ -146,6 +151,7 @@ moe_status ctx_layout(const Dims& D, moe_layout_t* L) {
   L->ctx_Gv = (D.act == MOE_ACT_SWIGLU) ? take(R * D.F * D.elem) : 0;
   L->ctx_H = take(R * D.F * D.elem);
   L->ctx_O = take(R * D.d * D.elem);
+  L->ctx_aux_loss = take(4);
   L->ctx_bytes = off;
   L->scratch_bytes = scratch_layout(D).total;
   return MOE_OK;
@@ -271,6 +277,16 @@ moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, con
   return launch_route(D, x, Wg, bias, logits, topk_idx, topk_w, nullptr, (cudaStream_t)stream);
 }
 
+moe_status moe_aux_loss(const moe_config_t* cfg, const float* logits, const int32_t* counts,
+                        float* loss, void* scratch, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({logits, counts, loss, scratch}));
+  const ScratchLayout S = scratch_layout(D);
+  return launch_aux_loss(D, logits, counts, (float*)((char*)scratch + S.aux_part), loss,
+                         (cudaStream_t)stream);
+}
+
 moe_status moe_route_from_logits(const moe_config_t* cfg, const float* logits, int32_t* topk_idx,
                                  float* topk_w, moe_stream_t stream) {
   Dims D;
@@ -344,6 +360,9 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   MOE_TRY(mark_fwd(1, st));
   MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
                           (int32_t*)(s + S.blk_counts), st));
+  if (D.aux_coef > 0.f)
+    MOE_TRY(launch_aux_loss(D, logits, counts, (float*)(s + S.aux_part), (float*)(c + L.ctx_aux_loss),
+                            st));
   MOE_TRY(mark_fwd(2, st));
   MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, (uint32_t*)(s + S.status), st,
                      /*phase_marks=*/true));
@@ -390,7 +409,9 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   // from a bf16 copy of dlogits; otherwise CUDA-core kernels read the fp32 dlogits
   const bool rtc = S.dl16 != 0;
   __nv_bfloat16* dl16 = rtc ? (__nv_bfloat16*)(s + S.dl16) : nullptr;
-  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, dg, dl, dl16, dO, st));
+  const int32_t* counts = (const int32_t*)(c + L.ctx_counts);
+  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, counts, dg, dl, dl16,
+                             dO, st));
   MOE_TRY(mark_bwd(1, st));
   if (rtc) {
     int n_chunks = 0;

@@ -83,15 +83,52 @@ combine_fwd_kernel(const T* __restrict__ O, const int32_t* __restrict__ slot,
 // dg[0..k-1] (0 at dropped assignments):
 //   gate_norm 0: p = softmax(l), dp[e] = sum_j [idx_j = e] dg_j, dl = p * (dp - <p, dp>)
 //   gate_norm 1: w = topk_w, dl[idx_j] = w_j * (dg_j - <w, dg>), 0 elsewhere
-// No gradient flows through the chosen indices.  Writes the E floats of dl, and when out16 is
-// given also their bf16 copy with the row padded by zeros to E8 entries.
+// No gradient flows through the chosen indices.  With aux_scale = coef * E / T > 0 the gradient
+// of the load-balancing loss, aux_scale * p * (f - <p, f>) with p the full softmax of the row and
+// f_e = counts[e] * inv_Tk, is added.  Writes the E floats of dl, and when out16 is given also
+// their bf16 copy with the row padded by zeros to E8 entries.
 __device__ __forceinline__ void dlogits_row(const float* __restrict__ lrow, const int (&e)[8],
                                             const float (&w)[8], const float (&g)[8], int E,
                                             int k, int gate_norm, float* __restrict__ out,
-                                            __nv_bfloat16* __restrict__ out16, int E8) {
+                                            __nv_bfloat16* __restrict__ out16, int E8,
+                                            const int32_t* __restrict__ counts, float aux_scale,
+                                            float inv_Tk) {
   const int lane = threadIdx.x & 31;
   if (out16 != nullptr)
     for (int ee = E + lane; ee < E8; ee += 32) out16[ee] = __float2bfloat16_rn(0.f);
+  float extra[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) extra[i] = 0.f;
+  if (aux_scale > 0.f) {
+    float p[8], f[8];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = lane + 32 * i;
+      p[i] = (ee < E) ? lrow[ee] : -INFINITY;
+      f[i] = (ee < E) ? (float)counts[ee] * inv_Tk : 0.f;
+      m = fmaxf(m, p[i]);
+    }
+    m = warp_max(m);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = lane + 32 * i;
+      p[i] = (ee < E) ? expf(p[i] - m) : 0.f;
+      s += p[i];
+    }
+    s = warp_sum(s);
+    const float inv = 1.f / s;
+    float pf = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      p[i] *= inv;
+      pf += p[i] * f[i];
+    }
+    pf = warp_sum(pf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) extra[i] = aux_scale * p[i] * (f[i] - pf);
+  }
   if (gate_norm == 0) {
     float l[8];
     float m = -INFINITY;
@@ -131,7 +168,7 @@ __device__ __forceinline__ void dlogits_row(const float* __restrict__ lrow, cons
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (j < k && e[j] == ee) dp += g[j];
-        const float v = l[i] * (dp - dot);
+        const float v = l[i] * (dp - dot) + extra[i];
         out[ee] = v;
         if (out16 != nullptr) out16[ee] = __float2bfloat16_rn(v);
       }
@@ -141,11 +178,15 @@ __device__ __forceinline__ void dlogits_row(const float* __restrict__ lrow, cons
 #pragma unroll
     for (int j = 0; j < 8; ++j)
       if (j < k) wd += w[j] * g[j];
-    for (int ee = lane; ee < E; ee += 32) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int ee = lane + 32 * i;
+      if (ee >= E) break;
       float v = 0.f;
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         if (j < k && e[j] == ee) v = w[j] * (g[j] - wd);
+      v += extra[i];
       out[ee] = v;
       if (out16 != nullptr) out16[ee] = __float2bfloat16_rn(v);
     }
@@ -157,7 +198,8 @@ __global__ void __launch_bounds__(256, 4)
 combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                    const int32_t* __restrict__ slot, const float* __restrict__ topk_w,
                    const int32_t* __restrict__ topk_idx, const float* __restrict__ logits,
-                   const int32_t* __restrict__ kept, const int32_t* __restrict__ offsets, int T_,
+                   const int32_t* __restrict__ kept, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ counts, float aux_scale, float inv_Tk, int T_,
                    int d, int E, int k, int gate_norm, int n_tok_blocks, float* __restrict__ dg,
                    float* __restrict__ dlogits, __nv_bfloat16* __restrict__ dl16, int E8,
                    T* __restrict__ dO) {
@@ -234,7 +276,7 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
     dg[(int64_t)t * k + lane] = mine;
   }
   dlogits_row(logits + (int64_t)t * E, ej, w, part, E, k, gate_norm, dlogits + (int64_t)t * E,
-              dl16 ? dl16 + (int64_t)t * E8 : nullptr, E8);
+              dl16 ? dl16 + (int64_t)t * E8 : nullptr, E8, counts, aux_scale, inv_Tk);
 }
 
 }  // namespace
@@ -273,40 +315,43 @@ template <typename T, int KS>
 static moe_status combine_bwd_t(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                                 const float* topk_w, const int32_t* topk_idx,
                                 const float* logits, const int32_t* kept, const int32_t* offsets,
-                                float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
-                                cudaStream_t st) {
+                                const int32_t* counts, float* dg, float* dlogits,
+                                __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
   const int n_tok_blocks = (D.T + 7) / 8;
   return launch_k(combine_bwd_kernel<T, KS>, n_tok_blocks + D.E, 256, 0, st, 1, (const T*)dy,
-                  (const T*)O, slot, topk_w, topk_idx, logits, kept, offsets, D.T, D.d, D.E, D.k,
+                  (const T*)O, slot, topk_w, topk_idx, logits, kept, offsets, counts,
+                  D.aux_coef > 0.f ? D.aux_coef * (float)D.E / (float)D.T : 0.f,
+                  1.f / ((float)D.T * (float)D.k), D.T, D.d, D.E, D.k,
                   D.gate_norm, n_tok_blocks, dg, dlogits, dl16, (int)round_up(D.E, 8), (T*)dO);
 }
 template <typename T>
 static moe_status combine_bwd_ks(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                                  const float* topk_w, const int32_t* topk_idx,
                                  const float* logits, const int32_t* kept,
-                                 const int32_t* offsets, float* dg, float* dlogits,
-                                 __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
+                                 const int32_t* offsets, const int32_t* counts, float* dg,
+                                 float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
   switch (pow2_at_least(D.k)) {
     case 1: case 2:
-      return combine_bwd_t<T, 2>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
-                                 dlogits, dl16, dO, st);
+      return combine_bwd_t<T, 2>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
+                                 counts, dg, dlogits, dl16, dO, st);
     case 4:
-      return combine_bwd_t<T, 4>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
-                                 dlogits, dl16, dO, st);
+      return combine_bwd_t<T, 4>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
+                                 counts, dg, dlogits, dl16, dO, st);
     default:
-      return combine_bwd_t<T, 8>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
-                                 dlogits, dl16, dO, st);
+      return combine_bwd_t<T, 8>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
+                                 counts, dg, dlogits, dl16, dO, st);
   }
 }
 
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
-                              const int32_t* kept, const int32_t* offsets, float* dg,
-                              float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
+                              const int32_t* kept, const int32_t* offsets, const int32_t* counts,
+                              float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
+                              cudaStream_t st) {
   if (D.dtype == MOE_DTYPE_BF16)
     return combine_bwd_ks<__nv_bfloat16>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
-                                         dg, dlogits, dl16, dO, st);
-  return combine_bwd_ks<float>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, dg,
+                                         counts, dg, dlogits, dl16, dO, st);
+  return combine_bwd_ks<float>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, counts, dg,
                                dlogits, dl16, dO, st);
 }
 

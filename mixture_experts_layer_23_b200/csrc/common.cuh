@@ -29,6 +29,7 @@ struct ScratchLayout {
   size_t dWg_part;      // [n_tchunk, E, d] float
   size_t dl16;          // [T, E8] bf16 copy of dlogits (tensor-core router backward), or 0
   size_t dxg;           // [T, d] bf16 dl Wg (tensor-core router backward), or 0
+  size_t aux_part;      // [n_aux, E] float partial probability sums of the load-balancing loss
   size_t total;
 };
 
@@ -40,9 +41,13 @@ struct Dims {
   int elem;             // bytes per activation element
   int n_blk;            // dispatch blocks
   int n_tchunk;         // token chunks of the router-weight gradient (two-level reduction)
+  float aux_coef;       // weight of the load-balancing loss (0: off)
+  int n_aux;            // token chunks of the load-balancing loss's probability sums
 };
 
 constexpr int kDispatchTokensPerBlock = 256;
+constexpr int kAuxTokensPerChunk = 64;   // load-balancing loss: tokens per CTA of the first level
+constexpr int kAuxMaxChunks = 296;       // and at most this many CTAs (more tokens per CTA)
 
 __host__ __device__ inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 

@@ -20,11 +20,15 @@ moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, con
                           void* y, cudaStream_t st);
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
-                              const int32_t* kept, const int32_t* offsets, float* dg,
-                              float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st);
+                              const int32_t* kept, const int32_t* offsets, const int32_t* counts,
+                              float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
+                              cudaStream_t st);
 // Router backward on the tensor cores (bf16, d a multiple of 64): dWg partials over token
 // chunks, their fixed-order sum, dl Wg, and the un-dispatch gather that adds it.
 bool router_bwd_tc_supported(const Dims& D);
+// Load-balancing loss (forward): loss[0] from the logits and the pre-drop counts.
+moe_status launch_aux_loss(const Dims& D, const float* logits, const int32_t* counts, float* part,
+                           float* loss, cudaStream_t st);
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
                                   float* part, int* n_chunks, uint32_t* status, cudaStream_t st);
 moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,

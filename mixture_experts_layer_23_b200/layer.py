@@ -72,6 +72,7 @@ class MoELayer:
             "Gv": (L.ctx_Gv, self.dt, (R, s.d_ff)),
             "H": (L.ctx_H, self.dt, (R, s.d_ff)),
             "O": (L.ctx_O, self.dt, (R, s.d)),
+            "aux_loss": (L.ctx_aux_loss, torch.float32, (1,)),
         }
         off, dt, shp = table[name]
         return self._view(off, dt, shp)

@@ -24,7 +24,7 @@ EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_bwd",
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
            "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
-           "moe_last_cuda_error")
+           "moe_last_cuda_error", "moe_aux_loss")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -45,7 +45,8 @@ class Config(ctypes.Structure):
                 ("k", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("n_shared", ctypes.c_int32),
                 ("act", ctypes.c_int32), ("gate_norm", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("capacity", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("has_bias", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("has_bias", ctypes.c_int32),
+                ("aux_loss_coef", ctypes.c_float)]
 
 
 class Layout(ctypes.Structure):
@@ -54,7 +55,7 @@ class Layout(ctypes.Structure):
         (n, ctypes.c_size_t) for n in (
             "ctx_logits", "ctx_topk_idx", "ctx_topk_w", "ctx_counts", "ctx_kept", "ctx_offsets",
             "ctx_slot", "ctx_row_token", "ctx_Xd", "ctx_Gu", "ctx_Gv", "ctx_H", "ctx_O",
-            "ctx_bytes", "scratch_bytes")]
+            "ctx_bytes", "scratch_bytes", "ctx_aux_loss")]
 
 
 def _load():
@@ -69,6 +70,7 @@ def _load():
         "moe_workspace_size": [CP, ctypes.POINTER(SZ), ctypes.POINTER(SZ)],
         "moe_route": [CP, P, P, P, P, P, P, P],
         "moe_route_from_logits": [CP, P, P, P, P],
+        "moe_aux_loss": [CP, P, P, P, P, P],
         "moe_dispatch": [CP, P, P, P, P, P, P, P, P, P, P],
         "moe_dispatch_noalloc": [CP, P, P, P, P, P, P, P, P, P],
         "moe_expert_ffn": [CP, P, P, P, P, P, P, P, P, P, P, P, P],
@@ -114,7 +116,8 @@ def make_config(shape: LayerShape, capacity: int | None = None) -> Config:
     return Config(T=shape.T, d=shape.d, E=shape.E, k=shape.k, d_ff=shape.d_ff,
                   n_shared=shape.n_shared, act=shape.act, gate_norm=shape.gate_norm,
                   capacity_factor=0.0 if shape.dropless else float(shape.capacity_factor),
-                  capacity=capacity, dtype=shape.dtype, has_bias=int(shape.bias != "none"))
+                  capacity=capacity, dtype=shape.dtype, has_bias=int(shape.bias != "none"),
+                  aux_loss_coef=float(shape.aux_loss_coef))
 
 
 def _p(t):
@@ -166,6 +169,11 @@ def gemm_engine(cfg: Config) -> int:
 def route(cfg, x, Wg, bias, logits, topk_idx, topk_w, stream=None):
     _check(_lib.moe_route(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(logits), _p(topk_idx),
                           _p(topk_w), _stream(stream)), "moe_route")
+
+
+def aux_loss(cfg, logits, counts, loss, scratch, stream=None):
+    _check(_lib.moe_aux_loss(ctypes.byref(cfg), _p(logits), _p(counts), _p(loss), _p(scratch),
+                             _stream(stream)), "moe_aux_loss")
 
 
 def route_from_logits(cfg, logits, topk_idx, topk_w, stream=None):

@@ -63,6 +63,8 @@ def run_gpu(shape: LayerShape, inp: dict, *, capacity=None, backward=True):
     out["Xd_bits"] = layer.view("Xd").contiguous().view(
         __import__("torch").int16 if shape.dtype == BF16 else __import__("torch").int32).cpu().numpy()
     out["y"] = act_to_np(layer.y)
+    if shape.aux_loss_coef:
+        out["aux_loss"] = float(layer.view("aux_loss").cpu().numpy()[0])
     out["C"] = layer.L.capacity
     out["routed_row0"] = layer.L.routed_row0
     out["rows"] = layer.L.rows
@@ -147,10 +149,16 @@ def full_compare(shape: LayerShape, seed=0, *, inp=None, capacity=None):
     check_dispatch(shape, gpu, gidx, x_bits_of(shape, inp), C)
     f = mo.layer_forward(x, Wg, inp["bias"], W1, W3, W2, k=shape.k, act=shape.act,
                          gate_norm=shape.gate_norm, capacity_factor=shape.capacity_factor,
-                         n_shared=shape.n_shared, idx_override=gidx, capacity_override=C)
+                         n_shared=shape.n_shared, idx_override=gidx, capacity_override=C,
+                         aux_loss_coef=shape.aux_loss_coef)
     rel = tol_for(shape)
     errs = {"topk_w": assert_close("topk_w", gpu["topk_w"], f["g"], rel),
             "y": assert_close("y", gpu["y"], f["y"], rel)}
+    if shape.aux_loss_coef:
+        # a scalar from fp32 softmax sums of fp32 logits: relative 1e-5
+        want = f["aux_loss"]
+        assert abs(gpu["aux_loss"] - want) <= 1e-5 * abs(want), (gpu["aux_loss"], want)
+        errs["aux_loss"] = abs(gpu["aux_loss"] - want)
     if not shape.fwd_only:
         dy = to_f64(inp["dy"], dt)
         g = mo.layer_backward(f, x, Wg, W1, W3, W2, dy)

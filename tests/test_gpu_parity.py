@@ -97,6 +97,43 @@ def test_edge_shapes(shape):
     _parity().full_compare(shape, seed=3)
 
 
+AUX = [
+    # load-balancing loss on: its value, and its gradient through dlogits into dx and dWg
+    LayerShape("aux_gelu_drops", T=700, d=64, E=8, k=2, d_ff=96, capacity_factor=0.9,
+               dtype=BF16, bias="zipf", aux_loss_coef=0.05),
+    LayerShape("aux_swiglu_renorm_shared", T=333, d=128, E=12, k=3, d_ff=64, n_shared=1,
+               gate_norm=1, act=SWIGLU, capacity_factor=None, dtype=BF16, aux_loss_coef=0.5),
+    LayerShape("aux_many_experts_tc", T=520, d=192, E=72, k=6, d_ff=128, capacity_factor=1.25,
+               act=SWIGLU, dtype=BF16, bias="normal", aux_loss_coef=0.01),
+    LayerShape("aux_fp32", T=150, d=48, E=5, k=2, d_ff=40, capacity_factor=1.0, dtype=FP32,
+               aux_loss_coef=1.0),
+]
+
+
+@pytest.mark.parametrize("shape", AUX, ids=lambda s: s.name)
+def test_aux_loss_layers_match_oracle(shape):
+    _parity().full_compare(shape, seed=5)
+
+
+def test_aux_loss_entry_point_matches_the_layer():
+    """moe_aux_loss on the layer's own logits and counts reproduces the forward's value bitwise."""
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import MoELayer, to_device
+    shape = AUX[0]
+    inp = make_inputs(shape, 7)
+    dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
+    bias = torch.from_numpy(inp["bias"]).cuda()
+    layer = MoELayer(shape)
+    layer.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"])
+    loss = torch.zeros(4, dtype=torch.float32, device="cuda")
+    scratch = torch.zeros(layer.L.scratch_bytes, dtype=torch.uint8, device="cuda")
+    moe.aux_loss(layer.cfg, layer.view("logits"), layer.view("counts"), loss, scratch)
+    torch.cuda.synchronize()
+    assert loss[0].item() == layer.view("aux_loss")[0].item()
+    assert layer.status() == moe.MOE_OK
+
+
 def test_zero_capacity_drops_everything():
     s = LayerShape("cap0", T=100, d=32, E=4, k=2, d_ff=32, n_shared=1, dtype=FP32)
     gpu, _ = _parity().full_compare(s, seed=1, capacity=0)

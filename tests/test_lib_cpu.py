@@ -84,6 +84,26 @@ def test_bad_capacity_factor_rejected(moe):
     assert moe.lib().moe_get_layout(ctypes.byref(cfg), ctypes.byref(L)) == 1
 
 
+@pytest.mark.parametrize("coef", [-0.5, float("nan"), float("inf")])
+def test_bad_aux_loss_coef_rejected(moe, coef):
+    s = LayerShape("t", T=64, d=64, E=4, k=2, d_ff=64, dtype=BF16)
+    cfg = moe.make_config(s)
+    cfg.aux_loss_coef = coef
+    L = moe.Layout()
+    assert moe.lib().moe_get_layout(ctypes.byref(cfg), ctypes.byref(L)) == 1
+
+
+def test_aux_loss_layout_and_argument_checks(moe):
+    s = LayerShape("t", T=300, d=64, E=6, k=2, d_ff=64, dtype=BF16, aux_loss_coef=0.01)
+    cfg = moe.make_config(s)
+    L = moe.get_layout(cfg)
+    assert L.ctx_aux_loss % 256 == 0 and L.ctx_aux_loss + 4 <= L.ctx_bytes
+    lib = moe.lib()
+    good = 0x10000
+    assert lib.moe_aux_loss(ctypes.byref(cfg), good, good, None, good, None) == 1
+    assert lib.moe_aux_loss(ctypes.byref(cfg), good, good + 4, good, good, None) == 3
+
+
 def test_pointer_checks_happen_before_any_cuda_call(moe):
     s = LayerShape("t", T=64, d=64, E=4, k=2, d_ff=64, dtype=BF16)
     cfg = moe.make_config(s)
