@@ -14,14 +14,17 @@ def topk_brute(row, k):
     return [e for _, e in sorted(((-v, e) for e, v in enumerate(row)))][:k]
 
 
-def dispatch_brute(idx_rows, E, C):
-    """For each expert, list its tokens in token order, then cut the list at C.
+def dispatch_brute(idx_rows, E, C, choice_major=False):
+    """For each expert, list its assignments in priority order -- token order, or with
+    choice_major by (choice index, token) -- then cut the list at C.
 
     Returns (counts, kept, pos) with pos[t][j] = -1 for dropped assignments."""
     per_expert = [[] for _ in range(E)]
     for t, row in enumerate(idx_rows):
         for j, e in enumerate(row):
             per_expert[e].append((t, j))
+    if choice_major:
+        per_expert = [sorted(lst, key=lambda tj: (tj[1], tj[0])) for lst in per_expert]
     pos = [[-1] * len(row) for row in idx_rows]
     counts = [len(lst) for lst in per_expert]
     kept = []

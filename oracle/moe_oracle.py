@@ -104,7 +104,7 @@ def capacity(capacity_factor, k: int, T: int, E: int):
     return int(math.ceil(cf * k * T / E))
 
 
-def dispatch(idx: np.ndarray, E: int, C):
+def dispatch(idx: np.ndarray, E: int, C, choice_major: bool = False):
     """Rank each expert's assignments by token index and keep rank < C.
 
     Ch.4 "All-to-All 通信模式" 二: device i sends subset S_ik of its tokens to the device of
@@ -113,19 +113,24 @@ def dispatch(idx: np.ndarray, E: int, C):
     assignments are ordered by token index (a token chooses an expert at most once, so this is
     a total order); the first C are kept.
 
+    choice_major (a routing variant; FSMoE summary: several routing functions): all first
+    choices in token order, then all second choices, and so on, so a token's j-th choice is only
+    dropped after every token's earlier choices at that expert were placed.
+
     Returns counts[e] (demand before the drop), kept[e] = min(counts[e], C) and pos[t, j] (the
     rank of assignment (t, j) within its expert, -1 when dropped).
     """
     T, k = idx.shape
     counts = np.zeros(E, dtype=np.int64)
     pos = np.full((T, k), -1, dtype=np.int64)
-    for t in range(T):                       # token order
-        for j in range(k):
-            e = idx[t, j]
-            r = counts[e]
-            counts[e] += 1
-            if C is None or r < C:
-                pos[t, j] = r
+    order = ([(t, j) for j in range(k) for t in range(T)] if choice_major
+             else [(t, j) for t in range(T) for j in range(k)])   # token order
+    for t, j in order:
+        e = idx[t, j]
+        r = counts[e]
+        counts[e] += 1
+        if C is None or r < C:
+            pos[t, j] = r
     kept = counts.copy() if C is None else np.minimum(counts, C)
     return counts, kept, pos
 
@@ -237,7 +242,7 @@ def aux_loss_grad(logits, counts, k: int, coef: float) -> np.ndarray:
 def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
                   capacity_factor, n_shared: int = 0, identity_experts: bool = False,
                   idx_override: np.ndarray | None = None, capacity_override=None,
-                  aux_loss_coef: float = 0.0):
+                  aux_loss_coef: float = 0.0, choice_major: bool = False):
     """Forward of the layer: route, dispatch under capacity, run experts, combine.
 
     Combine (Ch.4 "专家并行" 二 step 4: results return and sequence order is restored):
@@ -250,6 +255,7 @@ def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
     device whose logits differ from the oracle's inside a near-tie).
     capacity_override: an explicit capacity C instead of the one the capacity factor gives.
     aux_loss_coef: weight of the load-balancing loss (aux_loss); 0 leaves it out.
+    choice_major: the drop priority of dispatch (default: token order).
     """
     T, d = x.shape
     E = Wg.shape[0]
@@ -257,7 +263,7 @@ def layer_forward(x, Wg, bias, W1, W3, W2, *, k: int, act: int, gate_norm: int,
     idx = select_topk(logits, k) if idx_override is None else np.asarray(idx_override, np.int64)
     g = gate_weights(logits, idx, gate_norm)
     C = capacity(capacity_factor, k, T, E) if capacity_override is None else capacity_override
-    counts, kept, pos = dispatch(idx, E, C)
+    counts, kept, pos = dispatch(idx, E, C, choice_major)
     y = np.zeros((T, d))
     cache = {}
     for e in range(E):
@@ -349,7 +355,7 @@ def layer_backward(fwd: dict, x, Wg, W1, W3, W2, dy):
 # whole on the CPU.  Each is the full-layer formula evaluated on a subset; nothing is
 # approximated.
 
-def route(x, Wg, bias, *, k, gate_norm, capacity_factor):
+def route(x, Wg, bias, *, k, gate_norm, capacity_factor, choice_major=False):
     """Router + dispatch for all tokens (cheap: T*d*E multiply-adds)."""
     T = x.shape[0]
     E = Wg.shape[0]
@@ -357,7 +363,7 @@ def route(x, Wg, bias, *, k, gate_norm, capacity_factor):
     idx = select_topk(logits, k)
     g = gate_weights(logits, idx, gate_norm)
     C = capacity(capacity_factor, k, T, E)
-    counts, kept, pos = dispatch(idx, E, C)
+    counts, kept, pos = dispatch(idx, E, C, choice_major)
     return {"logits": logits, "idx": idx, "g": g, "C": C, "counts": counts, "kept": kept, "pos": pos}
 
 

@@ -53,22 +53,50 @@ def pin_dispatch_brute(seed=0):
         L = rng.standard_normal((T, E)) + np.linspace(0, 1.5, E)[None, :]
         idx = mo.select_topk(L, k)
         C = mo.capacity(cf, k, T, E)
-        counts, kept, pos = mo.dispatch(idx, E, C)
-        bc, bk, bp = brute.dispatch_brute(idx.tolist(), E, C)
-        if list(counts) != bc or list(kept) != bk or pos.tolist() != bp:
-            return False
+        for cm in (False, True):
+            counts, kept, pos = mo.dispatch(idx, E, C, choice_major=cm)
+            bc, bk, bp = brute.dispatch_brute(idx.tolist(), E, C, choice_major=cm)
+            if list(counts) != bc or list(kept) != bk or pos.tolist() != bp:
+                return False
     return True
 
 
-def pin_hand_dispatch():
-    g = _golden("hand_dispatch.json")
+def pin_hand_dispatch(name="hand_dispatch.json"):
+    g = _golden(name)
     L = np.array(g["logits"])
     idx = mo.select_topk(L, g["k"])
     C = mo.capacity(g["capacity_factor"], g["k"], g["T"], g["E"])
-    counts, kept, pos = mo.dispatch(idx, g["E"], C)
+    counts, kept, pos = mo.dispatch(idx, g["E"], C, choice_major=g.get("choice_major", False))
     ex = g["expect"]
     return (C == ex["C"] and idx.tolist() == ex["idx"] and counts.tolist() == ex["counts"]
             and kept.tolist() == ex["kept"] and pos.tolist() == ex["pos"])
+
+
+def pin_choice_major_priority(seed=3):
+    """Choice-major invariant: at every expert, once a choice index j has a dropped assignment,
+    no assignment with a later choice index is kept; and the kept counts equal token order's."""
+    rng = np.random.default_rng(seed)
+    for T, E, k, cf in [(60, 4, 2, 0.7), (45, 6, 3, 0.5), (33, 3, 3, 1.0)]:
+        idx = mo.select_topk(rng.standard_normal((T, E)), k)
+        C = mo.capacity(cf, k, T, E)
+        counts, kept, pos = mo.dispatch(idx, E, C, choice_major=True)
+        c0, k0, _ = mo.dispatch(idx, E, C)
+        if not (np.array_equal(counts, c0) and np.array_equal(kept, k0)):
+            return False
+        for e in range(E):
+            worst_kept = -1
+            best_dropped = k
+            for t in range(T):
+                for j in range(k):
+                    if idx[t, j] != e:
+                        continue
+                    if pos[t, j] >= 0:
+                        worst_kept = max(worst_kept, j)
+                    else:
+                        best_dropped = min(best_dropped, j)
+            if worst_kept > best_dropped:
+                return False
+    return True
 
 
 def pin_gelu_values():
@@ -166,6 +194,14 @@ def test_dispatch_matches_brute_force():
 
 def test_hand_worked_dispatch():
     assert pin_hand_dispatch()
+
+
+def test_hand_worked_choice_major_dispatch():
+    assert pin_hand_dispatch("hand_dispatch_choice_major.json")
+
+
+def test_choice_major_priority_invariant():
+    assert pin_choice_major_priority()
 
 
 def test_gelu_silu_values():
@@ -385,7 +421,7 @@ def test_planted_tie_toward_higher_index_is_caught(monkeypatch):
 
 
 def test_planted_choice_major_drop_order_is_caught(monkeypatch):
-    def wrong(idx, E, C):                                # all first choices before second choices
+    def wrong(idx, E, C, choice_major=False):            # always all first choices first
         T, k = idx.shape
         counts = np.zeros(E, dtype=np.int64)
         pos = np.full((T, k), -1, dtype=np.int64)
