@@ -80,6 +80,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--aux-loss-coef", type=float, default=0.0,
                     help="also compute the load-balancing loss (and its gradient) with this weight")
+    ap.add_argument("--choice-major", action="store_true",
+                    help="drop priority: all first choices, then second choices, ... (else token order)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -294,9 +296,9 @@ def run_ours(args):
     from mixture_experts_layer_23_b200.synth import make_inputs
 
     shape = BY_NAME[args.workload]
-    if args.aux_loss_coef:
+    if args.aux_loss_coef or args.choice_major:
         from dataclasses import replace
-        shape = replace(shape, aux_loss_coef=args.aux_loss_coef)
+        shape = replace(shape, aux_loss_coef=args.aux_loss_coef, choice_major=args.choice_major)
     inp = make_inputs(shape, 0)
     w = {n: to_device(inp[n], shape, dev) for n in ("Wg", "W1", "W3", "W2")}
     bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).to(dev)
@@ -464,6 +466,7 @@ def run_ours(args):
                    "d": shape.d, "E": shape.E, "k": shape.k, "d_ff": shape.d_ff,
                    "n_shared": shape.n_shared, "kept_assignments": n_kept,
                    "aux_loss_coef": shape.aux_loss_coef,
+                   "drop_order": "choice-major" if shape.choice_major else "token",
                    "gemm_engine": ["cuda_core", "tcgen05"][moe.gemm_engine(layer.cfg)],
                    "l2": "flushed between timed steps (256 MiB write outside the timed events)",
                    "parallelism": f"replicas x{world}"},

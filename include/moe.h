@@ -80,6 +80,10 @@ typedef struct {
                               (Ch.4 "框架" DeepSpeed loss_coef; "实践" 四 aux_loss_factor; the
                               pages give no formula, this is the reading taken).  0: the forward
                               does not compute it and the backward adds no gradient for it. */
+  int32_t drop_order;      /* capacity drop priority within an expert.  0: token order (position
+                              priority, "drop by token order");  1: choice-major -- all first
+                              choices in token order, then all second choices, ... (a routing
+                              variant; the FSMoE summary names several routing functions) */
 } moe_config_t;
 
 /* Sizes and the layout of the forward context (state saved for the backward pass).
@@ -115,7 +119,8 @@ moe_status moe_route_from_logits(const moe_config_t* cfg, const float* logits, i
                                  float* topk_w, moe_stream_t stream);
 
 /* Step 2, capacity-limited dispatch.  For each expert its assignments are ranked by token
- * index; rank < C is kept (position priority, "drop by token order").
+ * index (drop_order 0; drop_order 1: by choice index, then token index); rank < C is kept
+ * (position priority, "drop by token order").
  * Outputs: counts[E] demand before the drop; kept[E] = min(counts, C); offsets[E+1] first row
  * of each routed segment (offsets[E] = end); slot[T,k] row of each assignment or -1 if
  * dropped; row_token[R] token of each row (-1 for padding and shared rows); Xd[R,d] rows of x

@@ -38,6 +38,7 @@ class LayerShape:
     bias: str = "none"        # synthetic per-expert logit offset: "none" | "zipf" | "normal"
     fwd_only: bool = False
     aux_loss_coef: float = 0.0   # weight of the load-balancing loss (0: not computed)
+    choice_major: bool = False   # drop priority: all first choices, then second, ... (else token order)
 
     @property
     def E_tot(self) -> int:

@@ -54,6 +54,7 @@ moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
   if (c.dtype != MOE_DTYPE_F32 && c.dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
   if (c.has_bias != 0 && c.has_bias != 1) return MOE_ERR_INVALID_ARG;
   if (!(c.aux_loss_coef >= 0.f) || !isfinite(c.aux_loss_coef)) return MOE_ERR_INVALID_ARG;
+  if (c.drop_order != 0 && c.drop_order != 1) return MOE_ERR_INVALID_ARG;
   if (c.k > 8 || c.E > 256 || c.n_shared > 8 || c.T > (1 << 24)) return MOE_ERR_UNSUPPORTED;
   const int vec = (c.dtype == MOE_DTYPE_BF16) ? 8 : 4;
   if (c.d % vec != 0 || c.d_ff % vec != 0) return MOE_ERR_UNSUPPORTED;
@@ -96,6 +97,8 @@ moe_status resolve_dims(const moe_config_t* cfg, Dims* out) {
     D.n_tchunk = chunks;
   }
   D.aux_coef = c.aux_loss_coef;
+  D.choice_major = c.drop_order;
+  D.n_layers = c.drop_order ? c.k : 1;
   D.n_aux = (D.T + kAuxTokensPerChunk - 1) / kAuxTokensPerChunk;
   if (D.n_aux > kAuxMaxChunks) D.n_aux = kAuxMaxChunks;
   *out = D;
@@ -108,7 +111,7 @@ ScratchLayout scratch_layout(const Dims& D) {
   auto take = [&](size_t bytes) { const size_t o = off; off = align256(off + bytes); return o; };
   const size_t R = (size_t)D.R, T = (size_t)D.T;
   S.status = take(256);
-  S.blk_counts = take((size_t)D.n_blk * D.E * 4);
+  S.blk_counts = take((size_t)D.n_blk * D.n_layers * D.E * 4);
   S.local_rank = 0;  // the dispatch keeps local ranks in the slot array
   S.groups = take((size_t)D.E_tot * 16);
   S.dO = take(R * D.d * D.elem);

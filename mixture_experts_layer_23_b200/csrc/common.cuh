@@ -42,6 +42,8 @@ struct Dims {
   int n_blk;            // dispatch blocks
   int n_tchunk;         // token chunks of the router-weight gradient (two-level reduction)
   float aux_coef;       // weight of the load-balancing loss (0: off)
+  int choice_major;     // dispatch drop priority: 0 token order, 1 choice index then token
+  int n_layers;         // histogram layers of the dispatch: k when choice-major, else 1
   int n_aux;            // token chunks of the load-balancing loss's probability sums
 };
 

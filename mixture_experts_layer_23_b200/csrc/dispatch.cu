@@ -11,9 +11,12 @@
 //   1. rank:    each CTA takes 256 tokens; per warp, a shared-memory bitmask per expert marks the
 //               lanes (tokens) that chose it, so a popcount of the lower lanes gives each
 //               assignment's rank inside the warp; warp bases make it a rank inside the CTA.
-//               The CTA's per-expert histogram goes to scratch.
+//               The CTA's per-expert histogram goes to scratch.  Choice-major priority
+//               (drop_order 1) repeats this per choice index j: k histogram layers, and each
+//               assignment's rank inside its CTA's layer.
 //   2. scatter: every CTA scans the histograms (exclusive over rank CTAs in token order, per
-//               expert) for its bases, kept = min(counts, C) and the 128-row aligned offsets;
+//               expert; choice-major: over layers first, then rank CTAs) for its bases,
+//               kept = min(counts, C) and the 128-row aligned offsets;
 //               then one warp per token finalises its slots and copies its x row (16-byte
 //               vectors, read once, written to each kept slot); extra CTAs zero padding rows.
 #include <mutex>
@@ -26,6 +29,7 @@ namespace {
 constexpr int DT = kDispatchTokensPerBlock;  // 256 tokens = 8 warps x 32 lanes
 static_assert(DT == 256, "rank kernel assumes 8 warps of 32 tokens");
 
+template <bool CM>
 __global__ void __launch_bounds__(256)
 dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
                      int32_t* __restrict__ blk_counts, int32_t* __restrict__ local_rank) {
@@ -33,34 +37,36 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
   __shared__ uint32_t mask[8][256];
   __shared__ int32_t wbase[8][256];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  for (int i = tid; i < 8 * 256; i += 256) (&mask[0][0])[i] = 0u;
-  __syncthreads();
   const int t = blockIdx.x * DT + tid;
   int e_of[8];
-  if (t < T_) {
-    for (int j = 0; j < k; ++j) {
-      e_of[j] = topk_idx[(int64_t)t * k + j];
-      if ((unsigned)e_of[j] < (unsigned)E) atomicOr(&mask[warp][e_of[j]], 1u << lane);
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < E; e += 256) {
-    int run = 0;
+  if (t < T_)
+    for (int j = 0; j < k; ++j) e_of[j] = topk_idx[(int64_t)t * k + j];
+  const uint32_t below = (1u << lane) - 1u;
+  // token order: one pass over all choices; choice-major: one pass (layer) per choice index
+  for (int layer = 0; layer < (CM ? k : 1); ++layer) {
+    for (int i = tid; i < 8 * 256; i += 256) (&mask[0][0])[i] = 0u;
+    __syncthreads();
+    if (t < T_)
+      for (int j = CM ? layer : 0; j < (CM ? layer + 1 : k); ++j)
+        if ((unsigned)e_of[j] < (unsigned)E) atomicOr(&mask[warp][e_of[j]], 1u << lane);
+    __syncthreads();
+    for (int e = tid; e < E; e += 256) {
+      int run = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      wbase[w][e] = run;
-      run += __popc(mask[w][e]);
+      for (int w = 0; w < 8; ++w) {
+        wbase[w][e] = run;
+        run += __popc(mask[w][e]);
+      }
+      blk_counts[((int64_t)blockIdx.x * (CM ? k : 1) + layer) * E + e] = run;
     }
-    blk_counts[(int64_t)blockIdx.x * E + e] = run;
-  }
-  __syncthreads();
-  if (t < T_) {
-    const uint32_t below = (1u << lane) - 1u;
-    for (int j = 0; j < k; ++j) {
-      const int e = e_of[j];
-      local_rank[(int64_t)t * k + j] =
-          ((unsigned)e < (unsigned)E) ? wbase[warp][e] + __popc(mask[warp][e] & below) : 0;
-    }
+    __syncthreads();
+    if (t < T_)
+      for (int j = CM ? layer : 0; j < (CM ? layer + 1 : k); ++j) {
+        const int e = e_of[j];
+        local_rank[(int64_t)t * k + j] =
+            ((unsigned)e < (unsigned)E) ? wbase[warp][e] + __popc(mask[warp][e] & below) : 0;
+      }
+    __syncthreads();   // wbase and mask are reused by the next layer
   }
 }
 
@@ -74,7 +80,7 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
 constexpr int SC_TOK = 8;   // tokens per scatter CTA (one per warp)
 static_assert(DT % SC_TOK == 0, "a scatter CTA must not straddle two rank CTAs");
 
-template <typename T>
+template <typename T, bool CM>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
                         const int32_t* __restrict__ blk_counts, int n_blk, int T_, int d, int E,
@@ -84,7 +90,7 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
                         int32_t* __restrict__ slot /* in: local rank, out: slot */,
                         int32_t* __restrict__ row_token, T* __restrict__ Xd) {
   pdl_prologue();
-  __shared__ int32_t s_base[256];   // base of this CTA's rank block, per expert
+  __shared__ int32_t s_base[8 * 256];   // base of this CTA's rank block per (layer,) expert
   __shared__ int32_t s_kept[256];
   __shared__ int32_t s_off[257];
   constexpr int VN = Vec16<T>::N;
@@ -92,14 +98,16 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool tok_cta = (int)blockIdx.x < n_tok_blocks;
   const int my_blk = tok_cta ? (int)(blockIdx.x * SC_TOK / DT) : 0;
+  const int L = CM ? k : 1;
   for (int e = threadIdx.x; e < E; e += 256) {
-    int run = 0, base = 0;
-    for (int b = 0; b < n_blk; ++b) {
-      if (b == my_blk) base = run;
-      run += blk_counts[(int64_t)b * E + e];
+    int run = 0;
+    for (int layer = 0; layer < L; ++layer) {   // layers in priority order, then rank CTAs
+      for (int b = 0; b < n_blk; ++b) {
+        if (b == my_blk) s_base[layer * 256 + e] = run;
+        run += blk_counts[((int64_t)b * L + layer) * E + e];
+      }
     }
     const int kp = (int64_t)run < C ? run : (int)C;
-    s_base[e] = base;
     s_kept[e] = kp;
     s_off[e + 1] = (int)round_up(kp, MOE_ROW_ALIGN);
     if (blockIdx.x == 0) {
@@ -150,7 +158,7 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
     if (lane < k) {
       const int e = topk_idx[(int64_t)t * k + lane];
       const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
-      const int pos = valid ? s_base[e] + slot[(int64_t)t * k + lane] : 0;
+      const int pos = valid ? s_base[(CM ? lane : 0) * 256 + e] + slot[(int64_t)t * k + lane] : 0;
       if (valid && (int64_t)pos < C) {
         my_slot = s_off[e] + pos;
         row_token[my_slot] = t;
@@ -173,22 +181,35 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
 
 }  // namespace
 
-moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
-                           int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
-                           void* Xd, int32_t* blk_counts, cudaStream_t st) {
-  MOE_TRY_S(launch_k(dispatch_rank_kernel, D.n_blk, 256, 0, st, 1, topk_idx, D.T, D.E, D.k,
+template <typename T, bool CM>
+static moe_status dispatch_t(const Dims& D, const void* x, const int32_t* topk_idx,
+                             int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
+                             int32_t* row_token, void* Xd, int32_t* blk_counts, cudaStream_t st) {
+  MOE_TRY_S(launch_k(dispatch_rank_kernel<CM>, D.n_blk, 256, 0, st, 1, topk_idx, D.T, D.E, D.k,
                      blk_counts, slot));
   const int n_tok_blocks = (D.T + SC_TOK - 1) / SC_TOK;
   const int grid = n_tok_blocks + D.E + 1;
-  if (D.dtype == MOE_DTYPE_BF16)
-    return launch_k(dispatch_scatter_kernel<__nv_bfloat16>, grid, 256, 0, st, 1,
-                    (const __nv_bfloat16*)x, topk_idx, (const int32_t*)blk_counts, D.n_blk, D.T,
-                    D.d, D.E, D.k, D.C, (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0,
-                    counts, kept, offsets, slot, row_token, (__nv_bfloat16*)Xd);
-  return launch_k(dispatch_scatter_kernel<float>, grid, 256, 0, st, 1, (const float*)x, topk_idx,
+  return launch_k(dispatch_scatter_kernel<T, CM>, grid, 256, 0, st, 1, (const T*)x, topk_idx,
                   (const int32_t*)blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
                   (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets,
-                  slot, row_token, (float*)Xd);
+                  slot, row_token, (T*)Xd);
+}
+
+moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
+                           int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                           void* Xd, int32_t* blk_counts, cudaStream_t st) {
+  if (D.dtype == MOE_DTYPE_BF16) {
+    if (D.choice_major)
+      return dispatch_t<__nv_bfloat16, true>(D, x, topk_idx, counts, kept, offsets, slot,
+                                             row_token, Xd, blk_counts, st);
+    return dispatch_t<__nv_bfloat16, false>(D, x, topk_idx, counts, kept, offsets, slot,
+                                            row_token, Xd, blk_counts, st);
+  }
+  if (D.choice_major)
+    return dispatch_t<float, true>(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
+                                   blk_counts, st);
+  return dispatch_t<float, false>(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
+                                  blk_counts, st);
 }
 
 // ----------------------------------------------------------------------------- no-allocation form
@@ -200,7 +221,8 @@ moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx
 // race; it keeps the last call's contents, and needs no clearing because the rank kernel writes
 // every entry a call reads before the scan reads it.
 
-constexpr int kNoAllocMaxHistogram = 1 << 16;  // int32 entries: ceil(T / 256) * E must fit
+constexpr int kNoAllocMaxHistogram = 1 << 16;  // int32 entries: ceil(T / 256) * E (* k when
+                                               // choice-major) must fit
 static __device__ __align__(256) int32_t g_noalloc_histogram[kNoAllocMaxHistogram];
 
 // Device address of the array on the current device, looked up once per device (with that device
@@ -236,7 +258,8 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config_t* cfg, const void* 
     if (!p) return MOE_ERR_INVALID_ARG;
     if (((uintptr_t)p & 15u) != 0) return MOE_ERR_MISALIGNED;
   }
-  if ((int64_t)D.n_blk * D.E > moe::kNoAllocMaxHistogram) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if ((int64_t)D.n_blk * D.n_layers * D.E > moe::kNoAllocMaxHistogram)
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
   int32_t* hist = nullptr;
   const moe_status h = moe::noalloc_histogram(&hist);
   if (h != MOE_OK) return h;

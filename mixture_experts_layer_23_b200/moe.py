@@ -46,7 +46,7 @@ class Config(ctypes.Structure):
                 ("act", ctypes.c_int32), ("gate_norm", ctypes.c_int32),
                 ("capacity_factor", ctypes.c_float), ("capacity", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("has_bias", ctypes.c_int32),
-                ("aux_loss_coef", ctypes.c_float)]
+                ("aux_loss_coef", ctypes.c_float), ("drop_order", ctypes.c_int32)]
 
 
 class Layout(ctypes.Structure):
@@ -117,7 +117,7 @@ def make_config(shape: LayerShape, capacity: int | None = None) -> Config:
                   n_shared=shape.n_shared, act=shape.act, gate_norm=shape.gate_norm,
                   capacity_factor=0.0 if shape.dropless else float(shape.capacity_factor),
                   capacity=capacity, dtype=shape.dtype, has_bias=int(shape.bias != "none"),
-                  aux_loss_coef=float(shape.aux_loss_coef))
+                  aux_loss_coef=float(shape.aux_loss_coef), drop_order=int(shape.choice_major))
 
 
 def _p(t):

@@ -98,7 +98,7 @@ def check_routing(shape: LayerShape, gpu: dict, ol: np.ndarray):
 def check_dispatch(shape: LayerShape, gpu: dict, gidx: np.ndarray, x_bits: np.ndarray, C):
     """counts, kept, slot map and drop mask bit-exact against the oracle's dispatch of the same
     expert ids; the dispatched buffer holds exact copies of the token rows, padding rows zero."""
-    counts, kept, pos = mo.dispatch(gidx, shape.E, C)
+    counts, kept, pos = mo.dispatch(gidx, shape.E, C, choice_major=shape.choice_major)
     assert np.array_equal(gpu["counts"], counts)
     assert np.array_equal(gpu["kept"], kept)
     off = gpu["offsets"].astype(np.int64)
@@ -150,7 +150,7 @@ def full_compare(shape: LayerShape, seed=0, *, inp=None, capacity=None):
     f = mo.layer_forward(x, Wg, inp["bias"], W1, W3, W2, k=shape.k, act=shape.act,
                          gate_norm=shape.gate_norm, capacity_factor=shape.capacity_factor,
                          n_shared=shape.n_shared, idx_override=gidx, capacity_override=C,
-                         aux_loss_coef=shape.aux_loss_coef)
+                         aux_loss_coef=shape.aux_loss_coef, choice_major=shape.choice_major)
     rel = tol_for(shape)
     errs = {"topk_w": assert_close("topk_w", gpu["topk_w"], f["g"], rel),
             "y": assert_close("y", gpu["y"], f["y"], rel)}
@@ -181,13 +181,14 @@ def sampled_compare(shape: LayerShape, seed=0, n_tok=24, n_f=3, experts=None):
     W3 = None if inp["W3"] is None else LazyF64(inp["W3"], dt)
     dy = None if shape.fwd_only else to_f64(inp["dy"], dt)
     r = mo.route(x, Wg, inp["bias"], k=shape.k, gate_norm=shape.gate_norm,
-                 capacity_factor=shape.capacity_factor)
+                 capacity_factor=shape.capacity_factor, choice_major=shape.choice_major)
     gidx = check_routing(shape, gpu, r["logits"])
     check_dispatch(shape, gpu, gidx, x_bits_of(shape, inp), r["C"])
     # downstream comparisons use the GPU's expert ids (identical unless a near-tie flipped)
     r["idx"] = gidx
     r["g"] = mo.gate_weights(r["logits"], gidx, shape.gate_norm)
-    r["counts"], r["kept"], r["pos"] = mo.dispatch(gidx, shape.E, r["C"])
+    r["counts"], r["kept"], r["pos"] = mo.dispatch(gidx, shape.E, r["C"],
+                                                   choice_major=shape.choice_major)
     rel = tol_for(shape)
     assert_close("topk_w", gpu["topk_w"], r["g"], rel)
     rng = np.random.default_rng(seed + 1)
@@ -213,6 +214,10 @@ def sampled_compare(shape: LayerShape, seed=0, n_tok=24, n_f=3, experts=None):
         assert_close(f"dW2[{e}][:,fs]", gpu["dW2"][e][:, fs], c, rel)
         if b is not None:
             assert_close(f"dW3[{e}][fs]", gpu["dW3"][e][fs], b, rel)
+    # each token's logit gradient sums to zero over E, so the columns of dWg do too; on the bf16
+    # path the logit gradient is rounded to bf16 before the router-backward GEMMs (2^-9 relative
+    # per element), which the looser bf16 bound absorbs
     colsum = gpu["dWg"].sum(axis=0)
-    assert np.max(np.abs(colsum)) <= 1e-3 * np.max(np.abs(gpu["dWg"])) * np.sqrt(shape.E)
+    bound = (1e-2 if shape.dtype == BF16 else 1e-3) * np.max(np.abs(gpu["dWg"])) * np.sqrt(shape.E)
+    assert np.max(np.abs(colsum)) <= bound, (np.max(np.abs(colsum)), bound)
     return gpu

@@ -134,6 +134,30 @@ def test_aux_loss_entry_point_matches_the_layer():
     assert layer.status() == moe.MOE_OK
 
 
+CHOICE_MAJOR = [
+    # choice-major drop priority (all first choices before any second choice) with drops: the
+    # slot map must match the oracle's bit for bit
+    LayerShape("cm_gelu_tc", T=1500, d=128, E=8, k=2, d_ff=128, capacity_factor=0.6,
+               dtype=BF16, bias="zipf", choice_major=True),
+    LayerShape("cm_swiglu_shared_k6", T=900, d=64, E=24, k=6, d_ff=64, n_shared=1,
+               act=SWIGLU, capacity_factor=0.8, dtype=BF16, bias="normal", choice_major=True),
+    LayerShape("cm_fp32_k3", T=301, d=36, E=5, k=3, d_ff=20, capacity_factor=0.7, dtype=FP32,
+               choice_major=True, aux_loss_coef=0.2),
+]
+
+
+@pytest.mark.parametrize("shape", CHOICE_MAJOR, ids=lambda s: s.name)
+def test_choice_major_layers_match_oracle(shape):
+    gpu, _ = _parity().full_compare(shape, seed=6)
+    assert np.any(gpu["slot"] < 0), "the case must drop assignments"
+
+
+def test_choice_major_full_size_sampled():
+    from dataclasses import replace
+    from mixture_experts_layer_23_b200.configs import BY_NAME
+    _parity().sampled_compare(replace(BY_NAME["bert_large_skew"], choice_major=True), seed=0)
+
+
 def test_zero_capacity_drops_everything():
     s = LayerShape("cap0", T=100, d=32, E=4, k=2, d_ff=32, n_shared=1, dtype=FP32)
     gpu, _ = _parity().full_compare(s, seed=1, capacity=0)

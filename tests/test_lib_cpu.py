@@ -93,6 +93,22 @@ def test_bad_aux_loss_coef_rejected(moe, coef):
     assert moe.lib().moe_get_layout(ctypes.byref(cfg), ctypes.byref(L)) == 1
 
 
+def test_bad_drop_order_rejected(moe):
+    s = LayerShape("t", T=64, d=64, E=4, k=2, d_ff=64, dtype=BF16)
+    cfg = moe.make_config(s)
+    cfg.drop_order = 2
+    L = moe.Layout()
+    assert moe.lib().moe_get_layout(ctypes.byref(cfg), ctypes.byref(L)) == 1
+
+
+def test_choice_major_scratch_holds_k_histogram_layers(moe):
+    base = LayerShape("t", T=1000, d=64, E=16, k=4, d_ff=64, dtype=BF16)
+    from dataclasses import replace
+    a = moe.get_layout(moe.make_config(base)).scratch_bytes
+    b = moe.get_layout(moe.make_config(replace(base, choice_major=True))).scratch_bytes
+    assert b >= a + 3 * 4 * 16 * 4 - 256   # (k - 1) more layers of ceil(T/256) x E int32
+
+
 def test_aux_loss_layout_and_argument_checks(moe):
     s = LayerShape("t", T=300, d=64, E=6, k=2, d_ff=64, dtype=BF16, aux_loss_coef=0.01)
     cfg = moe.make_config(s)
