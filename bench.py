@@ -45,11 +45,11 @@ GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wg
 GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "act_fast.cuh", "common.cuh"]
 NCU_TRAFFIC = {
     # python bench.py --steps 1 --warmup 1 --no-cpu-baseline under ncu --set full, one launch of
-    # the up-projection GEMM: dram__bytes_read.sum 89.720064 MB + dram__bytes_write.sum 60.959232 MB
+    # the up-projection GEMM: dram__bytes_read.sum 89.732096 MB + dram__bytes_write.sum 60.708352 MB
     ("gpt2_gshard", "expert_up"): {
-        "bytes": 150679296,
+        "bytes": 150440448,
         "sources": GEMM_SOURCES,
-        "sha256": "be35e948941c8af985dc6e69584e6d6f598b5d6a7bc4e2d7e29029765e893ecd",
+        "sha256": "b7412286015775b8673a67b6a41166523ba9cc5be06084b44510b77b574f82bb",
         "profile": "profiles/expert_up_gpt2_gshard.md",
     },
 }
@@ -456,6 +456,36 @@ def run_ours(args):
     barrier()
     e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)))
 
+    # forward-only layers: the one-launch fused forward (moe_layer_fwd_fused), where it applies
+    fused = None
+    if dy is None:
+        yf = torch.empty_like(layer.y)
+
+        def fused_step():
+            moe.layer_fwd_fused(layer.cfg, x, w["Wg"], bias, w["W1"], w["W3"], w["W2"], yf)
+        try:
+            fused_step()
+        except moe.MoEError as err:
+            if err.status != 2:    # MOE_ERR_UNSUPPORTED: the layer is too large for it
+                raise
+        else:
+            for _ in range(args.warmup):
+                fused_step()
+                flush.zero_()
+            fs, fe = [mk() for _ in range(K)], [mk() for _ in range(K)]
+            barrier()
+            torch.cuda.synchronize(dev)
+            for i in range(K):
+                fs[i].record(stream)
+                fused_step()
+                fe[i].record(stream)
+                flush.zero_()
+            torch.cuda.synchronize(dev)
+            barrier()
+            f_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(fs, fe)))
+            fused = {"entry": "moe_layer_fwd_fused", "value": world * shape.T * K / (f_ms * 1e-3),
+                     "unit": "tokens/s", "ms_per_step": f_ms / K, "launches_per_step": 1}
+
     value = world * shape.T * K / (total_ms * 1e-3)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -472,6 +502,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world}"},
         "roofline": roof,
         "phases": phases,
+        "fused_fwd": fused,
         "phased_ms_per_step": phased_ms,
         "e2e": {"value": world * shape.T * K / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -181,6 +181,18 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
                          const float* bias, const void* W1, const void* W3, const void* W2,
                          void* y, void* ctx, void* scratch, moe_stream_t stream);
 
+/* The whole forward of a small layer in one launch, for inference (Ch.4 "框架": Tutel's fused
+ * MoE kernel; the four steps of "专家并行" 二).  Computes the same y [T,d] as moe_layer_fwd (routing,
+ * capacity drops in the configured order, experts, combine) but keeps every intermediate on chip
+ * and writes no ctx, so no backward can follow.  topk_idx [T,k], topk_w [T,k] and counts [E]
+ * receive the routing when given (all three or none).  Takes layers with T*E*d <= 2^19 whose
+ * routing state fits in shared memory, else returns MOE_ERR_UNSUPPORTED (use moe_layer_fwd);
+ * aux_loss_coef is ignored. */
+moe_status moe_layer_fwd_fused(const moe_config_t* cfg, const void* x, const void* Wg,
+                               const float* bias, const void* W1, const void* W3, const void* W2,
+                               void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                               moe_stream_t stream);
+
 /* Whole backward for upstream gradient dy [T,d], from the ctx of the matching forward.
  * dx [T,d] (activation dtype); dWg [E,d], dW1/dW3 [E_tot,F,d], dW2 [E_tot,d,F] float.
  * dW3 may be NULL for GELU.  Gradients do not flow through the chosen indices or the drops;

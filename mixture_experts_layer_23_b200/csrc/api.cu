@@ -280,6 +280,22 @@ moe_status moe_route(const moe_config_t* cfg, const void* x, const void* Wg, con
   return launch_route(D, x, Wg, bias, logits, topk_idx, topk_w, nullptr, (cudaStream_t)stream);
 }
 
+moe_status moe_layer_fwd_fused(const moe_config_t* cfg, const void* x, const void* Wg,
+                               const float* bias, const void* W1, const void* W3, const void* W2,
+                               void* y, int32_t* topk_idx, float* topk_w, int32_t* counts,
+                               moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({x, Wg, W1, W2, y}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3}));
+  if (D.has_bias) MOE_TRY(check_ptrs({bias}));
+  const bool routing = topk_idx || topk_w || counts;
+  if (routing) MOE_TRY(check_ptrs({topk_idx, topk_w, counts}));
+  if (!fused_small_supported(D)) return MOE_ERR_UNSUPPORTED;
+  return launch_fused_small_fwd(D, x, Wg, bias, W1, W3, W2, y, topk_idx, topk_w, counts,
+                                (cudaStream_t)stream);
+}
+
 moe_status moe_aux_loss(const moe_config_t* cfg, const float* logits, const int32_t* counts,
                         float* loss, void* scratch, moe_stream_t stream) {
   Dims D;

@@ -26,6 +26,12 @@ moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, cons
 // Router backward on the tensor cores (bf16, d a multiple of 64): dWg partials over token
 // chunks, their fixed-order sum, dl Wg, and the un-dispatch gather that adds it.
 bool router_bwd_tc_supported(const Dims& D);
+// One-launch forward of small layers (inference): routing recomputed per CTA, no ctx.
+bool fused_small_supported(const Dims& D);
+moe_status launch_fused_small_fwd(const Dims& D, const void* x, const void* Wg, const float* bias,
+                                  const void* W1, const void* W3, const void* W2, void* y,
+                                  int32_t* topk_idx, float* topk_w, int32_t* counts,
+                                  cudaStream_t st);
 // Load-balancing loss (forward): loss[0] from the logits and the pre-drop counts.
 moe_status launch_aux_loss(const Dims& D, const float* logits, const int32_t* counts, float* part,
                            float* loss, cudaStream_t st);

@@ -24,7 +24,7 @@ EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_bwd",
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
            "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
-           "moe_last_cuda_error", "moe_aux_loss")
+           "moe_last_cuda_error", "moe_aux_loss", "moe_layer_fwd_fused")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -71,6 +71,7 @@ def _load():
         "moe_route": [CP, P, P, P, P, P, P, P],
         "moe_route_from_logits": [CP, P, P, P, P],
         "moe_aux_loss": [CP, P, P, P, P, P],
+        "moe_layer_fwd_fused": [CP, P, P, P, P, P, P, P, P, P, P, P],
         "moe_dispatch": [CP, P, P, P, P, P, P, P, P, P, P],
         "moe_dispatch_noalloc": [CP, P, P, P, P, P, P, P, P, P],
         "moe_expert_ffn": [CP, P, P, P, P, P, P, P, P, P, P, P, P],
@@ -169,6 +170,13 @@ def gemm_engine(cfg: Config) -> int:
 def route(cfg, x, Wg, bias, logits, topk_idx, topk_w, stream=None):
     _check(_lib.moe_route(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(logits), _p(topk_idx),
                           _p(topk_w), _stream(stream)), "moe_route")
+
+
+def layer_fwd_fused(cfg, x, Wg, bias, W1, W3, W2, y, topk_idx=None, topk_w=None, counts=None,
+                    stream=None):
+    _check(_lib.moe_layer_fwd_fused(ctypes.byref(cfg), _p(x), _p(Wg), _p(bias), _p(W1), _p(W3),
+                                    _p(W2), _p(y), _p(topk_idx), _p(topk_w), _p(counts),
+                                    _stream(stream)), "moe_layer_fwd_fused")
 
 
 def aux_loss(cfg, logits, counts, loss, scratch, stream=None):

@@ -158,6 +158,57 @@ def test_choice_major_full_size_sampled():
     _parity().sampled_compare(replace(BY_NAME["bert_large_skew"], choice_major=True), seed=0)
 
 
+FUSED = [
+    # the one-launch forward: the tiny Switch layer at full size, and bf16 shapes with shared
+    # experts, drops, renormalised gates and choice-major priority
+    [l for l in LAYERS if l.name == "switch_tiny"][0],
+    LayerShape("fused_bf16_swiglu_shared", T=300, d=64, E=8, k=2, d_ff=96, n_shared=1,
+               act=SWIGLU, capacity_factor=0.8, dtype=BF16, bias="normal"),
+    LayerShape("fused_choice_major_renorm", T=500, d=32, E=6, k=3, d_ff=48, gate_norm=1,
+               capacity_factor=0.7, dtype=BF16, choice_major=True),
+]
+
+
+@pytest.mark.parametrize("shape", FUSED, ids=lambda s: s.name)
+def test_fused_small_forward_matches_oracle(shape):
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import act_dtype, to_device
+    from mixture_experts_layer_23_b200.synth import to_f64
+    from oracle import moe_oracle as mo
+    P = _parity()
+    inp = make_inputs(shape, 9)
+    dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).cuda()
+    cfg = moe.make_config(shape)
+    y = torch.empty(shape.T, shape.d, dtype=act_dtype(shape), device="cuda")
+    idx = torch.empty(shape.T, shape.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(shape.T, shape.k, dtype=torch.float32, device="cuda")
+    counts = torch.empty(shape.E, dtype=torch.int32, device="cuda")
+    moe.layer_fwd_fused(cfg, dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"], y,
+                        idx, w, counts)
+    torch.cuda.synchronize()
+    dt = shape.dtype
+    x, Wg = to_f64(inp["x"], dt), to_f64(inp["Wg"], dt)
+    W1, W3, W2 = to_f64(inp["W1"], dt), to_f64(inp["W3"], dt), to_f64(inp["W2"], dt)
+    ol = mo.gate_logits(x, Wg, inp["bias"])
+    gidx = idx.cpu().numpy().astype(np.int64)
+    oidx = mo.select_topk(ol, shape.k)
+    for t in np.nonzero(np.any(oidx != gidx, axis=1))[0]:   # only near-ties may differ
+        assert np.max(np.abs(ol[t, oidx[t]] - ol[t, gidx[t]])) <= 1e-5, t
+    C = P.oracle_capacity(shape)
+    f = mo.layer_forward(x, Wg, inp["bias"], W1, W3, W2, k=shape.k, act=shape.act,
+                         gate_norm=shape.gate_norm, capacity_factor=shape.capacity_factor,
+                         n_shared=shape.n_shared, idx_override=gidx, capacity_override=C,
+                         choice_major=shape.choice_major)
+    assert np.array_equal(counts.cpu().numpy(), f["counts"])
+    rel = P.tol_for(shape)
+    P.assert_close("topk_w", w.cpu().numpy(), f["g"], rel)
+    P.assert_close("y", P.act_to_np(y), f["y"], rel)
+    if shape.capacity_factor is not None and shape.name != "switch_tiny":
+        assert np.any(f["pos"] < 0), "the case must drop assignments"
+
+
 def test_zero_capacity_drops_everything():
     s = LayerShape("cap0", T=100, d=32, E=4, k=2, d_ff=32, n_shared=1, dtype=FP32)
     gpu, _ = _parity().full_compare(s, seed=1, capacity=0)

@@ -139,6 +139,19 @@ def test_pointer_checks_happen_before_any_cuda_call(moe):
                              good, None) == 1
 
 
+def test_fused_forward_rejects_large_layers_before_any_cuda_call(moe):
+    s = [l for l in LAYERS if l.name == "gpt2_gshard"][0]
+    cfg = moe.make_config(s)
+    good = 0x10000
+    lib = moe.lib()
+    assert lib.moe_layer_fwd_fused(ctypes.byref(cfg), good, good, None, good, None, good, good,
+                                   None, None, None, None) == 2
+    # routing outputs are all-or-none
+    t = [l for l in LAYERS if l.name == "switch_tiny"][0]
+    assert lib.moe_layer_fwd_fused(ctypes.byref(moe.make_config(t)), good, good, None, good, None,
+                                   good, good, good, None, None, None) == 1
+
+
 def test_status_strings(moe):
     for code in range(7):
         assert moe.lib().moe_status_string(code)
