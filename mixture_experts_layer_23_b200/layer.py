@@ -97,3 +97,29 @@ class MoELayer:
 
     def status(self, stream=None) -> int:
         return moe.read_status(self.scratch, stream)
+
+
+class MoEFunction(torch.autograd.Function):
+    """torch.autograd wrapper around one MoELayer: forward through moe_layer_fwd, backward through
+    moe_layer_bwd.  Convenience only: the returned y is a copy of the layer's output buffer, and
+    weight gradients (fp32 in the library) are cast to each weight's dtype, as autograd requires.
+    The logit bias is a constant (no gradient).  Usage: y = MoEFunction.apply(x, Wg, W1, W3, W2,
+    layer, bias) with W3 None for GELU layers."""
+
+    @staticmethod
+    def forward(ctx, x, Wg, W1, W3, W2, layer, bias):
+        x = x.contiguous()
+        y = layer.forward(x, Wg, bias, W1, W3, W2).clone()
+        ctx.layer = layer
+        ctx.has_w3 = W3 is not None
+        ctx.save_for_backward(x, Wg, W1, W3 if W3 is not None else x.new_empty(0), W2)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, Wg, W1, W3, W2 = ctx.saved_tensors
+        W3 = W3 if ctx.has_w3 else None
+        L = ctx.layer
+        L.backward(dy.contiguous(), x, Wg, W1, W3, W2)
+        return (L.dx.clone(), L.dWg.to(Wg.dtype), L.dW1.to(W1.dtype),
+                None if W3 is None else L.dW3.to(W3.dtype), L.dW2.to(W2.dtype), None, None)

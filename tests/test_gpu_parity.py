@@ -209,6 +209,28 @@ def test_fused_small_forward_matches_oracle(shape):
         assert np.any(f["pos"] < 0), "the case must drop assignments"
 
 
+def test_autograd_function_matches_the_c_abi():
+    """MoEFunction gives the same y and gradients as calling moe_layer_fwd / moe_layer_bwd."""
+    import torch
+    from mixture_experts_layer_23_b200.layer import MoEFunction, MoELayer, to_device
+    shape = LayerShape("autograd", T=300, d=64, E=6, k=2, d_ff=128, n_shared=1, act=SWIGLU,
+                       capacity_factor=1.0, dtype=BF16, bias="normal")
+    inp = make_inputs(shape, 8)
+    dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
+    bias = torch.from_numpy(inp["bias"]).cuda()
+    ref = MoELayer(shape)
+    y_ref = ref.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"]).clone()
+    ref.backward(dev["dy"], dev["x"], dev["Wg"], dev["W1"], dev["W3"], dev["W2"])
+    leaves = {n: dev[n].clone().requires_grad_(True) for n in ("x", "Wg", "W1", "W3", "W2")}
+    y = MoEFunction.apply(leaves["x"], leaves["Wg"], leaves["W1"], leaves["W3"], leaves["W2"],
+                          MoELayer(shape), bias)
+    y.backward(dev["dy"])
+    assert torch.equal(y, y_ref)
+    assert torch.equal(leaves["x"].grad, ref.dx)
+    for n, g in (("Wg", ref.dWg), ("W1", ref.dW1), ("W3", ref.dW3), ("W2", ref.dW2)):
+        assert torch.equal(leaves[n].grad, g.to(leaves[n].dtype)), n
+
+
 def test_zero_capacity_drops_everything():
     s = LayerShape("cap0", T=100, d=32, E=4, k=2, d_ff=32, n_shared=1, dtype=FP32)
     gpu, _ = _parity().full_compare(s, seed=1, capacity=0)
