@@ -87,6 +87,31 @@ def parse():
     return ap.parse_args()
 
 
+def rank_barrier(world):
+    """Barrier over the replicas (no-op on one rank)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(v: float, world: int, device) -> float:
+    """The maximum of v over all ranks (each rank's own device time: the job is as slow as its
+    slowest replica)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world: int, T: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every replica processes T tokens per step; total_ms is the
+    max-over-ranks time of the steps."""
+    return world * T * steps / (total_ms * 1e-3)
+
+
 def dist_env():
     return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
             int(os.environ.get("WORLD_SIZE", 1)))
@@ -314,15 +339,10 @@ def run_ours(args):
             layer.backward(dy, x, w["Wg"], w["W1"], w["W3"], w["W2"])
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        rank_barrier(world)
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -483,10 +503,10 @@ def run_ours(args):
             torch.cuda.synchronize(dev)
             barrier()
             f_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(fs, fe)))
-            fused = {"entry": "moe_layer_fwd_fused", "value": world * shape.T * K / (f_ms * 1e-3),
+            fused = {"entry": "moe_layer_fwd_fused", "value": job_tokens_per_s(world, shape.T, K, f_ms),
                      "unit": "tokens/s", "ms_per_step": f_ms / K, "launches_per_step": 1}
 
-    value = world * shape.T * K / (total_ms * 1e-3)
+    value = job_tokens_per_s(world, shape.T, K, total_ms)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
@@ -504,7 +524,7 @@ def run_ours(args):
         "phases": phases,
         "fused_fwd": fused,
         "phased_ms_per_step": phased_ms,
-        "e2e": {"value": world * shape.T * K / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(world, shape.T, K, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / K},
         "gpu_launches": launches,
