@@ -11,12 +11,13 @@ a barrier and a device synchronise, and the max over ranks is taken.  value = to
 by all ranks / that time.  Several GPUs run independent replicas (the layer has no exchange step
 on one device), so scaling is weak.
 
-Also reported: e2e (the same step through the C ABI with the step's inputs copied from pinned
-host memory and its outputs read back inside the timed region), per-phase device times from the
-library's profiling events (a separate pass after the timed one: events between phases would
-break the overlap of consecutive launches), the roofline of the dominant kernel, SM clocks sampled during the
-timed region, the number of library kernel launches in the timed region, and the CPU oracle
-timed on a bounded sample (rank 0, one GPU).
+Also reported: e2e (the same steps through the C ABI with every step's inputs copied from pinned
+host memory and its outputs read back inside the timed region, the copies on two streams
+overlapped with the compute), per-phase device times from the library's profiling events (a
+separate pass before the timed one: events between phases would break the overlap of
+consecutive launches), the roofline of the dominant kernel, SM clocks sampled during the timed
+region, the number of library kernel launches in the timed region, and the CPU oracle timed on
+a bounded sample (rank 0, one GPU).
 
 --impl reference times the CPU oracle itself on this host's cores as the reference arm.
 """
@@ -449,32 +450,68 @@ def run_ours(args):
         roof["traffic_unit"] = "bytes per launch"
         roof["traffic_source"] = traffic_src
 
-    # end to end through the C ABI with host buffers
+    # end to end through the C ABI with host buffers: every step copies its inputs up from pinned
+    # host memory and its results back down.  The copies run on two copy streams (one per
+    # direction) overlapped with the compute stream, as a training loop prefetching its next batch
+    # would: step i+1's inputs go up and step i-1's results come down while step i computes.  Two
+    # layer instances alternate, so no buffer is overwritten before it has been used or read back.
+    layers = [layer, MoELayer(shape, device=dev)]
+    xs = [x, torch.empty_like(x)]
+    dys = [dy, None if dy is None else torch.empty_like(dy)]
     x_pin = x.cpu().pin_memory()
     dy_pin = None if dy is None else dy.cpu().pin_memory()
-    y_host = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
-    dx_host = torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory()
+    y_host = [torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory() for _ in range(2)]
+    dx_host = [torch.empty(layer.dx.shape, dtype=layer.dx.dtype).pin_memory() for _ in range(2)]
     h2d = x_pin.numel() * x_pin.element_size() + (0 if dy_pin is None else
                                                   dy_pin.numel() * dy_pin.element_size())
-    d2h = y_host.numel() * y_host.element_size() + (0 if dy is None else
-                                                    dx_host.numel() * dx_host.element_size())
-    es, ee = [mk() for _ in range(K)], [mk() for _ in range(K)]
+    d2h = y_host[0].numel() * y_host[0].element_size() + (0 if dy is None else
+                                                          dx_host[0].numel() * dx_host[0].element_size())
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    loaded, computed, drained = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    e_start, e_end = mk(), mk()
     barrier()
     torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    up.wait_stream(stream)
+    down.wait_stream(stream)
     for i in range(K):
-        es[i].record(stream)
-        x.copy_(x_pin, non_blocking=True)
+        b = i % 2
+        L = layers[b]
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(computed[b])        # step i-2 is done reading xs[b], dys[b]
+            xs[b].copy_(x_pin, non_blocking=True)
+            if dy is not None:
+                dys[b].copy_(dy_pin, non_blocking=True)
+            loaded[b].record(up)
+        stream.wait_event(loaded[b])
+        if i >= 2:
+            stream.wait_event(drained[b])         # step i-2's results have been read back
+        L.forward(xs[b], w["Wg"], bias, w["W1"], w["W3"], w["W2"])
         if dy is not None:
-            dy.copy_(dy_pin, non_blocking=True)
-        step()
-        y_host.copy_(layer.y, non_blocking=True)
-        if dy is not None:
-            dx_host.copy_(layer.dx, non_blocking=True)
-        ee[i].record(stream)
-        flush.zero_()
+            L.backward(dys[b], xs[b], w["Wg"], w["W1"], w["W3"], w["W2"])
+        computed[b].record(stream)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            y_host[b].copy_(L.y, non_blocking=True)
+            if dy is not None:
+                dx_host[b].copy_(L.dx, non_blocking=True)
+            drained[b].record(down)
+    stream.wait_stream(down)
+    stream.wait_stream(up)
+    e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)))
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end))
+    del layers[1]
+    # no L2 flush between these steps: each step's inputs arrive fresh from the host, and the
+    # per-step working set (weights + saved forward state) is compared with L2 below
+    work_set = sum(t.numel() * t.element_size() for t in w.values() if t is not None) + \
+        layer.L.ctx_bytes
+    e2e_l2 = ("no flush; per-step working set %.0f MB > 126 MB L2" % (work_set / 1e6)
+              if work_set > 126e6 else
+              "no flush; per-step working set %.1f MB fits in L2 (warm)" % (work_set / 1e6))
 
     # forward-only layers: the one-launch fused forward (moe_layer_fwd_fused), where it applies
     fused = None
@@ -526,7 +563,10 @@ def run_ours(args):
         "phased_ms_per_step": phased_ms,
         "e2e": {"value": job_tokens_per_s(world, shape.T, K, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / K},
+                "ms_per_step": e2e_ms / K,
+                "copies": "pinned host <-> device every step, on two copy streams overlapped with "
+                          "the compute stream (next inputs up, previous results down)",
+                "l2": e2e_l2},
         "gpu_launches": launches,
         "clocks": clk,
     }
