@@ -180,15 +180,15 @@ static moe_status check_ptrs(std::initializer_list<const void*> ps) {
 // Expert FFN forward: the up-projection GEMM, then the down-projection GEMM.  With
 // phase_marks, the profiling event of phase 3 (expert_up) is recorded between the two.
 static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const int32_t* offsets,
-                             const void* W1, const void* W3, const void* W2, void* U, void* V,
+                             const void* W1, const void* W3, const void* W2, void* Gu, void* Gv,
                              void* H, void* O, uint32_t* status, cudaStream_t st,
                              bool phase_marks = false) {
   if (tc_supported(D)) {
-    MOE_TRY(launch_expert_up_tc(D, Xd, x, offsets, W1, W3, U, V, H, status, st));
+    MOE_TRY(launch_expert_up_tc(D, Xd, x, offsets, W1, W3, Gu, Gv, H, status, st));
     if (phase_marks) MOE_TRY(mark_fwd(3, st));
     return launch_expert_down_tc(D, H, offsets, W2, O, status, st);
   }
-  MOE_TRY(launch_expert_up_simt(D, Xd, x, offsets, W1, W3, U, V, H, st));
+  MOE_TRY(launch_expert_up_simt(D, Xd, x, offsets, W1, W3, Gu, Gv, H, st));
   if (phase_marks) MOE_TRY(mark_fwd(3, st));
   return launch_expert_down_simt(D, H, offsets, W2, O, st);
 }
@@ -197,11 +197,11 @@ static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const
 // weight gradients; profiling phases 3..6 of the backward pass.
 static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, const void* Xd,
                              const void* x, const int32_t* offsets, const void* W1,
-                             const void* W3, const void* W2, const void* U, const void* V,
+                             const void* W3, const void* W2, const void* Gu, const void* Gv,
                              const void* H, void* dU, void* dV, void* dXd, float* dW1, float* dW3,
                              float* dW2, uint32_t* status, cudaStream_t st) {
   if (tc_supported(D)) {
-    MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, U, V, dU, dV, status, st));
+    MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, status, st));
     MOE_TRY(mark_bwd(3, st));
     MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
     MOE_TRY(mark_bwd(4, st));
@@ -210,7 +210,7 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
     MOE_TRY(launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st));
     return MOE_OK;
   }
-  MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, U, V, dU, dV, st));
+  MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, st));
   MOE_TRY(mark_bwd(3, st));
   MOE_TRY(launch_dgrad_x_simt(D, dU, dV, offsets, W1, W3, dXd, st));
   MOE_TRY(mark_bwd(4, st));
@@ -327,14 +327,14 @@ moe_status moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* t
 
 moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x,
                           const int32_t* offsets, const void* W1, const void* W3, const void* W2,
-                          void* U, void* V, void* H, void* O, void* scratch,
+                          void* Gu, void* Gv, void* H, void* O, void* scratch,
                           moe_stream_t stream) {
   Dims D;
   MOE_TRY(resolve_dims(cfg, &D));
-  MOE_TRY(check_ptrs({Xd, x, offsets, W1, W2, U, H, O, scratch}));
-  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, V}));
+  MOE_TRY(check_ptrs({Xd, x, offsets, W1, W2, Gu, H, O, scratch}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, Gv}));
   const ScratchLayout S = scratch_layout(D);
-  return expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O,
+  return expert_fwd(D, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, O,
                     (uint32_t*)((char*)scratch + S.status), (cudaStream_t)stream);
 }
 
@@ -370,8 +370,8 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   int32_t* slot = (int32_t*)(c + L.ctx_slot);
   int32_t* row_token = (int32_t*)(c + L.ctx_row_token);
   void* Xd = c + L.ctx_Xd;
-  void* U = c + L.ctx_Gu;
-  void* V = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
+  void* Gu = c + L.ctx_Gu;
+  void* Gv = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
   void* H = c + L.ctx_H;
   void* O = c + L.ctx_O;
   MOE_TRY(mark_fwd(0, st));
@@ -383,7 +383,7 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
     MOE_TRY(launch_aux_loss(D, logits, counts, (float*)(s + S.aux_part), (float*)(c + L.ctx_aux_loss),
                             st));
   MOE_TRY(mark_fwd(2, st));
-  MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, U, V, H, O, (uint32_t*)(s + S.status), st,
+  MOE_TRY(expert_fwd(D, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, O, (uint32_t*)(s + S.status), st,
                      /*phase_marks=*/true));
   MOE_TRY(mark_fwd(4, st));
   MOE_TRY(launch_combine(D, O, slot, w, y, st));
@@ -412,8 +412,8 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   const int32_t* offsets = (const int32_t*)(c + L.ctx_offsets);
   const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
   const void* Xd = c + L.ctx_Xd;
-  const void* U = c + L.ctx_Gu;
-  const void* V = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
+  const void* Gu = c + L.ctx_Gu;
+  const void* Gv = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
   const void* H = c + L.ctx_H;
   const void* O = c + L.ctx_O;
   void* dO = s + S.dO;
@@ -440,7 +440,7 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
     MOE_TRY(launch_router_wgrad(D, dl, x, part, dWg, st));
   }
   MOE_TRY(mark_bwd(2, st));
-  MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, U, V, H, dU, dV, dXd, dW1, dW3, dW2,
+  MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, dU, dV, dXd, dW1, dW3, dW2,
                      (uint32_t*)(s + S.status), st));
   MOE_TRY(mark_bwd(6, st));
   if (rtc) {

@@ -202,9 +202,9 @@ def dispatch_noalloc(cfg, x, topk_idx, counts, kept, offsets, slot, row_token, X
                                      _stream(stream)), "moe_dispatch_noalloc")
 
 
-def expert_ffn(cfg, Xd, x, offsets, W1, W3, W2, U, V, H, O, scratch, stream=None):
+def expert_ffn(cfg, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, O, scratch, stream=None):
     _check(_lib.moe_expert_ffn(ctypes.byref(cfg), _p(Xd), _p(x), _p(offsets), _p(W1), _p(W3),
-                               _p(W2), _p(U), _p(V), _p(H), _p(O), _p(scratch), _stream(stream)),
+                               _p(W2), _p(Gu), _p(Gv), _p(H), _p(O), _p(scratch), _stream(stream)),
            "moe_expert_ffn")
 
 
