@@ -123,3 +123,35 @@ class MoEFunction(torch.autograd.Function):
         L.backward(dy.contiguous(), x, Wg, W1, W3, W2)
         return (L.dx.clone(), L.dWg.to(Wg.dtype), L.dW1.to(W1.dtype),
                 None if W3 is None else L.dW3.to(W3.dtype), L.dW2.to(W2.dtype), None, None)
+
+
+class MoEStepGraph:
+    """One forward (+ backward) of a MoELayer captured into a CUDA graph and replayed.
+
+    The library's launches, their programmatic-dependent-launch edges included, are recorded once
+    from the current torch stream; replay() re-issues them with one call, without the host cost of
+    each launch.  Every buffer is fixed at capture: to run a new batch, copy it into the same x and
+    dy tensors before replay().  Outputs land in the layer's buffers (layer.y, layer.dx, layer.dWg,
+    ...), as with direct calls."""
+
+    def __init__(self, layer, x, Wg, bias, W1, W3, W2, dy=None):
+        self.layer = layer
+        args = (x, Wg, bias, W1, W3, W2)
+
+        def run():
+            layer.forward(*args)
+            if dy is not None:
+                layer.backward(dy, x, Wg, W1, W3, W2)
+
+        side = torch.cuda.Stream(device=layer.device)
+        side.wait_stream(torch.cuda.current_stream(layer.device))
+        with torch.cuda.stream(side):   # one eager pass first: one-time host set-up stays out of the graph
+            run()
+        torch.cuda.current_stream(layer.device).wait_stream(side)
+        torch.cuda.synchronize(layer.device)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            run()
+
+    def replay(self):
+        self.graph.replay()
