@@ -236,6 +236,13 @@ def test_softmax_closed_forms():
     assert np.allclose(g1, g0, rtol=0, atol=1e-15)
     # invariance to a constant shift of the logits (large values do not overflow)
     assert np.allclose(mo.softmax(L + 700.0), mo.softmax(L), atol=1e-15)
+    # for any k, the softmax over the k chosen logits is the full softmax at the chosen experts
+    # renormalised over them (GShard-style renormalised top-k is gate_norm 1)
+    for k in (1, 2, 3):
+        idx = mo.select_topk(L, k)
+        p = np.take_along_axis(mo.softmax(L), idx, axis=1)
+        assert np.allclose(mo.gate_weights(L, idx, 1), p / p.sum(1, keepdims=True), rtol=0,
+                           atol=1e-15)
 
 
 @pytest.mark.parametrize("seed", [0, 1, 2])
