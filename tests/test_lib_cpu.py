@@ -152,6 +152,29 @@ def test_fused_forward_rejects_large_layers_before_any_cuda_call(moe):
                                    good, good, good, None, None, None) == 1
 
 
+def test_ctypes_structs_match_the_header(moe, tmp_path):
+    """The binding's ctypes mirrors of moe_config_t and moe_layout_t have the C compiler's layout:
+    the same size, and every field at the same offset with the same size."""
+    import subprocess
+    exe = tmp_path / "abi_layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "host", "abi_layout.c"), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    structs = {"moe_config_t": moe.Config, "moe_layout_t": moe.Layout}
+    seen = {name: set() for name in structs}
+    for line in filter(None, out):
+        parts = line.split()
+        S = structs[parts[0]]
+        if parts[1] == "sizeof":
+            assert ctypes.sizeof(S) == int(parts[2]), parts[0]
+            continue
+        field = getattr(S, parts[1])
+        assert (field.offset, field.size) == (int(parts[2]), int(parts[3])), line
+        seen[parts[0]].add(parts[1])
+    for name, S in structs.items():
+        assert seen[name] == {f for f, _ in S._fields_}, name
+
+
 def test_status_strings(moe):
     for code in range(7):
         assert moe.lib().moe_status_string(code)
