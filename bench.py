@@ -452,7 +452,7 @@ def run_ours(args):
 
     # the same step captured once into a CUDA graph and replayed (MoEStepGraph): one host call per
     # step instead of one per launch; reported beside the eager value, which stays the headline
-    graph = None
+    graph, sg = None, None
     try:
         from mixture_experts_layer_23_b200.layer import MoEStepGraph
         n0 = moe.kernel_launches()
@@ -460,6 +460,11 @@ def run_ours(args):
         per_step = (moe.kernel_launches() - n0) // 2   # the eager warm-up pass, then the capture
     except Exception as err:   # capture not possible here: report why, keep the eager numbers
         graph = {"error": str(err)[:300]}
+    # every rank takes the same collective steps: time the replays only if all ranks captured
+    if reduce_max(0.0 if sg is not None else 1.0, world, dev) > 0.0:
+        if graph is None:
+            graph = {"error": "graph capture failed on another rank"}
+        sg = None
     else:
         for _ in range(args.warmup):
             sg.replay()
