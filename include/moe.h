@@ -138,10 +138,14 @@ moe_status moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* t
  * `scratch`, produces identical outputs, and allocates nothing: the per-CTA expert histograms live
  * in a fixed 256 KB array inside the library, which every GPU that loads the library holds until
  * the process exits.
- * Limit: ceil(T / 256) * E <= 65536 (for example T = 65536 with E = 256, or T = 2^20 with E = 16);
- * larger configs return MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
+ * Limit: ceil(T / 256) * E * L <= 65536, with L = 1 for token-order drops (drop_order 0) and L = k
+ * for choice-major drops (drop_order 1), which keep one histogram layer per choice index (for
+ * example T = 65536 with E = 256 in token order, or T = 2^20 with E = 16); larger configs return
+ * MOE_ERR_WORKSPACE_TOO_SMALL and enqueue nothing.
  * The first call on a device looks up the array's device address with that device current; make
- * that first call before any stream capture.
+ * that first call before any stream capture.  The address is remembered per device together with
+ * the CUDA context it belongs to: after the caller resets the device (cudaDeviceReset), the next
+ * call looks it up again in the new context.
  * All calls share the one array: calls that overlap on the GPU (for example on two streams) race
  * and corrupt each other's results, so serialise them.  The array keeps the last call's contents;
  * each call rewrites every entry it reads, so nothing needs clearing. */
@@ -209,8 +213,26 @@ moe_status moe_scratch_grad_offsets(const moe_config_t* cfg, size_t* dg_offset,
 
 /* Synchronise `stream`, then report and clear the device status word kept in scratch:
  * MOE_ERR_DEVICE_TIMEOUT if a bounded device wait gave up since the last call, MOE_ERR_CUDA
- * if the stream reported an error, else MOE_OK. */
+ * if the stream reported an error, else MOE_OK.
+ * Failure detection (the tutorial's debugging notes on deadlocked or mismatched collectives,
+ * Ch.4 "分布式训练"): every wait of the tensor-core kernels on a barrier (a TMA copy, an MMA, the
+ * accumulator hand-off) is bounded.  When one runs out, the CTA stops taking work, lets its own
+ * copies and MMAs in flight finish, frees its tensor memory and sets MOE_STATUS_TIMEOUT in the
+ * status word; the context stays usable.  Outputs of that launch are then undefined, but well
+ * formed: the router writes the placeholder routing experts 0..k-1 with weight 0, so the kernels
+ * after it in the same pass stay in bounds.  moe_route and moe_combine take no scratch and cannot
+ * report a timeout. */
 moe_status moe_read_status(moe_stream_t stream, void* scratch);
+
+/* Time budget of every bounded device wait, in nanoseconds, for kernels launched after the call
+ * (default 2e9 = 2 s; accepted range 1e3 .. 6e10, else MOE_ERR_INVALID_ARG).  Process-wide. */
+moe_status moe_set_wait_budget_ns(uint64_t budget_ns);
+
+/* Test hook of the failure path: with on = 1, every tensor-core kernel launched afterwards first
+ * waits on a barrier that nothing arrives on, so that wait runs out after the budget and the
+ * kernel takes the abort path above (no fault, no hang: the wait is bounded).  on = 0 restores
+ * normal operation.  Process-wide; for tests only. */
+moe_status moe_set_wait_stall(int32_t on);
 
 /* Name and description of the CUDA error behind the most recent MOE_ERR_CUDA in this process
  * ("" if none).  Process-wide; the text stays valid until the next failure. */

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include "launch.h"
+#include "tc_host.h"
 
 namespace moe {
 
@@ -465,6 +466,18 @@ moe_status moe_set_profile_events(void* const* fwd_events, void* const* bwd_even
     g_fwd_events[i] = (cudaEvent_t)fwd_events[i];   // NULL entries are skipped
   for (int i = 0; g_bwd_prof && i <= MOE_BWD_PHASES; ++i)
     g_bwd_events[i] = (cudaEvent_t)bwd_events[i];
+  return MOE_OK;
+}
+
+moe_status moe_set_wait_budget_ns(uint64_t budget_ns) {
+  if (budget_ns < 1000 || budget_ns > 60ull * 1000000000ull) return MOE_ERR_INVALID_ARG;
+  tc::set_wait_budget_ns(budget_ns);
+  return MOE_OK;
+}
+
+moe_status moe_set_wait_stall(int32_t on) {
+  if (on != 0 && on != 1) return MOE_ERR_INVALID_ARG;
+  tc::set_wait_stall(on);
   return MOE_OK;
 }
 

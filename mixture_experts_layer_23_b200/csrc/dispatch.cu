@@ -225,20 +225,43 @@ constexpr int kNoAllocMaxHistogram = 1 << 16;  // int32 entries: ceil(T / 256) *
                                                // choice-major) must fit
 static __device__ __align__(256) int32_t g_noalloc_histogram[kNoAllocMaxHistogram];
 
+// The CUDA context current on this thread (through the runtime's driver entry point, so the
+// library does not link libcuda); null if it cannot be read.
+static void* current_context() {
+  typedef int (*CtxGetCurrentFn)(void**);
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
 // Device address of the array on the current device, looked up once per device (with that device
-// current, on its first call).  In host code the array's name is only a host-side stand-in, so the
-// kernels must be given this address, never the name.
+// current, on its first call) and again whenever that device's context has changed since (after a
+// cudaDeviceReset the module is loaded anew and the array may sit elsewhere).  In host code the
+// array's name is only a host-side stand-in, so the kernels must be given this address, never the
+// name.
 static moe_status noalloc_histogram(int32_t** out) {
   constexpr int kMaxDevices = 64;
   static int32_t* addr[kMaxDevices] = {};
+  static void* ctx_of[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+  void* ctx = current_context();   // null before the runtime has made a context current
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || !ctx || ctx != ctx_of[dev]) {
     void* p = nullptr;
+    // (this call also makes the device's primary context current on this thread)
     if (cudaGetSymbolAddress(&p, g_noalloc_histogram) != cudaSuccess || !p) return MOE_ERR_CUDA;
     addr[dev] = static_cast<int32_t*>(p);
+    ctx_of[dev] = current_context();
   }
   *out = addr[dev];
   return MOE_OK;

@@ -107,6 +107,8 @@ struct alignas(64) Params {
   int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
   int chunk;             // > 0: the groups are fixed chunks of this many token rows (router
                          // backward) instead of the experts' row ranges
+  int stall;             // failure-path test: the MMA issuer first waits on a barrier that
+                         // nothing arrives on, so the wait runs out and the CTA aborts
 };
 
 // Instruction descriptor of the pair MMA: bf16 x bf16 -> fp32, M = 256 (two CTAs), N = BN.
@@ -717,12 +719,13 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   constexpr bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == WGRAD);
   constexpr uint32_t IDESC = make_idesc(A_MN, B_MN);
 
+  // producer bookkeeping, read again after every role has finished (abort drain)
+  uint32_t outstanding = 0;            // stages with a load issued and not yet seen consumed
+  uint32_t out_phase = 0;              // bit s: phase parity of stage s's last issued load
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer (both CTAs)
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t outstanding = 0;          // stages with a load in flight not yet seen consumed
-    uint32_t out_phase = 0;            // bit s: phase parity of stage s's last issued load
     for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
@@ -739,14 +742,6 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       }
       if (!ok) break;
     }
-    if (*abort_flag && rank == 0) {
-      // let the pair's copies into stages we armed land before the CTAs exit
-      for (int s = 0; s < STAGES; ++s)
-        if (outstanding & (1u << s)) {
-          volatile int never = 0;
-          wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
-        }
-    }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ---------------- MMA issuer (leader CTA only)
     int stage = 0;
@@ -757,6 +752,9 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     const uint32_t b_step = B_MN ? 2048u : 32u;
     const uint32_t a_lbo = A_MN ? 8192u : 16u, b_lbo = B_MN ? 8192u : 16u;
     bool issued_any = false;
+    // test hook: `drain` gets no arrival before an abort, so this wait runs out after `budget`
+    // and raises the abort flag before any MMA is issued
+    if (P.stall) wait_bounded(drain, 0u, abort_flag, budget);
     for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
@@ -820,6 +818,25 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   }
   __syncwarp();
   tc_fence_before();
+  cluster_sync();   // every role of both CTAs has finished (the abort flag is final)
+  if (*abort_flag && warp == 0 && lane == 0 && outstanding) {
+    // An aborted CTA may still have TMA loads in flight into its shared memory: they must land
+    // before it exits.  The leader sees the pair's copies complete on its full barriers; the
+    // second CTA's copies are counted on the leader's barriers, so it waits a fixed grace period
+    // (far longer than a copy takes) instead.
+    if (rank == 0) {
+      for (int s = 0; s < STAGES; ++s)
+        if (outstanding & (1u << s)) {
+          volatile int never = 0;
+          wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
+        }
+    } else {
+      const unsigned long long t0 = globaltimer();
+      while (globaltimer() - t0 < 200000ull) {
+      }
+    }
+  }
+  __syncwarp();
   cluster_sync();   // the pair's MMAs, copies and TMEM reads are over before either CTA moves on
   if (*abort_flag && threadIdx.x == 0) atomicOr(P.status, MOE_STATUS_TIMEOUT);
   if (warp == 1) {
@@ -857,6 +874,7 @@ static Params base_params(const Dims& D, const int32_t* offsets, uint32_t* statu
   P.offsets = offsets;
   P.status = status;
   P.timeout_ns = wait_budget_ns();
+  P.stall = wait_stall();
   P.T_pad = D.T_pad;
   P.E = D.E;
   P.S = D.S;

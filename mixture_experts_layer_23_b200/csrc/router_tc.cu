@@ -42,6 +42,7 @@ struct alignas(64) RouterParams {
   int T, d, E, E_pad, k, gate_norm;
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages;
+  int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
 };
 
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
@@ -78,9 +79,10 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   const int nk = P.d / 64;
   const unsigned long long budget = P.timeout_ns;
 
+  uint32_t outstanding = 0, out_phase = 0;   // producer: stages loaded and not seen consumed
   if (warp == 0 && lane == 0) {
     int stage = 0;
-    uint32_t phase = 0, outstanding = 0, out_phase = 0;
+    uint32_t phase = 0;
     for (int kb = 0; kb < nk; ++kb) {
       if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) break;
       outstanding &= ~(1u << stage);
@@ -92,18 +94,13 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
     }
-    if (*abort_flag) {
-      for (int s = 0; s < RSTAGES; ++s)
-        if (outstanding & (1u << s)) {
-          volatile int never = 0;
-          wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
-        }
-    }
   } else if (warp == 1 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;
     bool issued = false, ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    // test hook: `drain` gets no arrival before an abort, so this wait runs out after `budget`
+    if (P.stall && !wait_bounded(drain, 0u, abort_flag, budget)) ok = false;
+    for (int kb = 0; ok && kb < nk; ++kb) {
       if (!wait_bounded(&full[stage], phase, abort_flag, budget)) { ok = false; break; }
       tc_fence_after();
       const uint32_t sa = smem_u32(smem + stage * P.stage_bytes);
@@ -147,10 +144,31 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       if (live)
         topk_finish(st, P.k, P.gate_norm, P.topk_idx + (size_t)t * P.k,
                     P.topk_w + (size_t)t * P.k);
+    } else {
+      // the accumulator never arrived (a wait ran out): write a well-formed placeholder routing
+      // (experts 0..k-1, weight 0, logits 0) so the kernels after this one stay in bounds; the
+      // status word reports the timeout
+      const int t = m0 + quarter * 32 + lane;
+      if (t < P.T) {
+        for (int e = 0; e < P.E; ++e) P.logits[(size_t)t * P.E + e] = 0.f;
+        for (int j = 0; j < P.k; ++j) {
+          P.topk_idx[(size_t)t * P.k + j] = j;
+          P.topk_w[(size_t)t * P.k + j] = 0.f;
+        }
+      }
     }
   }
   __syncwarp();
   tc_fence_before();
+  __syncthreads();   // every role has finished (the abort flag is final)
+  if (*abort_flag && warp == 0 && lane == 0) {
+    // TMA loads of an aborted CTA may still be in flight: let them land before it exits
+    for (int s = 0; s < RSTAGES; ++s)
+      if (outstanding & (1u << s)) {
+        volatile int never = 0;
+        wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
+      }
+  }
   __syncthreads();
   if (*abort_flag && threadIdx.x == 0 && P.status) atomicOr(P.status, MOE_STATUS_TIMEOUT);
   if (warp == 1) {
@@ -181,6 +199,7 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   P.topk_w = topk_w;
   P.status = status;
   P.timeout_ns = tc::wait_budget_ns();
+  P.stall = tc::wait_stall();
   P.T = D.T;
   P.d = D.d;
   P.E = D.E;

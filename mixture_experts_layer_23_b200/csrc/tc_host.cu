@@ -68,8 +68,11 @@ int num_sms() {
 }
 
 static unsigned long long g_wait_budget_ns = 2000000000ull;
+static int g_wait_stall = 0;
 unsigned long long wait_budget_ns() { return g_wait_budget_ns; }
 void set_wait_budget_ns(unsigned long long ns) { g_wait_budget_ns = ns; }
+int wait_stall() { return g_wait_stall; }
+void set_wait_stall(int on) { g_wait_stall = on ? 1 : 0; }
 
 }  // namespace tc
 }  // namespace moe

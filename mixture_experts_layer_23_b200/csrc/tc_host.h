@@ -26,6 +26,10 @@ int num_sms();
 // Time budget of every bounded device wait in the tcgen05 kernels (default 2 s).
 unsigned long long wait_budget_ns();
 void set_wait_budget_ns(unsigned long long ns);
+// Failure-path test hook: when set, the tcgen05 kernels launched afterwards first wait on a
+// barrier that nothing arrives on (moe_set_wait_stall).
+int wait_stall();
+void set_wait_stall(int on);
 
 }  // namespace tc
 }  // namespace moe

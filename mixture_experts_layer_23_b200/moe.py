@@ -24,7 +24,8 @@ EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_layer_fwd", "moe_layer_bwd",
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
            "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
-           "moe_last_cuda_error", "moe_aux_loss", "moe_layer_fwd_fused")
+           "moe_last_cuda_error", "moe_aux_loss", "moe_layer_fwd_fused",
+           "moe_set_wait_budget_ns", "moe_set_wait_stall")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -85,6 +86,8 @@ def _load():
         "moe_kernel_launches": [],
         "moe_set_profile_events": [P, P],
         "moe_last_cuda_error": [],
+        "moe_set_wait_budget_ns": [ctypes.c_uint64],
+        "moe_set_wait_stall": [I32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -254,3 +257,11 @@ def set_profile_events(fwd_events=None, bwd_events=None):
 
 
 _prof_keep = None
+
+
+def set_wait_budget_ns(budget_ns: int) -> None:
+    _check(_lib.moe_set_wait_budget_ns(int(budget_ns)), "moe_set_wait_budget_ns")
+
+
+def set_wait_stall(on: bool) -> None:
+    _check(_lib.moe_set_wait_stall(1 if on else 0), "moe_set_wait_stall")

@@ -439,3 +439,68 @@ def expert_weight_grad_rows(e, fs, r, x, W1, W3, W2, dy, *, act, n_shared):
     dW3_rows = None if dV is None else dV.T @ X
     dW2_cols = dO.T @ H           # [d, len(fs)]
     return dW1_rows, dW3_rows, dW2_cols
+
+
+def expert_input_grad(X, U, V, H, dO, W1e, W3e, W2e, act: int):
+    """dX of one expert alone: the input-gradient part of `expert_backward` (same chain rule,
+    without the weight gradients), for layers whose weight gradients are checked elsewhere."""
+    dH = dO @ W2e
+    if act == GELU:
+        return (dH * gelu_grad(U)) @ W1e
+    dU = dH * V * silu_grad(U)
+    dV = dH * silu(U)
+    return dU @ W1e + dV @ W3e
+
+
+def layer_by_expert(x, Wg, bias, W1, W3, W2, dy, *, k: int, act: int, gate_norm: int,
+                    capacity_factor, n_shared: int = 0, idx_override=None,
+                    choice_major: bool = False, aux_loss_coef: float = 0.0,
+                    with_dx: bool = True):
+    """y, dg, dlogits, dWg and (with_dx) dx of the whole layer, one expert at a time.
+
+    The same formulas as `layer_forward` followed by `layer_backward` (routing, dispatch, each
+    expert's FFN, combine; dg = <dy, o> at kept assignments, the router backward, dWg = dl^T x,
+    dx = the experts' input gradients + dl Wg), evaluated expert by expert so that no expert's
+    activations are kept once its rows are done: a layer with large experts then needs only one
+    expert's intermediates in memory.  W1, W3, W2 may be anything indexable by expert id.
+    Weight gradients of the experts are not formed (see expert_weight_grad_rows).
+    """
+    T, d = x.shape
+    E = Wg.shape[0]
+    logits = gate_logits(x, Wg, bias)
+    idx = select_topk(logits, k) if idx_override is None else np.asarray(idx_override, np.int64)
+    g = gate_weights(logits, idx, gate_norm)
+    C = capacity(capacity_factor, k, T, E)
+    counts, kept, pos = dispatch(idx, E, C, choice_major)
+    y = np.zeros((T, d))
+    dx = np.zeros((T, d)) if with_dx else None
+    dg = np.zeros((T, k))
+    for e in range(E + n_shared):
+        if e < E:
+            tt, jj = expert_rows(idx, pos, e)
+            if len(tt) == 0:
+                continue
+            X = x[tt]
+        else:
+            tt, jj, X = np.arange(T), None, x
+        W1e, W2e = W1[e], W2[e]
+        W3e = None if W3 is None else W3[e]
+        U, V, H, O = expert_forward(X, W1e, W3e, W2e, act)
+        if e < E:
+            np.add.at(y, tt, g[tt, jj][:, None] * O)
+            dg[tt, jj] = np.einsum("rd,rd->r", dy[tt], O)
+            dO = g[tt, jj][:, None] * dy[tt]
+        else:
+            y += O
+            dO = dy
+        if with_dx:
+            np.add.at(dx, tt, expert_input_grad(X, U, V, H, dO, W1e, W3e, W2e, act))
+        del U, V, H, O, dO
+    dl = router_backward(logits, idx, g, dg, gate_norm)
+    if aux_loss_coef:
+        dl = dl + aux_loss_grad(logits, counts, k, aux_loss_coef)
+    dWg = dl.T @ x
+    if with_dx:
+        dx += dl @ Wg
+    return {"logits": logits, "idx": idx, "g": g, "C": C, "counts": counts, "kept": kept,
+            "pos": pos, "y": y, "dg": dg, "dlogits": dl, "dWg": dWg, "dx": dx}

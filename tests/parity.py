@@ -28,13 +28,16 @@ def assert_close(name, got, ref, rel):
 
 
 class LazyF64:
-    """Per-expert float64 view of a large storage-form weight (converted on first use)."""
+    """Per-expert float64 view of a large storage-form weight (converted on use; kept for reuse
+    unless keep=False)."""
 
-    def __init__(self, a, dtype):
-        self.a, self.dtype, self.cache = a, dtype, {}
+    def __init__(self, a, dtype, keep=True):
+        self.a, self.dtype, self.cache, self.keep = a, dtype, {}, keep
         self.shape = a.shape
 
     def __getitem__(self, e):
+        if not self.keep:
+            return to_f64(self.a[e], self.dtype)
         if e not in self.cache:
             self.cache[e] = to_f64(self.a[e], self.dtype)
         return self.cache[e]
@@ -169,16 +172,19 @@ def full_compare(shape: LayerShape, seed=0, *, inp=None, capacity=None):
     return gpu, errs
 
 
-def sampled_compare(shape: LayerShape, seed=0, n_tok=24, n_f=3, experts=None):
-    """Full-size layers: routing and dispatch compared in full (bit-exact); y, dx and dg on
-    sampled tokens; rows of dW1/dW3 and columns of dW2 on sampled experts; dWg through the
-    property that its rows sum to zero (each token's logit gradient sums to zero over E)."""
+def large_compare(shape: LayerShape, seed=0, *, full_dx=True, n_tok=24, n_f=3, experts=None):
+    """Full-size layers.  Routing and dispatch in full (bit-exact).  y, dg and dWg in full, and
+    dx in full when full_dx, from the oracle's one-expert-at-a-time form of the whole layer;
+    otherwise dx on sampled tokens.  Rows of dW1/dW3 and columns of dW2 on sampled experts (each
+    an exact sum over all of the expert's rows).  Returns the GPU outputs and the oracle's CPU
+    seconds."""
+    import time
     inp = make_inputs(shape, seed)
     gpu = run_gpu(shape, inp)
     dt = shape.dtype
     x, Wg = to_f64(inp["x"], dt), to_f64(inp["Wg"], dt)
-    W1, W2 = LazyF64(inp["W1"], dt), LazyF64(inp["W2"], dt)
-    W3 = None if inp["W3"] is None else LazyF64(inp["W3"], dt)
+    W1, W2 = LazyF64(inp["W1"], dt, keep=False), LazyF64(inp["W2"], dt, keep=False)
+    W3 = None if inp["W3"] is None else LazyF64(inp["W3"], dt, keep=False)
     dy = None if shape.fwd_only else to_f64(inp["dy"], dt)
     r = mo.route(x, Wg, inp["bias"], k=shape.k, gate_norm=shape.gate_norm,
                  capacity_factor=shape.capacity_factor, choice_major=shape.choice_major)
@@ -191,20 +197,30 @@ def sampled_compare(shape: LayerShape, seed=0, n_tok=24, n_f=3, experts=None):
                                                    choice_major=shape.choice_major)
     rel = tol_for(shape)
     assert_close("topk_w", gpu["topk_w"], r["g"], rel)
+    assert not shape.fwd_only
+    t0 = time.perf_counter()
+    f = mo.layer_by_expert(x, Wg, inp["bias"], W1, W3, W2, dy, k=shape.k, act=shape.act,
+                           gate_norm=shape.gate_norm, capacity_factor=shape.capacity_factor,
+                           n_shared=shape.n_shared, idx_override=gidx,
+                           choice_major=shape.choice_major, aux_loss_coef=shape.aux_loss_coef,
+                           with_dx=full_dx)
+    cpu_s = time.perf_counter() - t0
+    assert np.array_equal(f["pos"], r["pos"])
+    assert_close("y", gpu["y"], f["y"], rel)
+    assert_close("dg", gpu["dg"], f["dg"], rel)
+    assert_close("dWg", gpu["dWg"], f["dWg"], rel)
     rng = np.random.default_rng(seed + 1)
-    dropped_tok = np.nonzero(np.any(r["pos"] < 0, axis=1))[0]
-    picks = [0, shape.T - 1] + list(rng.choice(shape.T, n_tok, replace=False))
-    if len(dropped_tok):
-        picks += list(rng.choice(dropped_tok, min(4, len(dropped_tok)), replace=False))
-    toks = sorted(set(int(t) for t in picks))
-    y, dx, dg = mo.token_forward_backward(toks, r, x, Wg, W1, W3, W2, dy, act=shape.act,
-                                          gate_norm=shape.gate_norm, n_shared=shape.n_shared)
-    # per-tensor scale from the sampled reference rows
-    assert_close("y[sampled]", gpu["y"][toks], y, rel)
-    if shape.fwd_only:
-        return gpu
-    assert_close("dx[sampled]", gpu["dx"][toks], dx, rel)
-    assert_close("dg[sampled]", gpu["dg"][toks], dg, rel)
+    if full_dx:
+        assert_close("dx", gpu["dx"], f["dx"], rel)
+    else:
+        dropped_tok = np.nonzero(np.any(r["pos"] < 0, axis=1))[0]
+        picks = [0, shape.T - 1] + list(rng.choice(shape.T, n_tok, replace=False))
+        if len(dropped_tok):
+            picks += list(rng.choice(dropped_tok, min(4, len(dropped_tok)), replace=False))
+        toks = sorted(set(int(t) for t in picks))
+        _, dx, _ = mo.token_forward_backward(toks, r, x, Wg, W1, W3, W2, dy, act=shape.act,
+                                             gate_norm=shape.gate_norm, n_shared=shape.n_shared)
+        assert_close("dx[sampled]", gpu["dx"][toks], dx, rel)
     exps = experts if experts is not None else sorted(set([0, shape.E - 1, shape.E_tot - 1]))
     for e in exps:
         fs = sorted(set([0, shape.d_ff - 1] + list(rng.choice(shape.d_ff, n_f, replace=False))))
@@ -214,10 +230,4 @@ def sampled_compare(shape: LayerShape, seed=0, n_tok=24, n_f=3, experts=None):
         assert_close(f"dW2[{e}][:,fs]", gpu["dW2"][e][:, fs], c, rel)
         if b is not None:
             assert_close(f"dW3[{e}][fs]", gpu["dW3"][e][fs], b, rel)
-    # each token's logit gradient sums to zero over E, so the columns of dWg do too; on the bf16
-    # path the logit gradient is rounded to bf16 before the router-backward GEMMs (2^-9 relative
-    # per element), which the looser bf16 bound absorbs
-    colsum = gpu["dWg"].sum(axis=0)
-    bound = (1e-2 if shape.dtype == BF16 else 1e-3) * np.max(np.abs(gpu["dWg"])) * np.sqrt(shape.E)
-    assert np.max(np.abs(colsum)) <= bound, (np.max(np.abs(colsum)), bound)
-    return gpu
+    return gpu, cpu_s

@@ -179,3 +179,18 @@ def test_status_strings(moe):
     for code in range(7):
         assert moe.lib().moe_status_string(code)
     assert moe.lib().moe_status_string(99) == b"unknown status"
+
+
+def test_wait_hooks_validate_their_arguments(moe):
+    """The bounded-wait settings are host-only setters: out-of-range values are refused, valid
+    ones accepted (and the defaults put back)."""
+    lib = moe.lib()
+    assert lib.moe_set_wait_budget_ns(0) == 1
+    assert lib.moe_set_wait_budget_ns(999) == 1
+    assert lib.moe_set_wait_budget_ns(61 * 10**9) == 1
+    assert lib.moe_set_wait_stall(2) == 1
+    assert lib.moe_set_wait_stall(-1) == 1
+    assert lib.moe_set_wait_budget_ns(1000) == 0
+    assert lib.moe_set_wait_stall(1) == 0
+    assert lib.moe_set_wait_stall(0) == 0
+    assert lib.moe_set_wait_budget_ns(2 * 10**9) == 0

@@ -72,6 +72,33 @@ def pin_hand_dispatch(name="hand_dispatch.json"):
             and kept.tolist() == ex["kept"] and pos.tolist() == ex["pos"])
 
 
+def pin_gate_bias_golden():
+    """The hand-worked gate with a per-expert logit bias: the bias flips every token's top-1 and
+    sets the softmax weights (exact fractions), for the full and the top-k softmax."""
+    g = _golden("hand_gate_bias.json")
+    x, Wg, b = np.array(g["x"]), np.array(g["Wg"]), np.array(g["bias"])
+    logits = mo.gate_logits(x, Wg, b)
+    if mo.select_topk(mo.gate_logits(x, Wg, None), 1).tolist() != g["without_bias_top1"]:
+        return False
+    for c in g["cases"]:
+        idx = mo.select_topk(logits, c["k"])
+        want = np.array([[n / m for n, m in row] for row in c["w_frac"]])
+        if idx.tolist() != c["idx"]:
+            return False
+        if not np.allclose(mo.gate_weights(logits, idx, c["gate_norm"]), want, rtol=0,
+                           atol=1e-12):
+            return False
+        # the same through the layer: identity experts, nothing dropped -> y_t = sum_j w_tj x_t
+        f = mo.layer_forward(x, Wg, b, None, None, None, k=c["k"], act=mo.GELU,
+                             gate_norm=c["gate_norm"], capacity_factor=None,
+                             identity_experts=True)
+        if f["idx"].tolist() != c["idx"]:
+            return False
+        if not np.allclose(f["y"], want.sum(axis=1, keepdims=True) * x, rtol=0, atol=1e-12):
+            return False
+    return True
+
+
 def pin_choice_major_priority(seed=3):
     """Choice-major invariant: at every expert, once a choice index j has a dropped assignment,
     no assignment with a later choice index is kept; and the kept counts equal token order's."""
@@ -194,6 +221,10 @@ def test_dispatch_matches_brute_force():
 
 def test_hand_worked_dispatch():
     assert pin_hand_dispatch()
+
+
+def test_hand_worked_gate_bias():
+    assert pin_gate_bias_golden()
 
 
 def test_hand_worked_choice_major_dispatch():
@@ -355,6 +386,44 @@ def test_aux_loss_gradient_matches_finite_differences():
     assert pin_aux_grad_fd()
 
 
+@pytest.mark.parametrize("case", [
+    dict(act=1, gate_norm=0, cf=1.0, n_shared=1, bias="normal", choice_major=False, aux=0.0),
+    dict(act=0, gate_norm=0, cf=0.7, n_shared=0, bias="zipf", choice_major=True, aux=0.3),
+    dict(act=1, gate_norm=1, cf=None, n_shared=2, bias="none", choice_major=False, aux=0.0),
+])
+def test_by_expert_form_equals_full_layer(case):
+    """layer_by_expert (one expert's intermediates at a time) gives layer_forward's y and
+    layer_backward's dg, dlogits, dWg and dx; expert_input_grad gives expert_backward's dX."""
+    from mixture_experts_layer_23_b200.configs import LayerShape
+    from mixture_experts_layer_23_b200.synth import make_inputs, to_f64
+    sh = LayerShape("s", T=150, d=16, E=7, k=3, d_ff=24, n_shared=case["n_shared"],
+                    act=case["act"], gate_norm=case["gate_norm"], capacity_factor=case["cf"],
+                    dtype=1, bias=case["bias"])
+    inp = make_inputs(sh, 4)
+    x, Wg, W1, W3, W2, dy = (to_f64(inp[n], 1) for n in ("x", "Wg", "W1", "W3", "W2", "dy"))
+    kw = dict(k=sh.k, act=sh.act, gate_norm=sh.gate_norm, capacity_factor=sh.capacity_factor,
+              n_shared=sh.n_shared, choice_major=case["choice_major"],
+              aux_loss_coef=case["aux"])
+    f = mo.layer_forward(x, Wg, inp["bias"], W1, W3, W2, **kw)
+    g = mo.layer_backward(f, x, Wg, W1, W3, W2, dy)
+    s = mo.layer_by_expert(x, Wg, inp["bias"], W1, W3, W2, dy, **kw)
+    if case["cf"] is not None:
+        assert np.any(s["pos"] < 0)
+    for n in ("idx", "counts", "kept", "pos"):
+        assert np.array_equal(s[n], f[n]), n
+    assert np.allclose(s["y"], f["y"], rtol=0, atol=1e-12)
+    for n in ("dg", "dlogits", "dWg", "dx"):
+        assert np.allclose(s[n], g[n], rtol=0, atol=1e-12), n
+    s2 = mo.layer_by_expert(x, Wg, inp["bias"], W1, W3, W2, dy, with_dx=False, **kw)
+    assert s2["dx"] is None and np.array_equal(s2["dWg"], s["dWg"])
+    for e, (tt, jj, X, U, V, H, O) in f["cache"].items():
+        dO = dy[tt] if jj is None else f["g"][tt, jj][:, None] * dy[tt]
+        w3 = None if W3 is None else W3[e]
+        want = mo.expert_backward(X, U, V, H, dO, W1[e], w3, W2[e], sh.act)[0]
+        got = mo.expert_input_grad(X, U, V, H, dO, W1[e], w3, W2[e], sh.act)
+        assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
 def test_sampled_forms_equal_full_layer():
     from mixture_experts_layer_23_b200.configs import LayerShape, SWIGLU as SW
     from mixture_experts_layer_23_b200.synth import make_inputs, to_f64
@@ -387,6 +456,25 @@ def test_sampled_forms_equal_full_layer():
 
 def _planted(monkeypatch, name, fn):
     monkeypatch.setattr(mo, name, fn)
+
+
+def test_planted_gate_bias_dropped_is_caught(monkeypatch):
+    _planted(monkeypatch, "gate_logits", lambda x, Wg, bias: x @ Wg.T)   # forgets the bias
+    assert not pin_gate_bias_golden()
+
+
+def test_planted_gate_bias_misapplied_is_caught(monkeypatch):
+    def per_token(x, Wg, bias):          # adds b[t] to token t's logits instead of b[e] to e's
+        l = x @ Wg.T
+        return l if bias is None else l + np.asarray(bias)[:x.shape[0], None]
+
+    def subtracted(x, Wg, bias):
+        l = x @ Wg.T
+        return l if bias is None else l - np.asarray(bias)[None, :]
+    _planted(monkeypatch, "gate_logits", per_token)
+    assert not pin_gate_bias_golden()
+    _planted(monkeypatch, "gate_logits", subtracted)
+    assert not pin_gate_bias_golden()
 
 
 def test_planted_gelu_grad_missing_term_is_caught(monkeypatch):

@@ -83,6 +83,9 @@ SHAPES = [
                dtype=BF16, bias="zipf"),
     LayerShape("noalloc_small", T=700, d=64, E=8, k=2, d_ff=64, capacity_factor=1.25,
                dtype=FP32),
+    # choice-major drops keep one histogram layer per choice index in the array
+    LayerShape("noalloc_choice_major", T=2000, d=64, E=32, k=4, d_ff=64, capacity_factor=0.7,
+               dtype=BF16, bias="normal", choice_major=True),
 ]
 
 
@@ -99,11 +102,27 @@ def test_noalloc_dispatch_repeated_call_same_shape():
         _assert_same(L, ref, got, shape.E)
 
 
-def test_noalloc_dispatch_refuses_configs_beyond_its_array():
+def _refused(shape):
     from mixture_experts_layer_23_b200 import moe
-    big = LayerShape("too_big", T=1 << 20, d=64, E=256, k=2, d_ff=64, dtype=BF16)
-    cfg = moe.make_config(big)
+    cfg = moe.make_config(shape)
     fake = 1 << 20  # aligned, never dereferenced: the size check comes before any CUDA call
     st = moe.lib().moe_dispatch_noalloc(ctypes.byref(cfg), fake, fake, fake, fake, fake, fake,
                                         fake, fake, None)
-    assert st == 4  # MOE_ERR_WORKSPACE_TOO_SMALL
+    return st == 4  # MOE_ERR_WORKSPACE_TOO_SMALL
+
+
+# ceil(T / 256) * E = 256 * 256 = 65536 histogram entries: exactly the array in token order
+AT_LIMIT = LayerShape("noalloc_at_limit", T=65536, d=64, E=256, k=2, d_ff=64,
+                      capacity_factor=1.0, dtype=BF16)
+
+
+def test_noalloc_dispatch_refuses_configs_beyond_its_array():
+    assert _refused(LayerShape("too_big", T=1 << 20, d=64, E=256, k=2, d_ff=64, dtype=BF16))
+    # the same size in token order fits exactly; choice-major needs k layers of it, which do not
+    assert _refused(AT_LIMIT.with_(name="at_limit_choice_major", choice_major=True))
+    assert _refused(AT_LIMIT.with_(name="one_block_more", T=65536 + 1))
+
+
+def test_noalloc_dispatch_at_its_size_limit():
+    L, ref, got = _dispatch_both(AT_LIMIT, seed=21)
+    _assert_same(L, ref, got, AT_LIMIT.E)
