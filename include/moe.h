@@ -206,6 +206,37 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
                          void* dx, float* dWg, float* dW1, float* dW3, float* dW2, void* scratch,
                          moe_stream_t stream);
 
+/* The backward pass in its three steps, for callers that run the expert step elsewhere (expert
+ * parallelism: the experts' rows cross to the GPU that owns them and back, Ch.4 "All-to-All
+ * 通信模式" 二 and "专家并行与数据并行的结合" 三.3).  moe_layer_bwd is exactly
+ * moe_combine_bwd, then moe_expert_ffn_bwd on the ctx's row space, then moe_router_bwd, with
+ * dO and dXd kept in scratch.
+ *
+ * Step 4 backward, from the ctx of the matching forward: dg [T,k] and dlogits [T,E] (with the
+ * router's softmax backward and, when aux_loss_coef > 0, the load-balancing loss gradient) into
+ * scratch (moe_scratch_grad_offsets); dO [R,d] (the row space of ctx) receives g * dy at every kept
+ * row and zero at padding rows; shared experts' rows are not written (their dO is dy itself). */
+moe_status moe_combine_bwd(const moe_config_t* cfg, const void* ctx, const void* dy, void* dO,
+                           void* scratch, moe_stream_t stream);
+
+/* Step 3 backward over a row space with the layout of moe_expert_ffn (offsets [E+1] on the
+ * device, padding rows of dO and Xd zero): dXd [R,d] = the rows' input gradients, dW1, dW3
+ * [E_tot,F,d] and dW2 [E_tot,d,F] float (overwritten), from the forward's saved Gu, Gv, H.  dy and
+ * x (the shared experts' dO and input rows) may be NULL when n_shared == 0.  Uses scratch as
+ * moe_layer_bwd does (dU, dV). */
+moe_status moe_expert_ffn_bwd(const moe_config_t* cfg, const void* dO, const void* dy,
+                              const void* Xd, const void* x, const int32_t* offsets,
+                              const void* W1, const void* W3, const void* W2, const void* Gu,
+                              const void* Gv, const void* H, void* dXd, float* dW1, float* dW3,
+                              float* dW2, void* scratch, moe_stream_t stream);
+
+/* Steps 1-2 backward on the token side, after moe_combine_bwd on the same scratch:
+ * dWg [E,d] = dlogits^T x (float, overwritten) and dx [T,d] = dlogits Wg + the sum of each
+ * token's kept rows of dXd and its shared experts' rows (fixed order, no atomics). */
+moe_status moe_router_bwd(const moe_config_t* cfg, const void* ctx, const void* x, const void* Wg,
+                          const void* dXd, void* dx, float* dWg, void* scratch,
+                          moe_stream_t stream);
+
 /* Byte offset, inside scratch, of dg [T,k] float (dL/dg of each assignment, 0 if dropped) and
  * of dlogits [T,E] float, both valid after moe_layer_bwd until the scratch is reused. */
 moe_status moe_scratch_grad_offsets(const moe_config_t* cfg, size_t* dg_offset,

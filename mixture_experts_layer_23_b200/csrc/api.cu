@@ -195,28 +195,29 @@ static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const
 }
 
 // Expert FFN backward: dgrad through W2 and the activation, dgrad through W1 (and W3), then the
-// weight gradients; profiling phases 3..6 of the backward pass.
+// weight gradients; with phase_marks, the profiling events of backward phases 3..5 between them.
 static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, const void* Xd,
                              const void* x, const int32_t* offsets, const void* W1,
                              const void* W3, const void* W2, const void* Gu, const void* Gv,
                              const void* H, void* dU, void* dV, void* dXd, float* dW1, float* dW3,
-                             float* dW2, uint32_t* status, cudaStream_t st) {
+                             float* dW2, uint32_t* status, cudaStream_t st,
+                             bool phase_marks = false) {
   if (tc_supported(D)) {
     MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, status, st));
-    MOE_TRY(mark_bwd(3, st));
+    if (phase_marks) MOE_TRY(mark_bwd(3, st));
     MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
-    MOE_TRY(mark_bwd(4, st));
+    if (phase_marks) MOE_TRY(mark_bwd(4, st));
     MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, status, st));
-    MOE_TRY(mark_bwd(5, st));
+    if (phase_marks) MOE_TRY(mark_bwd(5, st));
     MOE_TRY(launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st));
     return MOE_OK;
   }
   MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, st));
-  MOE_TRY(mark_bwd(3, st));
+  if (phase_marks) MOE_TRY(mark_bwd(3, st));
   MOE_TRY(launch_dgrad_x_simt(D, dU, dV, offsets, W1, W3, dXd, st));
-  MOE_TRY(mark_bwd(4, st));
+  if (phase_marks) MOE_TRY(mark_bwd(4, st));
   MOE_TRY(launch_wgrad_w13_simt(D, dU, dV, Xd, x, offsets, dW1, dW3, st));
-  MOE_TRY(mark_bwd(5, st));
+  if (phase_marks) MOE_TRY(mark_bwd(5, st));
   MOE_TRY(launch_wgrad_w2_simt(D, H, dO, dy, offsets, dW2, st));
   return MOE_OK;
 }
@@ -392,6 +393,56 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace moe {
+
+// Pieces of the backward pass, shared by moe_layer_bwd and the per-step entry points.
+
+// Step 4 backward: dg, dlogits (and their bf16 copy for the tensor-core router backward) into
+// scratch, dO = g * dy into the caller's row-space buffer (padding rows zeroed).
+static moe_status bwd_combine(const Dims& D, const moe_layout_t& L, const ScratchLayout& S,
+                              const char* c, char* s, const void* dy, void* dO, cudaStream_t st) {
+  __nv_bfloat16* dl16 = S.dl16 ? (__nv_bfloat16*)(s + S.dl16) : nullptr;
+  return launch_combine_bwd(D, dy, c + L.ctx_O, (const int32_t*)(c + L.ctx_slot),
+                            (const float*)(c + L.ctx_topk_w), (const int32_t*)(c + L.ctx_topk_idx),
+                            (const float*)(c + L.ctx_logits), (const int32_t*)(c + L.ctx_kept),
+                            (const int32_t*)(c + L.ctx_offsets), (const int32_t*)(c + L.ctx_counts),
+                            (float*)(s + S.dg), (float*)(s + S.dlogits), dl16, dO, st);
+}
+
+// Router weight gradient dWg = dl^T x (tensor cores over token chunks for bf16 with d % 64 == 0,
+// else CUDA cores), both with fixed-order reductions.
+static moe_status bwd_router_wgrad(const Dims& D, const ScratchLayout& S, char* s, const void* x,
+                                   float* dWg, cudaStream_t st) {
+  float* part = (float*)(s + S.dWg_part);
+  if (S.dl16) {
+    int n_chunks = 0;
+    MOE_TRY(launch_router_wgrad_tc(D, (const __nv_bfloat16*)(s + S.dl16), x, part, &n_chunks,
+                                   (uint32_t*)(s + S.status), st));
+    return launch_router_wgrad_reduce(D, part, n_chunks, dWg, st);
+  }
+  return launch_router_wgrad(D, (const float*)(s + S.dlogits), x, part, dWg, st);
+}
+
+// Steps 1-2 backward on the token side: dx = dl Wg + the token's routed and shared dXd rows.
+static moe_status bwd_router_dx(const Dims& D, const moe_layout_t& L, const ScratchLayout& S,
+                                const char* c, char* s, const void* Wg, const void* dXd, void* dx,
+                                cudaStream_t st) {
+  const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
+  if (S.dl16) {
+    void* dxg = s + S.dxg;
+    MOE_TRY(launch_router_dx_tc(D, (const __nv_bfloat16*)(s + S.dl16), Wg, dxg,
+                                (uint32_t*)(s + S.status), st));
+    return launch_undispatch_gather(D, dxg, dXd, slot, dx, st);
+  }
+  return launch_undispatch(D, (const float*)(s + S.dlogits), Wg, dXd, slot, dx, st);
+}
+
+}  // namespace moe
+
+extern "C" {
+
 moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* dy, const void* x,
                          const void* Wg, const void* W1, const void* W3, const void* W2,
                          void* dx, float* dWg, float* dW1, float* dW3, float* dW2, void* scratch,
@@ -406,53 +457,67 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   cudaStream_t st = (cudaStream_t)stream;
   const char* c = (const char*)ctx;
   char* s = (char*)scratch;
-  const float* logits = (const float*)(c + L.ctx_logits);
-  const int32_t* idx = (const int32_t*)(c + L.ctx_topk_idx);
-  const float* w = (const float*)(c + L.ctx_topk_w);
-  const int32_t* kept = (const int32_t*)(c + L.ctx_kept);
-  const int32_t* offsets = (const int32_t*)(c + L.ctx_offsets);
-  const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
-  const void* Xd = c + L.ctx_Xd;
-  const void* Gu = c + L.ctx_Gu;
-  const void* Gv = L.ctx_Gv ? c + L.ctx_Gv : nullptr;
-  const void* H = c + L.ctx_H;
-  const void* O = c + L.ctx_O;
   void* dO = s + S.dO;
-  void* dU = s + S.dU;
-  void* dV = S.dV ? s + S.dV : nullptr;
   void* dXd = s + S.dXd;
-  float* dg = (float*)(s + S.dg);
-  float* dl = (float*)(s + S.dlogits);
-  float* part = (float*)(s + S.dWg_part);
   MOE_TRY(mark_bwd(0, st));
-  // bf16 with d a multiple of 64: both router-backward contractions run on the tensor cores
-  // from a bf16 copy of dlogits; otherwise CUDA-core kernels read the fp32 dlogits
-  const bool rtc = S.dl16 != 0;
-  __nv_bfloat16* dl16 = rtc ? (__nv_bfloat16*)(s + S.dl16) : nullptr;
-  const int32_t* counts = (const int32_t*)(c + L.ctx_counts);
-  MOE_TRY(launch_combine_bwd(D, dy, O, slot, w, idx, logits, kept, offsets, counts, dg, dl, dl16,
-                             dO, st));
+  MOE_TRY(bwd_combine(D, L, S, c, s, dy, dO, st));
   MOE_TRY(mark_bwd(1, st));
-  if (rtc) {
-    int n_chunks = 0;
-    MOE_TRY(launch_router_wgrad_tc(D, dl16, x, part, &n_chunks, (uint32_t*)(s + S.status), st));
-    MOE_TRY(launch_router_wgrad_reduce(D, part, n_chunks, dWg, st));
-  } else {
-    MOE_TRY(launch_router_wgrad(D, dl, x, part, dWg, st));
-  }
+  MOE_TRY(bwd_router_wgrad(D, S, s, x, dWg, st));
   MOE_TRY(mark_bwd(2, st));
-  MOE_TRY(expert_bwd(D, dO, dy, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, dU, dV, dXd, dW1, dW3, dW2,
-                     (uint32_t*)(s + S.status), st));
+  MOE_TRY(expert_bwd(D, dO, dy, c + L.ctx_Xd, x, (const int32_t*)(c + L.ctx_offsets), W1, W3, W2,
+                     c + L.ctx_Gu, L.ctx_Gv ? c + L.ctx_Gv : nullptr, c + L.ctx_H, s + S.dU,
+                     S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, (uint32_t*)(s + S.status),
+                     st, /*phase_marks=*/true));
   MOE_TRY(mark_bwd(6, st));
-  if (rtc) {
-    void* dxg = s + S.dxg;
-    MOE_TRY(launch_router_dx_tc(D, dl16, Wg, dxg, (uint32_t*)(s + S.status), st));
-    MOE_TRY(launch_undispatch_gather(D, dxg, dXd, slot, dx, st));
-  } else {
-    MOE_TRY(launch_undispatch(D, dl, Wg, dXd, slot, dx, st));
-  }
+  MOE_TRY(bwd_router_dx(D, L, S, c, s, Wg, dXd, dx, st));
   MOE_TRY(mark_bwd(7, st));
   return MOE_OK;
+}
+
+moe_status moe_combine_bwd(const moe_config_t* cfg, const void* ctx, const void* dy, void* dO,
+                           void* scratch, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({ctx, dy, dO, scratch}));
+  moe_layout_t L;
+  ctx_layout(D, &L);
+  const ScratchLayout S = scratch_layout(D);
+  return bwd_combine(D, L, S, (const char*)ctx, (char*)scratch, dy, dO, (cudaStream_t)stream);
+}
+
+moe_status moe_expert_ffn_bwd(const moe_config_t* cfg, const void* dO, const void* dy,
+                              const void* Xd, const void* x, const int32_t* offsets,
+                              const void* W1, const void* W3, const void* W2, const void* Gu,
+                              const void* Gv, const void* H, void* dXd, float* dW1, float* dW3,
+                              float* dW2, void* scratch, moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({dO, Xd, offsets, W1, W2, Gu, H, dXd, dW1, dW2, scratch}));
+  if (D.S > 0) MOE_TRY(check_ptrs({dy, x}));
+  if (D.act == MOE_ACT_SWIGLU) MOE_TRY(check_ptrs({W3, Gv, dW3}));
+  const ScratchLayout S = scratch_layout(D);
+  char* s = (char*)scratch;
+  // with no shared experts dy and x are never read; any valid pointer stands in for them
+  const void* dy_ = D.S > 0 ? dy : dO;
+  const void* x_ = D.S > 0 ? x : Xd;
+  return expert_bwd(D, dO, dy_, Xd, x_, offsets, W1, W3, W2, Gu, Gv, H, s + S.dU,
+                    S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, (uint32_t*)(s + S.status),
+                    (cudaStream_t)stream);
+}
+
+moe_status moe_router_bwd(const moe_config_t* cfg, const void* ctx, const void* x, const void* Wg,
+                          const void* dXd, void* dx, float* dWg, void* scratch,
+                          moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  MOE_TRY(check_ptrs({ctx, x, Wg, dXd, dx, dWg, scratch}));
+  moe_layout_t L;
+  ctx_layout(D, &L);
+  const ScratchLayout S = scratch_layout(D);
+  cudaStream_t st = (cudaStream_t)stream;
+  char* s = (char*)scratch;
+  MOE_TRY(bwd_router_wgrad(D, S, s, x, dWg, st));
+  return bwd_router_dx(D, L, S, (const char*)ctx, s, Wg, dXd, dx, st);
 }
 
 int64_t moe_kernel_launches(void) {

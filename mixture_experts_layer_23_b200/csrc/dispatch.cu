@@ -7,18 +7,20 @@
 //
 // Ranking rule: within one expert, assignments are ordered by token index; the first C are kept
 // ("drop by token order").  The rank must be bit-exact and deterministic, so it is computed as a
-// stable counting sort in two launches, neither of which waits on another CTA:
+// stable counting sort in three launches, none of which waits on another CTA:
 //   1. rank:    each CTA takes 256 tokens; per warp, a shared-memory bitmask per expert marks the
 //               lanes (tokens) that chose it, so a popcount of the lower lanes gives each
 //               assignment's rank inside the warp; warp bases make it a rank inside the CTA.
 //               The CTA's per-expert histogram goes to scratch.  Choice-major priority
 //               (drop_order 1) repeats this per choice index j: k histogram layers, and each
 //               assignment's rank inside its CTA's layer.
-//   2. scatter: every CTA scans the histograms (exclusive over rank CTAs in token order, per
-//               expert; choice-major: over layers first, then rank CTAs) for its bases,
-//               kept = min(counts, C) and the 128-row aligned offsets;
-//               then one warp per token finalises its slots and copies its x row (16-byte
-//               vectors, read once, written to each kept slot); extra CTAs zero padding rows.
+//   2. scan:    one warp per expert turns its histogram column into exclusive bases (over rank
+//               CTAs in token order; choice-major: over layers first, then rank CTAs), in place,
+//               and writes counts and kept = min(counts, C);
+//   3. scatter: every CTA derives the 128-row aligned offsets from kept; one warp per token
+//               finalises its slots (its rank CTA's base + its rank inside the CTA) and copies its
+//               x row (16-byte vectors, read once, written to each kept slot); extra CTAs zero
+//               padding rows.
 #include <mutex>
 
 #include "common.cuh"
@@ -70,27 +72,57 @@ dispatch_rank_kernel(const int32_t* __restrict__ topk_idx, int T_, int E, int k,
   }
 }
 
-// Scan + scatter.  Every CTA first turns the per-rank-CTA histograms into what it needs: the
-// exclusive token-order base of its own tokens' rank-CTA for each expert, the per-expert totals
-// (counts), kept = min(counts, C) and the 128-row aligned segment offsets (CTA 0 also writes
-// counts, kept and offsets out).  This is E x n_blk integer adds per CTA, cheaper than a
-// separate one-CTA launch.  Then one warp per token finalises its slots and copies its x row
+// Scan: one warp per expert turns that expert's column of the rank CTAs' histograms into
+// exclusive bases in drop-priority order (token order: rank CTAs in order; choice-major: choice
+// layers first, then rank CTAs), in place, and writes counts (the total) and kept = min(counts, C).
+__global__ void __launch_bounds__(256)
+dispatch_scan_kernel(int32_t* __restrict__ blk /* in: block counts, out: exclusive bases */,
+                     int n_blk, int E, int L, int64_t C, int32_t* __restrict__ counts_out,
+                     int32_t* __restrict__ kept_out) {
+  pdl_prologue();
+  const int lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (e >= E) return;
+  const int n = n_blk * L;
+  int carry = 0;
+#pragma unroll 4
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int layer = i / n_blk, b = i - layer * n_blk;
+    const int64_t at = ((int64_t)b * L + layer) * E + e;
+    const int v = (i < n) ? blk[at] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (i < n) blk[at] = carry + incl - v;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    counts_out[e] = carry;
+    kept_out[e] = (int64_t)carry < C ? carry : (int)C;
+  }
+}
+
+// Scatter.  Every CTA turns kept into the 128-row aligned segment offsets (an exclusive prefix
+// over at most 256 experts; CTA 0 also writes them out).  Then one warp per token finalises its
+// slots (base of its rank CTA from the scan + its rank inside that CTA) and copies its x row
 // (16-byte vectors, read once, written to each kept slot); the last E + 1 CTAs zero the padding
 // rows and mark shared rows in row_token.
-constexpr int SC_TOK = 8;   // tokens per scatter CTA (one per warp)
+constexpr int SC_TOK = 32;   // tokens per scatter CTA (four per warp)
 static_assert(DT % SC_TOK == 0, "a scatter CTA must not straddle two rank CTAs");
 
 template <typename T, bool CM>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
-                        const int32_t* __restrict__ blk_counts, int n_blk, int T_, int d, int E,
-                        int k, int64_t C, int routed_row0, int n_tok_blocks, int shared_rows,
-                        int32_t* __restrict__ counts_out, int32_t* __restrict__ kept_out,
-                        int32_t* __restrict__ offsets_out,
+                        const int32_t* __restrict__ blk_base, const int32_t* __restrict__ kept,
+                        int T_, int d, int E, int k, int64_t C, int routed_row0, int n_tok_blocks,
+                        int shared_rows, int32_t* __restrict__ offsets_out,
                         int32_t* __restrict__ slot /* in: local rank, out: slot */,
                         int32_t* __restrict__ row_token, T* __restrict__ Xd) {
   pdl_prologue();
-  __shared__ int32_t s_base[8 * 256];   // base of this CTA's rank block per (layer,) expert
   __shared__ int32_t s_kept[256];
   __shared__ int32_t s_off[257];
   constexpr int VN = Vec16<T>::N;
@@ -100,20 +132,9 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
   const int my_blk = tok_cta ? (int)(blockIdx.x * SC_TOK / DT) : 0;
   const int L = CM ? k : 1;
   for (int e = threadIdx.x; e < E; e += 256) {
-    int run = 0;
-    for (int layer = 0; layer < L; ++layer) {   // layers in priority order, then rank CTAs
-      for (int b = 0; b < n_blk; ++b) {
-        if (b == my_blk) s_base[layer * 256 + e] = run;
-        run += blk_counts[((int64_t)b * L + layer) * E + e];
-      }
-    }
-    const int kp = (int64_t)run < C ? run : (int)C;
+    const int kp = kept[e];
     s_kept[e] = kp;
     s_off[e + 1] = (int)round_up(kp, MOE_ROW_ALIGN);
-    if (blockIdx.x == 0) {
-      counts_out[e] = run;
-      kept_out[e] = kp;
-    }
   }
   __syncthreads();
   if (warp == 0) {  // exclusive prefix of the segment sizes
@@ -158,7 +179,10 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
     if (lane < k) {
       const int e = topk_idx[(int64_t)t * k + lane];
       const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
-      const int pos = valid ? s_base[(CM ? lane : 0) * 256 + e] + slot[(int64_t)t * k + lane] : 0;
+      const int layer = CM ? lane : 0;
+      const int pos = valid ? blk_base[((int64_t)my_blk * L + layer) * E + e] +
+                                  slot[(int64_t)t * k + lane]
+                            : 0;
       if (valid && (int64_t)pos < C) {
         my_slot = s_off[e] + pos;
         row_token[my_slot] = t;
@@ -169,7 +193,7 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
 #pragma unroll
     for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
     const T* src = x + (int64_t)t * d;
-#pragma unroll 4
+#pragma unroll 8
     for (int v = lane; v < nv; v += 32) {
       const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
 #pragma unroll
@@ -187,12 +211,14 @@ static moe_status dispatch_t(const Dims& D, const void* x, const int32_t* topk_i
                              int32_t* row_token, void* Xd, int32_t* blk_counts, cudaStream_t st) {
   MOE_TRY_S(launch_k(dispatch_rank_kernel<CM>, D.n_blk, 256, 0, st, 1, topk_idx, D.T, D.E, D.k,
                      blk_counts, slot));
+  MOE_TRY_S(launch_k(dispatch_scan_kernel, (D.E + 7) / 8, 256, 0, st, 1, blk_counts, D.n_blk, D.E,
+                     D.n_layers, D.C, counts, kept));
   const int n_tok_blocks = (D.T + SC_TOK - 1) / SC_TOK;
   const int grid = n_tok_blocks + D.E + 1;
   return launch_k(dispatch_scatter_kernel<T, CM>, grid, 256, 0, st, 1, (const T*)x, topk_idx,
-                  (const int32_t*)blk_counts, D.n_blk, D.T, D.d, D.E, D.k, D.C,
-                  (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, counts, kept, offsets,
-                  slot, row_token, (T*)Xd);
+                  (const int32_t*)blk_counts, (const int32_t*)kept, D.T, D.d, D.E, D.k, D.C,
+                  (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, offsets, slot, row_token,
+                  (T*)Xd);
 }
 
 moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,

@@ -25,7 +25,8 @@ EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_
            "moe_scratch_grad_offsets", "moe_read_status", "moe_status_string", "moe_gemm_engine",
            "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
            "moe_last_cuda_error", "moe_aux_loss", "moe_layer_fwd_fused",
-           "moe_set_wait_budget_ns", "moe_set_wait_stall")
+           "moe_set_wait_budget_ns", "moe_set_wait_stall", "moe_combine_bwd",
+           "moe_expert_ffn_bwd", "moe_router_bwd")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -88,6 +89,9 @@ def _load():
         "moe_last_cuda_error": [],
         "moe_set_wait_budget_ns": [ctypes.c_uint64],
         "moe_set_wait_stall": [I32],
+        "moe_combine_bwd": [CP, P, P, P, P, P],
+        "moe_expert_ffn_bwd": [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
+        "moe_router_bwd": [CP, P, P, P, P, P, P, P, P],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -225,6 +229,24 @@ def layer_bwd(cfg, ctx, dy, x, Wg, W1, W3, W2, dx, dWg, dW1, dW3, dW2, scratch, 
     _check(_lib.moe_layer_bwd(ctypes.byref(cfg), _p(ctx), _p(dy), _p(x), _p(Wg), _p(W1), _p(W3),
                               _p(W2), _p(dx), _p(dWg), _p(dW1), _p(dW3), _p(dW2), _p(scratch),
                               _stream(stream)), "moe_layer_bwd")
+
+
+def combine_bwd(cfg, ctx, dy, dO, scratch, stream=None):
+    _check(_lib.moe_combine_bwd(ctypes.byref(cfg), _p(ctx), _p(dy), _p(dO), _p(scratch),
+                                _stream(stream)), "moe_combine_bwd")
+
+
+def expert_ffn_bwd(cfg, dO, dy, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, dXd, dW1, dW3, dW2,
+                   scratch, stream=None):
+    _check(_lib.moe_expert_ffn_bwd(ctypes.byref(cfg), _p(dO), _p(dy), _p(Xd), _p(x), _p(offsets),
+                                   _p(W1), _p(W3), _p(W2), _p(Gu), _p(Gv), _p(H), _p(dXd),
+                                   _p(dW1), _p(dW3), _p(dW2), _p(scratch), _stream(stream)),
+           "moe_expert_ffn_bwd")
+
+
+def router_bwd(cfg, ctx, x, Wg, dXd, dx, dWg, scratch, stream=None):
+    _check(_lib.moe_router_bwd(ctypes.byref(cfg), _p(ctx), _p(x), _p(Wg), _p(dXd), _p(dx),
+                               _p(dWg), _p(scratch), _stream(stream)), "moe_router_bwd")
 
 
 def read_status(scratch, stream=None) -> int:

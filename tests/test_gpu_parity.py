@@ -371,3 +371,41 @@ def test_step_entry_points_compose_to_the_layer():
     torch.cuda.synchronize()
     assert torch.equal(y, y_ref)
     assert torch.equal(slot, layer.view("slot"))
+
+
+@pytest.mark.parametrize("shape", [PARITY_SMALL[4], PARITY_SMALL[1], PARITY_FP32[1]],
+                         ids=lambda s: s.name)
+def test_backward_steps_compose_to_the_layer(shape):
+    """combine_bwd -> expert_ffn_bwd -> router_bwd on the forward's ctx equals moe_layer_bwd bit
+    for bit (tensor-core and CUDA-core paths, with and without shared experts)."""
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import MoELayer, to_device
+    inp = make_inputs(shape, 2)
+    dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).cuda()
+    layer = MoELayer(shape)
+    layer.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"])
+    layer.backward(dev["dy"], dev["x"], dev["Wg"], dev["W1"], dev["W3"], dev["W2"])
+    assert layer.status() == moe.MOE_OK
+    cfg, L, dt = layer.cfg, layer.L, layer.dt
+    R, T, d, E, F, Et = L.rows, shape.T, shape.d, shape.E, shape.d_ff, shape.E_tot
+    dO = torch.zeros(R, d, dtype=dt, device="cuda")
+    dXd = torch.zeros(R, d, dtype=dt, device="cuda")
+    dx = torch.empty(T, d, dtype=dt, device="cuda")
+    dWg = torch.empty(E, d, device="cuda")
+    dW1, dW2 = torch.empty(Et, F, d, device="cuda"), torch.empty(Et, d, F, device="cuda")
+    dW3 = torch.empty(Et, F, d, device="cuda") if shape.act == SWIGLU else None
+    scratch = torch.zeros(L.scratch_bytes, dtype=torch.uint8, device="cuda")
+    gv = layer.view("Gv") if shape.act == SWIGLU else None
+    moe.combine_bwd(cfg, layer.ctx, dev["dy"], dO, scratch)
+    moe.expert_ffn_bwd(cfg, dO, dev["dy"], layer.view("Xd"), dev["x"], layer.view("offsets"),
+                       dev["W1"], dev["W3"], dev["W2"], layer.view("Gu"), gv, layer.view("H"), dXd,
+                       dW1, dW3, dW2, scratch)
+    moe.router_bwd(cfg, layer.ctx, dev["x"], dev["Wg"], dXd, dx, dWg, scratch)
+    assert moe.read_status(scratch) == moe.MOE_OK
+    assert torch.equal(dx, layer.dx)
+    assert torch.equal(dWg, layer.dWg)
+    assert torch.equal(dW1, layer.dW1) and torch.equal(dW2, layer.dW2)
+    if dW3 is not None:
+        assert torch.equal(dW3, layer.dW3)
