@@ -27,8 +27,13 @@ namespace tc {
 namespace {
 
 constexpr int MAX_RSTAGES = 16;
-constexpr size_t RSMEM_BUDGET = 200 * 1024;   // stage ring bytes
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
+constexpr int SPLIT_MAX_EPAD = 64;            // split-K clusters reduce rows of at most 64 logits
+
+// Shared memory per CTA: a whole-d CTA keeps up to ~200 KB of loads in flight; the CTAs of a
+// split-K cluster stay within 112 KB so that two of them share an SM.
+constexpr size_t RSMEM_WHOLE = 226 * 1024;
+constexpr size_t RSMEM_SPLIT = 112 * 1024;
 
 struct alignas(64) RouterParams {
   CUtensorMap x_map;  // x [T, d], box {64, 128}
@@ -42,16 +47,42 @@ struct alignas(64) RouterParams {
   int T, d, E, E_pad, k, gate_norm;
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages;
+  int n_ks;           // CTAs per cluster, each contracting d / n_ks of the 128-token tile
   int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
 };
 
+__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void epi_bar() {   // the 128 epilogue threads (warps 2..5)
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+// One cluster of n_ks CTAs per 128-token tile; CTA r of the cluster contracts the k blocks
+// [r nk / n_ks, (r + 1) nk / n_ks).  With n_ks > 1 (at most 64 experts) every CTA parks its
+// partial logits in shared memory and the cluster's first CTA adds the others' partials to its
+// own in rank order (a fixed order: bit-reproducible) before the softmax and top-k.  Logits,
+// expert ids and gate weights are staged in shared memory and leave as contiguous rows.
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
   pdl_prologue();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const int RSTAGES = P.nstages;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RSTAGES * P.stage_bytes);
+  const bool split = P.n_ks > 1;
+  const bool small = P.E_pad <= SPLIT_MAX_EPAD;   // rows staged in shared memory
+  const int PS = P.E_pad + 1;                     // staging row stride (floats): no bank conflicts
+  float* part = reinterpret_cast<float*>(smem + RSTAGES * P.stage_bytes);   // [128][PS]
+  int32_t* sidx = reinterpret_cast<int32_t*>(part + (small ? 128 * PS : 0));  // [128][9]
+  float* sw = reinterpret_cast<float*>(sidx + 128 * 9);                     // [128][9]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sw + 128 * 9);
   uint64_t* full = bars;
   uint64_t* empty = bars + RSTAGES;
   uint64_t* tfull = bars + 2 * RSTAGES;
@@ -60,6 +91,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int crank = split ? (int)cluster_ctarank() : 0;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < RSTAGES; ++i) {
@@ -75,8 +107,10 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int m0 = blockIdx.x * 128;
-  const int nk = P.d / 64;
+  const int m0 = (blockIdx.x / P.n_ks) * 128;
+  const int nk_all = P.d / 64;
+  const int kb0 = crank * nk_all / P.n_ks, kb1 = (crank + 1) * nk_all / P.n_ks;
+  const int nk = kb1 - kb0;
   const unsigned long long budget = P.timeout_ns;
 
   uint32_t outstanding = 0, out_phase = 0;   // producer: stages loaded and not seen consumed
@@ -88,8 +122,8 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       outstanding &= ~(1u << stage);
       mbar_expect_tx(&full[stage], P.stage_bytes);
       uint8_t* sA = smem + stage * P.stage_bytes;
-      tma_load_2d(sA, &P.x_map, &full[stage], kb * 64, m0);
-      tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], kb * 64, 0);
+      tma_load_2d(sA, &P.x_map, &full[stage], (kb0 + kb) * 64, m0);
+      tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], (kb0 + kb) * 64, 0);
       outstanding |= 1u << stage;
       out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
@@ -119,13 +153,84 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       volatile int never = 0;
       wait_bounded(drain, 0, &never, 20000000ull);
     }
-  } else if (warp >= 2) {
-    const int quarter = warp & 3;
-    if (wait_bounded(tfull, 0, abort_flag, budget)) {
-      __syncwarp();
-      tc_fence_after();
-      const int t = m0 + quarter * 32 + lane;
-      const bool live = t < P.T;
+  }
+
+  // ---- epilogue: warps 2..5, one token (TMEM lane) per thread
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;          // token row inside the tile
+  const int t = m0 + row;
+  const bool epi = warp >= 2;
+  bool have = false;                             // this warp holds its accumulator rows
+  float acc[SPLIT_MAX_EPAD];
+  if (epi) {
+    // warp-uniform: the TMEM loads below need the whole warp
+    have = __all_sync(0xffffffffu, wait_bounded(tfull, 0, abort_flag, budget));
+  }
+  if (have) {
+    tc_fence_after();
+    if (small) {
+      const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll
+      for (int c = 0; c < SPLIT_MAX_EPAD / 16; ++c) {
+        if (c * 16 < P.E_pad) {
+          float v[16];
+          tmem_ld16(ta + (uint32_t)(c * 16), v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[c * 16 + i] = v[i];
+        }
+      }
+      if (split && crank != 0)
+        for (int e = 0; e < P.E; ++e) part[row * PS + e] = acc[e];
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  if (split) cluster_sync();   // #1: every CTA's roles are done; partials and abort flags visible
+
+  if (epi && crank == 0) {
+    // a placeholder routing (experts 0..k-1, weight 0, logits 0) when any wait of the tile ran
+    // out, so that the kernels after this one stay in bounds; the status word reports it
+    bool ok = have && !*abort_flag;
+    if (split)
+      for (int r = 1; r < P.n_ks; ++r)
+        ok = ok && ld_cluster_s32(mapa_shared(smem_u32((const void*)abort_flag), r)) == 0;
+    const bool live = t < P.T;
+    if (small) {
+      TopK8 st;
+      topk_init(st);
+      for (int e = 0; e < P.E; ++e) {
+        float l = 0.f;
+        if (ok) {
+          l = acc[e];
+          for (int r = 1; r < P.n_ks; ++r)   // partials of the other CTAs, in rank order
+            l += ld_cluster_f32(mapa_shared(smem_u32(&part[row * PS + e]), r));
+          l += P.bias ? P.bias[e] : 0.f;
+        }
+        part[row * PS + e] = l;
+        topk_push(st, l, e);
+      }
+      int32_t* oi = sidx + row * 9;
+      float* ow = sw + row * 9;
+      if (ok) {
+        topk_finish(st, P.k, P.gate_norm, oi, ow);
+      } else {
+        for (int j = 0; j < P.k; ++j) {
+          oi[j] = j;
+          ow[j] = 0.f;
+        }
+      }
+      epi_bar();
+      // the tile's rows are contiguous in logits, topk_idx and topk_w: coalesced stores
+      const int nrow = min(128, P.T - m0);
+      const int tid = threadIdx.x - 64;
+      for (int i = tid; i < nrow * P.E; i += 128)
+        P.logits[(size_t)m0 * P.E + i] = part[(i / P.E) * PS + i % P.E];
+      for (int i = tid; i < nrow * P.k; i += 128) {
+        P.topk_idx[(size_t)m0 * P.k + i] = sidx[(i / P.k) * 9 + i % P.k];
+        P.topk_w[(size_t)m0 * P.k + i] = sw[(i / P.k) * 9 + i % P.k];
+      }
+    } else if (ok) {
+      // wide rows (more than 64 experts, never split): stream them out of TMEM 16 at a time
       TopK8 st;
       topk_init(st);
       float v[16];
@@ -144,23 +249,18 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       if (live)
         topk_finish(st, P.k, P.gate_norm, P.topk_idx + (size_t)t * P.k,
                     P.topk_w + (size_t)t * P.k);
-    } else {
-      // the accumulator never arrived (a wait ran out): write a well-formed placeholder routing
-      // (experts 0..k-1, weight 0, logits 0) so the kernels after this one stay in bounds; the
-      // status word reports the timeout
-      const int t = m0 + quarter * 32 + lane;
-      if (t < P.T) {
-        for (int e = 0; e < P.E; ++e) P.logits[(size_t)t * P.E + e] = 0.f;
-        for (int j = 0; j < P.k; ++j) {
-          P.topk_idx[(size_t)t * P.k + j] = j;
-          P.topk_w[(size_t)t * P.k + j] = 0.f;
-        }
+    } else if (live) {
+      for (int e = 0; e < P.E; ++e) P.logits[(size_t)t * P.E + e] = 0.f;
+      for (int j = 0; j < P.k; ++j) {
+        P.topk_idx[(size_t)t * P.k + j] = j;
+        P.topk_w[(size_t)t * P.k + j] = 0.f;
       }
     }
   }
   __syncwarp();
+  if (split) cluster_sync();   // #2: the first CTA has read the others' partials
   tc_fence_before();
-  __syncthreads();   // every role has finished (the abort flag is final)
+  __syncthreads();             // every role has finished (the abort flag is final)
   if (*abort_flag && warp == 0 && lane == 0) {
     // TMA loads of an aborted CTA may still be in flight: let them land before it exits
     for (int s = 0; s < RSTAGES; ++s)
@@ -211,13 +311,32 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   while ((int)cols < E_pad) cols <<= 1;
   P.tmem_cols = cols;
   P.stage_bytes = RA_BYTES + (uint32_t)E_pad * 128u;
-  P.nstages = (int)std::min<size_t>(std::min<size_t>(MAX_RSTAGES, RSMEM_BUDGET / P.stage_bytes),
-                                    (size_t)(D.d / 64));
-  const size_t smem = 1024 + (size_t)P.nstages * P.stage_bytes + 512;
-  if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return launch_k(router_tc_kernel, (D.T + 127) / 128, 192, smem, st, 1, P);
+  // Split the contraction over a cluster when the token tiles alone leave the GPU short of CTAs:
+  // the smallest power-of-two split (at most 8) that brings the grid to two CTAs per SM, each
+  // keeping at least two k blocks.
+  const int n_tiles = (D.T + 127) / 128;
+  const int nk = D.d / 64;
+  int n_ks = 1;
+  if (E_pad <= SPLIT_MAX_EPAD)
+    while (n_ks < 8 && n_tiles * n_ks < 2 * num_sms() && nk / (2 * n_ks) >= 2) n_ks *= 2;
+  P.n_ks = n_ks;
+  const int nk_cta = (nk + n_ks - 1) / n_ks;
+  const size_t stage_rows = E_pad <= SPLIT_MAX_EPAD ? (size_t)128 * (E_pad + 1) * 4 : 0;
+  // alignment slack, staged rows, expert ids and weights, barriers (2 per stage + 2), TMEM slot
+  const size_t fixed = 1024 + stage_rows + 2 * 128 * 9 * 4 + 2 * 8 + 16;
+  const size_t budget = n_ks > 1 ? RSMEM_SPLIT : RSMEM_WHOLE;
+  const size_t fit = (budget - fixed) / (P.stage_bytes + 2 * 8);
+  P.nstages = (int)std::max<size_t>(
+      1, std::min<size_t>(std::min<size_t>(MAX_RSTAGES, fit), (size_t)nk_cta));
+  const size_t smem = fixed + (size_t)P.nstages * (P.stage_bytes + 2 * 8);
+  static int smem_set = 0;
+  if ((int)smem > smem_set) {
+    if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    smem_set = (int)smem;
+  }
+  return launch_k(router_tc_kernel, n_tiles * n_ks, 192, smem, st, n_ks, P);
 }
 
 }  // namespace moe
