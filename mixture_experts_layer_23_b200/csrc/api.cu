@@ -122,11 +122,8 @@ ScratchLayout scratch_layout(const Dims& D) {
   S.dg = take(T * D.k * 4);
   S.dlogits = take(T * D.E * 4);
   S.dWg_part = take((size_t)D.n_tchunk * D.E * D.d * 4);
-  S.dl16 = S.dxg = 0;
-  if (router_bwd_tc_supported(D)) {
-    S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
-    S.dxg = take(T * D.d * 2);
-  }
+  S.dl16 = 0;
+  if (router_bwd_tc_supported(D)) S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
   S.aux_part = take((size_t)D.n_aux * D.E * 4);
   S.total = off;
   return S;
@@ -430,12 +427,9 @@ static moe_status bwd_router_dx(const Dims& D, const moe_layout_t& L, const Scra
                                 const char* c, char* s, const void* Wg, const void* dXd, void* dx,
                                 cudaStream_t st) {
   const int32_t* slot = (const int32_t*)(c + L.ctx_slot);
-  if (S.dl16) {
-    void* dxg = s + S.dxg;
-    MOE_TRY(launch_router_dx_tc(D, (const __nv_bfloat16*)(s + S.dl16), Wg, dxg,
-                                (uint32_t*)(s + S.status), st));
-    return launch_undispatch_gather(D, dxg, dXd, slot, dx, st);
-  }
+  if (S.dl16)
+    return launch_undispatch_tc(D, (const __nv_bfloat16*)(s + S.dl16), Wg, dXd, slot, dx,
+                                (uint32_t*)(s + S.status), st);
   return launch_undispatch(D, (const float*)(s + S.dlogits), Wg, dXd, slot, dx, st);
 }
 

@@ -28,7 +28,6 @@ struct ScratchLayout {
   size_t dlogits;       // [T, E] float
   size_t dWg_part;      // [n_tchunk, E, d] float
   size_t dl16;          // [T, E8] bf16 copy of dlogits (tensor-core router backward), or 0
-  size_t dxg;           // [T, d] bf16 dl Wg (tensor-core router backward), or 0
   size_t aux_part;      // [n_aux, E] float partial probability sums of the load-balancing loss
   size_t total;
 };

@@ -63,7 +63,13 @@ constexpr int TILE_GROUP_M = 16;  // m tiles per band of the tile order (see dec
 constexpr uint32_t SLOT_BYTES = 32 * 128;
 constexpr size_t MISC_BYTES = 1536;   // barriers, TMEM slot, abort flag, tile prefix
 
-enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4 };
+enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4, UNDISPATCH = 5 };
+
+// UNDISPATCH epilogue gathers: per epilogue warp, buffers of 32 rows x 64 bf16 columns, one
+// 128-byte bulk copy per row, rows 144 bytes apart (16-byte reads of a row by 8 lanes at a time hit
+// 8 distinct bank groups).
+constexpr uint32_t GROW = 144;
+constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 
 // Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
 // up-projection's activation epilogue is the heaviest per output, so it gets 8 epilogue warps (two
@@ -78,15 +84,19 @@ template <int KIND>
 struct Cfg {
   static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
   static constexpr int SPLIT = EPI_WARPS / 4;   // epilogue warps per TMEM lane quarter
-  static constexpr int STAGES = (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4 : 6;
+  // UNDISPATCH contracts K = E (at most 4 k blocks): two stages are plenty, and the room goes to
+  // the gather buffers of its epilogue
+  static constexpr int STAGES = (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4 : (KIND == UNDISPATCH) ? 2 : 6;
   static constexpr int NIN = (KIND == DGRAD_H) ? 4 : 0;   // epilogue input slots per warp
+  static constexpr int NGATH = (KIND == UNDISPATCH) ? 6 : 0;   // epilogue gather buffers per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NSLOT = 2;                          // output staging slots per warp
   static constexpr uint32_t RING_BYTES = EPI_WARPS * NSLOT * SLOT_BYTES;
   static constexpr uint32_t IN_BYTES = EPI_WARPS * NIN * SLOT_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN;
+  static constexpr uint32_t GATH_BYTES = EPI_WARPS * NGATH * GATHER_BUF_BYTES;
+  static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN + EPI_WARPS * NGATH;
   static constexpr size_t SMEM_BYTES =
-      1024 + STAGES * STAGE_BYTES + RING_BYTES + IN_BYTES + MISC_BYTES;
+      1024 + STAGES * STAGE_BYTES + RING_BYTES + IN_BYTES + GATH_BYTES + MISC_BYTES;
   static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
   static_assert(8 * NBARS + 16 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc too small");
 };
@@ -109,6 +119,10 @@ struct alignas(64) Params {
                          // backward) instead of the experts' row ranges
   int stall;             // failure-path test: the MMA issuer first waits on a barrier that
                          // nothing arrives on, so the wait runs out and the CTA aborts
+  // UNDISPATCH: the rows its epilogue gathers and adds
+  const __nv_bfloat16* gsrc;   // dXd [rows, gd]
+  const int32_t* gslot;        // slot [T, gk]: routed row of each assignment, -1 if dropped
+  int gk, gS, gd;              // routed choices, shared experts (rows s * T_pad + t), row length
 };
 
 // Instruction descriptor of the pair MMA: bf16 x bf16 -> fp32, M = 256 (two CTAs), N = BN.
@@ -229,7 +243,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 #pragma unroll
     for (int j = 0; j < BNH / 64; ++j)
       tma_load_3d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, k0, t.g);
-  } else if (KIND == DGRAD_X) {
+  } else if (KIND == DGRAD_X || KIND == UNDISPATCH) {
     const int nkF = P.K / BK;
     const bool second = kb >= nkF;
     const int kk = (second ? kb - nkF : kb) * BK;
@@ -269,6 +283,13 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 // swizzle (16-byte unit c of row r lands at unit c ^ (r % 8): conflict-free), the warp fences the
 // writes into the async proxy, and lane 0 hands the 32 x 128 B box to a TMA store.  Stores that
 // fall outside the tensor (a partial last N tile) are clipped by TMA.
+
+// A bounded wait taken by a whole warp: every lane returns the same answer (the warp goes on only
+// when all its lanes saw the phase complete), so the warp never splits between success and abort.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long budget) {
+  return __all_sync(0xffffffffu, wait_bounded(bar, parity, abort_flag, budget));
+}
 
 template <int NSLOT>
 struct Ring {
@@ -344,7 +365,7 @@ template <int NIN>
 __device__ __forceinline__ const uint8_t* in_wait(InRing& r, volatile int* abort_flag,
                                                   unsigned long long budget) {
   const int j = r.consumed;
-  if (!wait_bounded(&r.bars[j % NIN], (uint32_t)(j / NIN) & 1u, abort_flag, budget))
+  if (!warp_wait(&r.bars[j % NIN], (uint32_t)(j / NIN) & 1u, abort_flag, budget))
     return nullptr;   // still counted as in flight: the exit path waits for it
   ++r.consumed;
   return r.base + (j % NIN) * SLOT_BYTES;
@@ -435,14 +456,14 @@ template <int KIND>
 __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
                                               int q, int sub, int lane,
                                               Ring<Cfg<KIND>::NSLOT>& ring,
-                                              InRing& inr, int tcount, uint64_t* tfull,
+                                              InRing& inr, InRing& gr, int tcount, uint64_t* tfull,
                                               uint32_t parity, volatile int* abort_flag) {
   constexpr int SPLIT = Cfg<KIND>::SPLIT;
   const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
   const bool swiglu = P.act == MOE_ACT_SWIGLU;
   float a[64];
   if (KIND == WGRAD) {
-    if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+    if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
     if (!t.live) return true;  // this CTA's half of the pair tile lies past the weight rows
@@ -486,7 +507,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
       if (swiglu) in_issue<NIN>(inr, &P.i1, n, row0, lane);
     };
     for (int i = 0; i < nch && i < depth; ++i) issue_chunk(i);
-    if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+    if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
 #pragma unroll 1
@@ -530,7 +551,79 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     }
     return true;
   }
-  if (!wait_bounded(tfull, parity, abort_flag, P.timeout_ns)) return false;
+  if constexpr (KIND == UNDISPATCH) {
+    // dx = dl Wg (the accumulator) + the token's kept routed rows of dXd (choices 0..k-1) + its
+    // shared experts' rows, summed in that fixed order.  The rows are gathered as 128-byte bulk
+    // copies (one per lane: the lane's token, one 64-column chunk, one source) into the warp's
+    // gather buffers, up to NGATH ahead; the first ones are issued before the wait for the
+    // accumulator, so the gathers overlap the MMAs.
+    constexpr int NG = Cfg<KIND>::NGATH;
+    const int nsrc = P.gk + P.gS;
+    const int tok = row0 + lane;
+    const bool live_row = t.live && tok < P.T;
+    int src[16];   // gathered row of each source, -1 when there is none (dropped, or past T)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      int r = -1;
+      if (j < nsrc && live_row)
+        r = (j < P.gk) ? P.gslot[(size_t)tok * P.gk + j] : (int)((j - P.gk) * P.T_pad + tok);
+      src[j] = r;
+    }
+    int nch = 0;
+    if (t.live)
+      for (int ch = 0; ch < BN / 64 && t.n * BN + ch * 64 < P.N; ++ch) ++nch;
+    const int total = nch * nsrc;
+    auto g_issue = [&](int i) {   // the i-th gather of this tile: chunk i / nsrc, source i % nsrc
+      const int ch = i / nsrc, j = i - ch * nsrc;
+      const int b = gr.issued % NG;
+      uint8_t* buf = gr.base + b * GATHER_BUF_BYTES;
+      const int r = src[j];
+      const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
+      fence_async_smem();   // this lane's earlier reads of its row before the copy rewrites it
+      __syncwarp();
+      if (lane == 0) mbar_expect_tx(&gr.bars[b], 128u * (uint32_t)__popc(m));
+      __syncwarp();
+      if (r >= 0)
+        bulk_g2s(buf + lane * GROW, P.gsrc + (size_t)r * P.gd + t.n * BN + ch * 64, 128u,
+                 &gr.bars[b]);
+      ++gr.issued;
+    };
+    int next = 0;
+    for (; next < total && next < NG; ++next) g_issue(next);
+    if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
+    __syncwarp();
+    tc_fence_after();
+#pragma unroll 1
+    for (int ch = 0; ch < nch; ++ch) {
+      const int n = t.n * BN + ch * 64;
+      tmem_ld64(tl + ch * 64, a);
+#pragma unroll 1
+      for (int j = 0; j < nsrc; ++j) {
+        const int b = gr.consumed % NG;
+        if (!warp_wait(&gr.bars[b], (uint32_t)(gr.consumed / NG) & 1u, abort_flag,
+                       P.timeout_ns))
+          return false;   // still counted as in flight: the exit path waits for it
+        ++gr.consumed;
+        if (src[j] >= 0) {
+          const uint8_t* row = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float v[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c * 16), v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) a[8 * c + i] += v[i];
+          }
+        }
+        __syncwarp();   // every lane has read this buffer before it is refilled
+        if (next < total) g_issue(next++);
+      }
+      uint8_t* slot = ring_take(ring, lane);
+      slot_put_bf16(slot, lane, a);
+      ring_store_2d(&P.o0, slot, n, row0, lane);
+    }
+    return true;
+  }
+  if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
   __syncwarp();
   tc_fence_after();
   if (!t.live) return true;  // this CTA's half of the pair tile lies past the group's rows
@@ -655,14 +748,17 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   uint8_t* ring_base = smem + STAGES * STAGE_BYTES;            // epilogue warps x NSLOT slots
   constexpr int NIN = Cfg<KIND>::NIN;
   uint8_t* in_base = ring_base + RING_BYTES;                     // epilogue warps x NIN slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(in_base + Cfg<KIND>::IN_BYTES);
+  constexpr int NG = Cfg<KIND>::NGATH;
+  uint8_t* g_base = in_base + Cfg<KIND>::IN_BYTES;               // epilogue warps x NG buffers
+  uint64_t* bars = reinterpret_cast<uint64_t*>(g_base + Cfg<KIND>::GATH_BYTES);
   uint64_t* full = bars;                 // [STAGES]  (the leader's are the ones used)
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
   uint64_t* tempty = tfull + 2;          // [2]       (the leader's are the ones used)
   uint64_t* drain = tempty + 2;          // [1]
   uint64_t* in_bars = drain + 1;         // [EPI_WARPS * NIN]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(in_bars + NUM_EPI_WARPS * NIN);
+  uint64_t* g_bars = in_bars + NUM_EPI_WARPS * NIN;   // [EPI_WARPS * NG]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(g_bars + NUM_EPI_WARPS * NG);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tile_start = reinterpret_cast<int*>(tmem_slot + 4);   // [MAX_GROUPS + 1]
 
@@ -691,6 +787,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     }
     mbar_init(drain, 1);
     for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
+    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -716,7 +813,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   const int n_tiles = tile_start[n_groups];
   const unsigned long long budget = P.timeout_ns;
   constexpr bool A_MN = (KIND == WGRAD);
-  constexpr bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == WGRAD);
+  constexpr bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == WGRAD || KIND == UNDISPATCH);
   constexpr uint32_t IDESC = make_idesc(A_MN, B_MN);
 
   // producer bookkeeping, read again after every role has finished (abort drain)
@@ -792,6 +889,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     const int sub = (warp - 2) >> 2;   // which of the quarter's SPLIT warps
     Ring<Cfg<KIND>::NSLOT> ring{ring_base + (warp - 2) * Cfg<KIND>::NSLOT * SLOT_BYTES, 0};
     InRing inr{in_base + (warp - 2) * NIN * SLOT_BYTES, in_bars + (warp - 2) * NIN, 0, 0};
+    InRing gr{g_base + (warp - 2) * NG * GATHER_BUF_BYTES, g_bars + (warp - 2) * NG, 0, 0};
     const uint32_t tempty_leader[2] = {mapa_shared(smem_u32(&tempty[0]), 0),
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0, tcount = 0;
@@ -800,7 +898,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, sub, lane,
-                               ring, inr, tcount, &tfull[acc], acc_phase, abort_flag))
+                               ring, inr, gr, tcount, &tfull[acc], acc_phase, abort_flag))
         break;
       tc_fence_before();
       __syncwarp();
@@ -812,6 +910,11 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     for (int j = inr.consumed; j < inr.issued; ++j) {
       volatile int never = 0;
       wait_bounded(&inr.bars[j % (NIN > 0 ? NIN : 1)], (uint32_t)(j / (NIN > 0 ? NIN : 1)) & 1u,
+                   &never, 20000000ull);
+    }
+    for (int j = gr.consumed; j < gr.issued; ++j) {
+      volatile int never = 0;
+      wait_bounded(&gr.bars[j % (NG > 0 ? NG : 1)], (uint32_t)(j / (NG > 0 ? NG : 1)) & 1u,
                    &never, 20000000ull);
     }
     __syncwarp();
@@ -1003,7 +1106,8 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
 // fixed token chunks as its groups:
 //   dWg partials  (WGRAD form): part[c] = dl16[chunk c]^T x[chunk c]  -> [n_chunks, E, d] fp32,
 //                 M = E, N = d, K = the chunk's tokens; summed over c in order afterwards
-//   dl Wg         (DGRAD_X form): dxg = dl16 Wg -> [T, d] bf16, one chunk of all T rows, K = E
+//   dl Wg         (DGRAD_X form, UNDISPATCH epilogue): dx = dl16 Wg + the gathered dXd rows, one
+//                 chunk of all T rows, K = E
 
 bool router_bwd_tc_supported(const Dims& D) {
   return D.dtype == MOE_DTYPE_BF16 && D.d % 64 == 0 && tc::encoder() != nullptr;
@@ -1034,22 +1138,32 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
   return launch<WGRAD>(P, nc * n_tiles, st);
 }
 
-moe_status launch_router_dx_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
-                               void* dxg, uint32_t* status, cudaStream_t st) {
+// dx = dl16 Wg + the token's kept routed rows of dXd + its shared experts' rows, in one launch:
+// the DGRAD_X-form contraction over one chunk of all T rows (K = E), whose epilogue gathers and
+// adds the rows (UNDISPATCH), so dl Wg never goes through memory.
+moe_status launch_undispatch_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
+                                const void* dXd, const int32_t* slot, void* dx, uint32_t* status,
+                                cudaStream_t st) {
   using namespace tc;
   Params P = base_params(D, nullptr, status);
   P.act = MOE_ACT_GELU;   // one operand pair per K block (not the SwiGLU pair of DGRAD_X)
   const int E8 = (int)round_up(D.E, 8);
   if (!(map2(&P.a_main, dl16, E8, D.T, 64, BM) && map3(&P.b_main, Wg, D.d, D.E, 1, 64, 64) &&
-        map2(&P.o0, dxg, D.d, D.T, 64, 32)))
+        map2(&P.o0, dx, D.d, D.T, 64, 32)))
     return MOE_ERR_CUDA;
+  if (D.k + D.S > 16) return MOE_ERR_UNSUPPORTED;
   P.E = 1;
-  P.S = 0;
+  P.S = 0;                 // one token chunk is the only group
   P.chunk = (int)round_up(D.T, BK);
   P.N = D.d;
   P.K = (int)round_up(D.E, BK);
+  P.gsrc = (const __nv_bfloat16*)dXd;
+  P.gslot = slot;
+  P.gk = D.k;
+  P.gS = D.S;
+  P.gd = D.d;
   const int tiles = (int)(((D.T + BMP - 1) / BMP) * ((D.d + BN - 1) / BN));
-  return launch<DGRAD_X>(P, tiles, st);
+  return launch<UNDISPATCH>(P, tiles, st);
 }
 
 }  // namespace moe

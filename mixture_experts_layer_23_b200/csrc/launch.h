@@ -24,7 +24,7 @@ moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, cons
                               float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
                               cudaStream_t st);
 // Router backward on the tensor cores (bf16, d a multiple of 64): dWg partials over token
-// chunks, their fixed-order sum, dl Wg, and the un-dispatch gather that adds it.
+// chunks and their fixed-order sum; dl Wg with the un-dispatch gather fused into its epilogue.
 bool router_bwd_tc_supported(const Dims& D);
 // One-launch forward of small layers (inference): routing recomputed per CTA, no ctx.
 bool fused_small_supported(const Dims& D);
@@ -39,10 +39,9 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
                                   float* part, int* n_chunks, uint32_t* status, cudaStream_t st);
 moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,
                                       cudaStream_t st);
-moe_status launch_router_dx_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
-                               void* dxg, uint32_t* status, cudaStream_t st);
-moe_status launch_undispatch_gather(const Dims& D, const void* dxg, const void* dXd,
-                                    const int32_t* slot, void* dx, cudaStream_t st);
+moe_status launch_undispatch_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
+                                const void* dXd, const int32_t* slot, void* dx, uint32_t* status,
+                                cudaStream_t st);
 moe_status launch_router_wgrad(const Dims& D, const float* dlogits, const void* x, float* part,
                                float* dWg, cudaStream_t st);
 moe_status launch_undispatch(const Dims& D, const float* dlogits, const void* Wg, const void* dXd,

@@ -280,82 +280,7 @@ undispatch_warp_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
   }
 }
 
-// Un-dispatch when dl Wg comes precomputed (tensor-core path): dx = dxg + routed rows j = 0..k-1
-// + (sum of shared rows), one warp per token, U = 8 / KR vectors per lane with all loads in flight.
-template <typename T, int KR>
-__global__ void __launch_bounds__(256)
-undispatch_gather_kernel(const T* __restrict__ dxg, const T* __restrict__ dXd,
-                         const int32_t* __restrict__ slot, int T_, int d, int k, int S,
-                         int64_t T_pad, T* __restrict__ dx) {
-  pdl_prologue();
-  constexpr int VN = Vec16<T>::N;
-  constexpr int U = KR >= 8 ? 1 : 8 / KR;
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T_) return;
-  int my_s = -1;
-  if (lane < k)
-    my_s = slot[(int64_t)t * k + lane];
-  else if (lane < k + S)
-    my_s = (int)((int64_t)(lane - k) * T_pad + t);
-  int s[KR];
-#pragma unroll
-  for (int j = 0; j < KR; ++j) {
-    s[j] = __shfl_sync(0xffffffffu, my_s, j);
-    if (j >= k + S) s[j] = -1;
-  }
-  const int nv = d / VN;
-  for (int v0 = lane; v0 < nv; v0 += 32 * U) {
-    Vec16<T> g0[U], g[U][KR];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = v0 + 32 * u;
-      if (v < nv) {
-        g0[u] = ld_vec_stream(dxg + (int64_t)t * d + (int64_t)v * VN);
-#pragma unroll
-        for (int j = 0; j < KR; ++j)
-          if (s[j] >= 0) g[u][j] = ld_vec_stream(dXd + (int64_t)s[j] * d + (int64_t)v * VN);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int v = v0 + 32 * u;
-      if (v >= nv) break;
-      Vec16<T> out;
-#pragma unroll
-      for (int i = 0; i < VN; ++i) {
-        float r = g0[u].get(i), sh = 0.f;
-#pragma unroll
-        for (int j = 0; j < KR; ++j)
-          if (s[j] >= 0) {
-            if (j < k) r += g[u][j].get(i);
-            else sh += g[u][j].get(i);
-          }
-        out.set(i, r + sh);
-      }
-      st_vec(dx + (int64_t)t * d + (int64_t)v * VN, out);
-    }
-  }
-}
-
 }  // namespace
-
-template <int KR>
-static moe_status undispatch_gather_t(const Dims& D, const void* dxg, const void* dXd,
-                                      const int32_t* slot, void* dx, cudaStream_t st) {
-  using T = __nv_bfloat16;
-  return launch_k(undispatch_gather_kernel<T, KR>, (D.T + 7) / 8, 256, 0, st, 1, (const T*)dxg,
-                  (const T*)dXd, slot, D.T, D.d, D.k, D.S, D.T_pad, (T*)dx);
-}
-
-moe_status launch_undispatch_gather(const Dims& D, const void* dxg, const void* dXd,
-                                    const int32_t* slot, void* dx, cudaStream_t st) {
-  const int r = D.k + D.S;
-  if (r <= 2) return undispatch_gather_t<2>(D, dxg, dXd, slot, dx, st);
-  if (r <= 4) return undispatch_gather_t<4>(D, dxg, dXd, slot, dx, st);
-  if (r <= 8) return undispatch_gather_t<8>(D, dxg, dXd, slot, dx, st);
-  return undispatch_gather_t<16>(D, dxg, dXd, slot, dx, st);
-}
 
 moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,
                                       cudaStream_t st) {
