@@ -1101,41 +1101,13 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
 //
 // The router's two backward contractions are GEMMs worth the tensor cores (2 T E d FLOPs each;
 // 4.3 GFLOP for T = 16384, E = 64, d = 2048; measured faster than the CUDA-core kernels from
-// E = 16 up, by 2x at E = 32).  Both read a bf16 copy of
-// dlogits, dl16 [T, E8] (E8 = E rounded up to 8, zero padded), and reuse the grouped kernel with
-// fixed token chunks as its groups:
-//   dWg partials  (WGRAD form): part[c] = dl16[chunk c]^T x[chunk c]  -> [n_chunks, E, d] fp32,
-//                 M = E, N = d, K = the chunk's tokens; summed over c in order afterwards
-//   dl Wg         (DGRAD_X form, UNDISPATCH epilogue): dx = dl16 Wg + the gathered dXd rows, one
-//                 chunk of all T rows, K = E
+// E = 16 up, by 2x at E = 32).  Both read a bf16 copy of dlogits, dl16 [T, E8] (E8 = E rounded up
+// to 8, zero padded).  dl Wg reuses the grouped kernel with all T rows as one group (DGRAD_X form,
+// UNDISPATCH epilogue): dx = dl16 Wg + the gathered dXd rows, K = E.  (The weight gradient dWg has
+// its own kernel next to the router's, router_tc.cu.)
 
 bool router_bwd_tc_supported(const Dims& D) {
   return D.dtype == MOE_DTYPE_BF16 && D.d % 64 == 0 && tc::encoder() != nullptr;
-}
-
-moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
-                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st) {
-  using namespace tc;
-  Params P = base_params(D, nullptr, status);
-  const int E8 = (int)round_up(D.E, 8);
-  if (!(map2(&P.a_main, dl16, E8, D.T, 64, 64) && map2(&P.b_main, x, D.d, D.T, 64, 64)))
-    return MOE_ERR_CUDA;
-  const int n_tiles = (int)(((D.E + BMP - 1) / BMP) * ((D.d + BN - 1) / BN));
-  // enough chunks to give every CTA pair a tile, within the partial buffer and the group table
-  int nc = (num_sms() / 2 + n_tiles - 1) / n_tiles;
-  nc = std::min(nc, std::min(D.n_tchunk, MAX_GROUPS));
-  nc = std::max(1, std::min<int>(nc, (int)((D.T + BK - 1) / BK)));
-  const int chunk = (int)round_up((D.T + nc - 1) / nc, BK);
-  nc = (D.T + chunk - 1) / chunk;
-  if (!map3_f32(&P.o0, part, D.d, D.E, nc, 32, 32)) return MOE_ERR_CUDA;
-  P.E = nc;
-  P.S = 0;
-  P.chunk = chunk;
-  P.Mw = D.E;
-  P.N = D.d;
-  P.which = 0;
-  *n_chunks = nc;
-  return launch<WGRAD>(P, nc * n_tiles, st);
 }
 
 // dx = dl16 Wg + the token's kept routed rows of dXd + its shared experts' rows, in one launch:

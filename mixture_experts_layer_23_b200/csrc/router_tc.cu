@@ -277,6 +277,141 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   }
 }
 
+// ----------------------------------------------------------------------------- router weight gradient
+//
+// dWg = dl^T x, computed as its transpose dWg^T = x^T dl so that the long side, d, is the MMA's M:
+// each CTA takes 128 columns of d (M = 128, x read MN-major) and one chunk of tokens (K), against
+// every expert at once (N = E rounded up to 64, dl16 read MN-major, one 64-expert swizzle atom per
+// 64 experts).  The MMA work is then 2 d N T flops, a few percent of the time it takes to read x,
+// and x is read exactly once.  Each CTA writes its chunk's partial dWg[e][d] in fp32 (a warp's lanes
+// hold 32 consecutive columns: coalesced); router_wgrad_reduce adds the chunks in order.
+
+struct alignas(64) RWParams {
+  CUtensorMap x_map;   // x [T, d], box {64 (d), 64 (tokens)}
+  CUtensorMap l_map;   // dl16 [T, E8], box {64 (experts), 64 (tokens)}
+  float* part;         // [n_chunks][E][d]
+  uint32_t* status;
+  unsigned long long timeout_ns;
+  int T, d, E, N, chunk, n_dt;
+  uint32_t idesc, tmem_cols, stage_bytes;
+  int nstages, stall;
+};
+
+__global__ void __launch_bounds__(192, 1) router_wgrad_tc_kernel(const __grid_constant__ RWParams P) {
+  pdl_prologue();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const int RSTAGES = P.nstages;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + RSTAGES * P.stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + RSTAGES;
+  uint64_t* tfull = bars + 2 * RSTAGES;
+  uint64_t* drain = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int i = 0; i < RSTAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, P.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int dt = blockIdx.x % P.n_dt, c = blockIdx.x / P.n_dt;
+  const int d0 = dt * 128, t0 = c * P.chunk;
+  const int t1 = min(P.T, t0 + P.chunk);
+  const int nk = (t1 - t0 + 63) / 64;   // chunks are multiples of 64 tokens: only T ends one early
+  const unsigned long long budget = P.timeout_ns;
+
+  uint32_t outstanding = 0, out_phase = 0;   // producer: stages loaded and not seen consumed
+  if (warp == 0 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) break;
+      outstanding &= ~(1u << stage);
+      mbar_expect_tx(&full[stage], P.stage_bytes);
+      uint8_t* sA = smem + stage * P.stage_bytes;
+      uint8_t* sB = sA + 16384;
+      const int tk = t0 + kb * 64;
+      tma_load_2d(sA, &P.x_map, &full[stage], d0, tk);
+      tma_load_2d(sA + 8192, &P.x_map, &full[stage], d0 + 64, tk);
+      for (int j = 0; j < P.N / 64; ++j) tma_load_2d(sB + j * 8192, &P.l_map, &full[stage], 64 * j, tk);
+      outstanding |= 1u << stage;
+      out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
+      if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
+    }
+  } else if (warp == 1 && lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    bool issued = false, ok = true;
+    // test hook: `drain` gets no arrival before an abort, so this wait runs out after `budget`
+    if (P.stall && !wait_bounded(drain, 0u, abort_flag, budget)) ok = false;
+    for (int kb = 0; ok && kb < nk; ++kb) {
+      if (!wait_bounded(&full[stage], phase, abort_flag, budget)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sa = smem_u32(smem + stage * P.stage_bytes);
+      const uint32_t sb = sa + 16384;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)   // both operands MN-major: a K step of 16 rows is 2 KB
+        umma_bf16(tmem_base, sw128_desc(sa + k * 2048, 8192, 1024),
+                  sw128_desc(sb + k * 2048, 8192, 1024), P.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+      issued = true;
+      umma_commit(&empty[stage]);
+      if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
+    }
+    if (ok) umma_commit(tfull);
+    if (*abort_flag && issued) {
+      umma_commit(drain);
+      volatile int never = 0;
+      wait_bounded(drain, 0, &never, 20000000ull);
+    }
+  } else if (warp >= 2) {
+    const int quarter = warp & 3;
+    const int col = d0 + quarter * 32 + lane;   // this thread's TMEM lane = column of d
+    if (__all_sync(0xffffffffu, wait_bounded(tfull, 0, abort_flag, budget))) {
+      tc_fence_after();
+      float* out = P.part + (size_t)c * P.E * P.d;
+      for (int e0 = 0; e0 < P.E; e0 += 16) {
+        float v[16];
+        tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)e0, v);
+        if (col < P.d) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (e0 + i < P.E) out[(size_t)(e0 + i) * P.d + col] = v[i];
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();   // every role has finished (the abort flag is final)
+  if (*abort_flag && warp == 0 && lane == 0) {
+    // TMA loads of an aborted CTA may still be in flight: let them land before it exits
+    for (int s = 0; s < RSTAGES; ++s)
+      if (outstanding & (1u << s)) {
+        volatile int never = 0;
+        wait_bounded(&full[s], (out_phase >> s) & 1u, &never, 20000000ull);
+      }
+  }
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0 && P.status) atomicOr(P.status, MOE_STATUS_TIMEOUT);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, P.tmem_cols);
+  }
+}
+
 }  // namespace
 }  // namespace tc
 
@@ -337,6 +472,49 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
     smem_set = (int)smem;
   }
   return launch_k(router_tc_kernel, n_tiles * n_ks, 192, smem, st, n_ks, P);
+}
+
+moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
+                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st) {
+  using namespace tc;
+  RWParams P;
+  memset(&P, 0, sizeof(P));
+  const int E8 = (int)round_up(D.E, 8);
+  if (!map2(&P.x_map, x, D.d, D.T, 64, 64) || !map2(&P.l_map, dl16, E8, D.T, 64, 64))
+    return MOE_ERR_CUDA;
+  P.part = part;
+  P.status = status;
+  P.timeout_ns = tc::wait_budget_ns();
+  P.stall = tc::wait_stall();
+  P.T = D.T;
+  P.d = D.d;
+  P.E = D.E;
+  P.N = (int)round_up(D.E, 64);                 // 64..256
+  P.n_dt = (D.d + 127) / 128;
+  // token chunks: about two CTAs per SM in all, within the partial buffer (D.n_tchunk chunks)
+  int nc = (2 * num_sms() + P.n_dt - 1) / P.n_dt;
+  nc = std::max(1, std::min(nc, std::min(D.n_tchunk, (D.T + 63) / 64)));
+  P.chunk = (int)round_up((D.T + nc - 1) / nc, 64);
+  nc = (D.T + P.chunk - 1) / P.chunk;
+  P.idesc = idesc_bf16_m128(P.N, true, true);
+  uint32_t cols = 64;
+  while ((int)cols < P.N) cols <<= 1;
+  P.tmem_cols = cols;
+  P.stage_bytes = 16384u + (uint32_t)P.N * 128u;
+  const int nk_cta = P.chunk / 64;
+  const size_t fixed = 1024 + 2 * 8 + 16;
+  const size_t fit = (RSMEM_SPLIT - fixed) / (P.stage_bytes + 2 * 8);
+  P.nstages = (int)std::max<size_t>(1, std::min<size_t>(std::min<size_t>(8, fit), (size_t)nk_cta));
+  const size_t smem = fixed + (size_t)P.nstages * (P.stage_bytes + 2 * 8);
+  static int smem_set = 0;
+  if ((int)smem > smem_set) {
+    if (cudaFuncSetAttribute(router_wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    smem_set = (int)smem;
+  }
+  *n_chunks = nc;
+  return launch_k(router_wgrad_tc_kernel, P.n_dt * nc, 192, smem, st, 1, P);
 }
 
 }  // namespace moe
