@@ -206,6 +206,20 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
                          void* dx, float* dWg, float* dW1, float* dW3, float* dW2, void* scratch,
                          moe_stream_t stream);
 
+/* One training step of the layer from and to HOST memory: copies x and dy (host, ideally pinned)
+ * into the device buffers x_dev and dy_dev, runs moe_layer_fwd and moe_layer_bwd, and copies y and
+ * dx back into y_host and dx_host, all enqueued on `stream` (plain cudaMemcpyAsync, one per
+ * tensor).  Weights and weight gradients stay on the device.  Returns after enqueueing; the host
+ * buffers must stay valid until the stream has passed the step.  Two calls on two streams with
+ * separate buffers overlap one step's copies with the other's compute.  bias may be NULL when
+ * has_bias == 0; W3 and dW3 may be NULL for GELU. */
+moe_status moe_layer_step_host(const moe_config_t* cfg, const void* x_host, const void* dy_host,
+                               void* y_host, void* dx_host, void* x_dev, void* dy_dev,
+                               const void* Wg, const float* bias, const void* W1, const void* W3,
+                               const void* W2, void* y_dev, void* dx_dev, float* dWg, float* dW1,
+                               float* dW3, float* dW2, void* ctx, void* scratch,
+                               moe_stream_t stream);
+
 /* The backward pass in its three steps, for callers that run the expert step elsewhere (expert
  * parallelism: the experts' rows cross to the GPU that owns them and back, Ch.4 "All-to-All
  * 通信模式" 二 and "专家并行与数据并行的结合" 三.3).  moe_layer_bwd is exactly

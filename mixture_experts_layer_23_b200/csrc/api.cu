@@ -468,6 +468,36 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   return MOE_OK;
 }
 
+moe_status moe_layer_step_host(const moe_config_t* cfg, const void* x_host, const void* dy_host,
+                               void* y_host, void* dx_host, void* x_dev, void* dy_dev,
+                               const void* Wg, const float* bias, const void* W1, const void* W3,
+                               const void* W2, void* y_dev, void* dx_dev, float* dWg, float* dW1,
+                               float* dW3, float* dW2, void* ctx, void* scratch,
+                               moe_stream_t stream) {
+  Dims D;
+  MOE_TRY(resolve_dims(cfg, &D));
+  if (!x_host || !dy_host || !y_host || !dx_host) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_ptrs({x_dev, dy_dev, y_dev, dx_dev}));
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)D.T * D.d * D.elem;
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dy_dev, dy_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) {
+    note_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  MOE_TRY(moe_layer_fwd(cfg, x_dev, Wg, bias, W1, W3, W2, y_dev, ctx, scratch, stream));
+  MOE_TRY(moe_layer_bwd(cfg, ctx, dy_dev, x_dev, Wg, W1, W3, W2, dx_dev, dWg, dW1, dW3, dW2, scratch,
+                        stream));
+  e = cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dx_host, dx_dev, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) {
+    note_cuda_error(e);
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
 moe_status moe_combine_bwd(const moe_config_t* cfg, const void* ctx, const void* dy, void* dO,
                            void* scratch, moe_stream_t stream) {
   Dims D;

@@ -26,7 +26,7 @@ EXPORTS = ("moe_get_layout", "moe_workspace_size", "moe_route", "moe_route_from_
            "moe_kernel_launches", "moe_set_profile_events", "moe_dispatch_noalloc",
            "moe_last_cuda_error", "moe_aux_loss", "moe_layer_fwd_fused",
            "moe_set_wait_budget_ns", "moe_set_wait_stall", "moe_combine_bwd",
-           "moe_expert_ffn_bwd", "moe_router_bwd")
+           "moe_expert_ffn_bwd", "moe_router_bwd", "moe_layer_step_host")
 
 FWD_PHASES = ("router", "dispatch", "expert_up", "expert_down", "combine")
 BWD_PHASES = ("combine_bwd", "router_bwd", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2",
@@ -92,6 +92,7 @@ def _load():
         "moe_combine_bwd": [CP, P, P, P, P, P],
         "moe_expert_ffn_bwd": [CP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         "moe_router_bwd": [CP, P, P, P, P, P, P, P, P],
+        "moe_layer_step_host": [CP] + [P] * 20,
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -247,6 +248,16 @@ def expert_ffn_bwd(cfg, dO, dy, Xd, x, offsets, W1, W3, W2, Gu, Gv, H, dXd, dW1,
 def router_bwd(cfg, ctx, x, Wg, dXd, dx, dWg, scratch, stream=None):
     _check(_lib.moe_router_bwd(ctypes.byref(cfg), _p(ctx), _p(x), _p(Wg), _p(dXd), _p(dx),
                                _p(dWg), _p(scratch), _stream(stream)), "moe_router_bwd")
+
+
+def layer_step_host(cfg, x_host, dy_host, y_host, dx_host, x_dev, dy_dev, Wg, bias, W1, W3, W2,
+                    y_dev, dx_dev, dWg, dW1, dW3, dW2, ctx, scratch, stream=None):
+    """One forward + backward from pinned host x, dy to host y, dx (moe_layer_step_host)."""
+    _check(_lib.moe_layer_step_host(ctypes.byref(cfg), _p(x_host), _p(dy_host), _p(y_host),
+                                    _p(dx_host), _p(x_dev), _p(dy_dev), _p(Wg), _p(bias), _p(W1),
+                                    _p(W3), _p(W2), _p(y_dev), _p(dx_dev), _p(dWg), _p(dW1),
+                                    _p(dW3), _p(dW2), _p(ctx), _p(scratch), _stream(stream)),
+           "moe_layer_step_host")
 
 
 def read_status(scratch, stream=None) -> int:

@@ -409,3 +409,32 @@ def test_backward_steps_compose_to_the_layer(shape):
     assert torch.equal(dW1, layer.dW1) and torch.equal(dW2, layer.dW2)
     if dW3 is not None:
         assert torch.equal(dW3, layer.dW3)
+
+
+def test_step_from_host_buffers_matches_the_layer():
+    """moe_layer_step_host (host x, dy in; host y, dx out) gives moe_layer_fwd + moe_layer_bwd's
+    results bit for bit, on two calls in a row on one stream."""
+    import torch
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.layer import MoELayer, to_device
+    s = PARITY_SMALL[3]
+    ref = MoELayer(s)
+    got = MoELayer(s)
+    for seed in (4, 5):
+        inp = make_inputs(s, seed)
+        dev = {k: to_device(v, s) for k, v in inp.items() if k != "bias"}
+        ref.forward(dev["x"], dev["Wg"], None, dev["W1"], dev["W3"], dev["W2"])
+        ref.backward(dev["dy"], dev["x"], dev["Wg"], dev["W1"], dev["W3"], dev["W2"])
+        x_h = dev["x"].cpu().pin_memory()
+        dy_h = dev["dy"].cpu().pin_memory()
+        y_h = torch.empty_like(x_h).pin_memory()
+        dx_h = torch.empty_like(x_h).pin_memory()
+        x_d, dy_d = torch.empty_like(dev["x"]), torch.empty_like(dev["dy"])
+        moe.layer_step_host(got.cfg, x_h, dy_h, y_h, dx_h, x_d, dy_d, dev["Wg"], None, dev["W1"],
+                            dev["W3"], dev["W2"], got.y, got.dx, got.dWg, got.dW1, got.dW3,
+                            got.dW2, got.ctx, got.scratch)
+        torch.cuda.synchronize()
+        assert got.status() == moe.MOE_OK and ref.status() == moe.MOE_OK
+        assert torch.equal(y_h, ref.y.cpu()) and torch.equal(dx_h, ref.dx.cpu())
+        assert torch.equal(got.dWg, ref.dWg) and torch.equal(got.dW1, ref.dW1)
+        assert torch.equal(got.dW2, ref.dW2) and torch.equal(got.dW3, ref.dW3)
