@@ -321,19 +321,25 @@ def phase_work(shape, n_kept):
     rows = n_kept + S * T
     g = 2 if shape.act == 1 else 1
     Td, Nd = T * d * b, n_kept * d * b
+    # dlogits travel as fp32 on the CUDA-core path and as a bf16 copy (rows padded to 8) on the
+    # tensor-core path
+    dl = T * ((E + 7) // 8 * 8) * 2 if shape.dtype == 1 and d % 64 == 0 else T * E * 4
     return {
         "router": ("hbm", Td + E * d * b + T * E * 4 + T * k * 8),
         "dispatch": ("hbm", Td + Nd + T * k * 8 + (T * E * 4 if shape.aux_loss_coef else 0)),
         "expert_up": (mm, 2.0 * rows * d * F * g),
         "expert_down": (mm, 2.0 * rows * F * d),
-        "combine": ("hbm", Nd + S * Td + Td),
-        "combine_bwd": ("hbm", Td + 2 * Nd),
-        "router_bwd": ("hbm", Td + 2 * T * E * 4),
+        "combine": ("hbm", Nd + S * Td + Td + T * k * 8),
+        # read dy, the kept O rows and the logits; write dO rows, dg and the logit gradient
+        "combine_bwd": ("hbm", Td + 2 * Nd + T * E * 4 + T * k * 12 + dl),
+        # read x and the logit gradient, write dWg
+        "router_bwd": ("hbm", Td + dl + E * d * 4),
         "dgrad_h": (mm, 2.0 * rows * d * F),
         "dgrad_x": (mm, 2.0 * rows * F * d * g),
         "wgrad_w1": (mm, 2.0 * rows * F * d * g),
         "wgrad_w2": (mm, 2.0 * rows * d * F),
-        "undispatch": ("hbm", Nd + S * Td + Td),
+        # read the kept and shared dXd rows, the logit gradient and Wg; write dx
+        "undispatch": ("hbm", Nd + S * Td + Td + dl + E * d * b + T * k * 4),
     }
 
 
