@@ -101,6 +101,29 @@ def test_edge_shapes(shape):
     _parity().full_compare(shape, seed=3)
 
 
+EDGE_SPLIT = [
+    # the router's contraction split over a cluster of 8 CTAs (two k blocks each), ragged last tile
+    LayerShape("router_split8_ragged", T=700, d=1024, E=8, k=2, d_ff=64, capacity_factor=1.0,
+               dtype=BF16, bias="normal"),
+    # one token tile split 8 ways; fewer tokens than a tile
+    LayerShape("router_split8_one_tile", T=100, d=2048, E=16, k=2, d_ff=64, capacity_factor=2.0,
+               dtype=BF16),
+    # 64 experts (split router at its widest row), 6 routed + 2 shared rows gathered per token by
+    # the un-dispatch epilogue, router weight gradient with N = 64
+    LayerShape("router_split_e64_shared", T=1111, d=512, E=64, k=6, d_ff=64, n_shared=2,
+               act=SWIGLU, capacity_factor=1.25, dtype=BF16, bias="normal"),
+    # 200 experts (whole-d router), k = 8 with 8 shared experts: 16 gathered rows per token;
+    # router weight gradient with N = 256 and d = 192 (its second 128-column tile half outside d)
+    LayerShape("wide_e_max_gathers", T=600, d=192, E=200, k=8, d_ff=128, n_shared=8,
+               capacity_factor=2.0, dtype=BF16, bias="normal"),
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_SPLIT, ids=lambda s: s.name)
+def test_split_router_and_fused_backward_shapes(shape):
+    _parity().full_compare(shape, seed=4)
+
+
 AUX = [
     # load-balancing loss on: its value, and its gradient through dlogits into dx and dWg
     LayerShape("aux_gelu_drops", T=700, d=64, E=8, k=2, d_ff=96, capacity_factor=0.9,
