@@ -80,18 +80,27 @@ constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 // sub-partitions by warp index and each sub-partition has a quarter of the register file
 // (16384 registers): 10 warps put 3 on one sub-partition, capping threads at 168 registers;
 // 6 warps allow 255.
+#ifndef MOE_GEMM_DIRECT_STORE
+#define MOE_GEMM_DIRECT_STORE 0
+#endif
+
 template <int KIND>
 struct Cfg {
   static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
   static constexpr int SPLIT = EPI_WARPS / 4;   // epilogue warps per TMEM lane quarter
+  // plain-output kinds may store straight from registers, which frees the staging ring for a
+  // seventh stage of loads in flight
+  static constexpr bool DIRECT =
+      MOE_GEMM_DIRECT_STORE && (KIND == DOWN || KIND == DGRAD_X || KIND == WGRAD);
   // UNDISPATCH contracts K = E (at most 4 k blocks): two stages are plenty, and the room goes to
   // the gather buffers of its epilogue
-  static constexpr int STAGES = (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4 : (KIND == UNDISPATCH) ? 2 : 6;
+  static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4
+                                       : (KIND == UNDISPATCH) ? 2 : 6;
   static constexpr int NIN = (KIND == DGRAD_H) ? 4 : 0;   // epilogue input slots per warp
   static constexpr int NGATH = (KIND == UNDISPATCH) ? 6 : 0;   // epilogue gather buffers per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NSLOT = 2;                          // output staging slots per warp
-  static constexpr uint32_t RING_BYTES = EPI_WARPS * NSLOT * SLOT_BYTES;
+  static constexpr uint32_t RING_BYTES = DIRECT ? 0 : EPI_WARPS * NSLOT * SLOT_BYTES;
   static constexpr uint32_t IN_BYTES = EPI_WARPS * NIN * SLOT_BYTES;
   static constexpr uint32_t GATH_BYTES = EPI_WARPS * NGATH * GATHER_BUF_BYTES;
   static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN + EPI_WARPS * NGATH;
@@ -119,6 +128,8 @@ struct alignas(64) Params {
                          // backward) instead of the experts' row ranges
   int stall;             // failure-path test: the MMA issuer first waits on a barrier that
                          // nothing arrives on, so the wait runs out and the CTA aborts
+  void* out;              // the output's base and row stride (elements), for direct stores
+  long long out_ld;
   // UNDISPATCH: the rows its epilogue gathers and adds
   const __nv_bfloat16* gsrc;   // dXd [rows, gd]
   const int32_t* gslot;        // slot [T, gk]: routed row of each assignment, -1 if dropped
@@ -443,6 +454,22 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
   }
 }
 
+// Straight from registers to global memory: 64 bf16 / 32 fp32 values (128 bytes) of one row.
+__device__ __forceinline__ void st_row_bf16(void* base, long long ld, long long row, int col,
+                                            const float* v) {
+  uint4* p = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + row * ld + col);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    p[c] = make_uint4(pack_bf16(v[8 * c + 0], v[8 * c + 1]), pack_bf16(v[8 * c + 2], v[8 * c + 3]),
+                      pack_bf16(v[8 * c + 4], v[8 * c + 5]), pack_bf16(v[8 * c + 6], v[8 * c + 7]));
+}
+__device__ __forceinline__ void st_row_f32(void* base, long long ld, long long row, int col,
+                                           const float* v) {
+  float4* p = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + row * ld + col);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) p[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+
 // First chunk of warp `sub` (of `split` warps sharing a TMEM lane quarter) when `before` chunks
 // of the quarter were dealt before this tile: chunk c goes to warp (before + c) % split.
 __device__ __forceinline__ int q_sub_first(int sub, int before, int split) {
@@ -483,9 +510,13 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
 #pragma unroll
         for (int i = 0; i < 32; ++i) a[i] = 0.f;
       }
-      uint8_t* slot = ring_take(ring, lane);
-      slot_put_f32(slot, lane, a);
-      ring_store_3d(&P.o0, slot, n, m_row0, t.g, lane);
+      if constexpr (Cfg<KIND>::DIRECT) {
+        st_row_f32(P.out, P.out_ld, (long long)t.g * P.Mw + m_row0 + lane, n, a);
+      } else {
+        uint8_t* slot = ring_take(ring, lane);
+        slot_put_f32(slot, lane, a);
+        ring_store_3d(&P.o0, slot, n, m_row0, t.g, lane);
+      }
     }
     return true;
   }
@@ -725,9 +756,13 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     const int n = t.n * BN + ch * 64;
     if (n >= P.N) break;
     tmem_ld64(tl + ch * 64, a);
-    uint8_t* slot = ring_take(ring, lane);
-    slot_put_bf16(slot, lane, a);
-    ring_store_2d(&P.o0, slot, n, row0, lane);
+    if constexpr (Cfg<KIND>::DIRECT) {
+      st_row_bf16(P.out, P.out_ld, row0 + lane, n, a);
+    } else {
+      uint8_t* slot = ring_take(ring, lane);
+      slot_put_bf16(slot, lane, a);
+      ring_store_2d(&P.o0, slot, n, row0, lane);
+    }
   }
   return true;
 }
@@ -1026,6 +1061,8 @@ moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* of
   if (!(map2(&P.a_main, H, D.F, D.R, 64, BM) && map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, BNH)))
     return MOE_ERR_CUDA;
   if (!map2(&P.o0, O, D.d, D.R, 64, 32)) return MOE_ERR_CUDA;
+  P.out = O;
+  P.out_ld = D.d;
   P.N = D.d;
   P.K = D.F;
   return launch<DOWN>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
@@ -1056,6 +1093,8 @@ moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, cons
     ok = ok && map2(&P.a_alt, dV, D.F, D.R, 64, BM) && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, 64);
   if (!ok) return MOE_ERR_CUDA;
   if (!map2(&P.o0, dXd, D.d, D.R, 64, 32)) return MOE_ERR_CUDA;
+  P.out = dXd;
+  P.out_ld = D.d;
   P.N = D.d;
   P.K = D.F;
   return launch<DGRAD_X>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
@@ -1071,6 +1110,8 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
           map2(&P.b_alt, x, D.d, D.T, 64, 64)))
       return MOE_ERR_CUDA;
     if (!map3_f32(&P.o0, pass ? dW3 : dW1, D.d, D.F, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
+    P.out = pass ? dW3 : dW1;
+    P.out_ld = D.d;
     P.Mw = D.F;
     P.N = D.d;
     P.which = 0;
@@ -1090,6 +1131,8 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, cons
         map2(&P.b_main, H, D.F, D.R, 64, 64)))
     return MOE_ERR_CUDA;
   if (!map3_f32(&P.o0, dW2, D.F, D.d, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
+  P.out = dW2;
+  P.out_ld = D.F;
   P.Mw = D.d;
   P.N = D.F;
   P.which = 2;
