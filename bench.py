@@ -87,6 +87,11 @@ def parse():
                     help="drop priority: all first choices, then second choices, ... (else token order)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism instead of replicas: each of the N ranks owns E/N "
+                         "experts and its own batch (layers without shared experts)")
+    ap.add_argument("--ep-chunks", type=int, default=1,
+                    help="expert groups per rank whose exchange overlaps the previous group's GEMMs")
     return ap.parse_args()
 
 
@@ -678,10 +683,86 @@ def run_ours(args):
     return 0
 
 
+def run_ep(args):
+    """Expert-parallel layer over the N ranks (mixture_experts_layer_23_b200.ep): every rank routes
+    its own batch of T tokens, owns E/N experts, and exchanges rows with the others through NCCL.
+    K steps timed with CUDA events after W warm-up steps, max over ranks; prints one JSON line."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29541")
+    dist.init_process_group("nccl", rank=rank, world_size=world, timeout=timedelta(seconds=120),
+                            device_id=dev)
+    from mixture_experts_layer_23_b200 import build as moe_build
+    moe_build.build()
+    from mixture_experts_layer_23_b200 import moe
+    from mixture_experts_layer_23_b200.ep import DistExchange, EPRank, step
+    from mixture_experts_layer_23_b200.layer import to_device
+    from mixture_experts_layer_23_b200.synth import make_inputs
+    shape = bench_shape(args)
+    El = shape.E // world
+    base = make_inputs(shape, 0, with_dy=False)
+    mine = make_inputs(shape, 100 + rank)
+    W = {n: to_device(base[n], shape, dev) for n in ("Wg", "W1", "W3", "W2")}
+    bias = None if base["bias"] is None else torch.from_numpy(base["bias"]).to(dev)
+    sl = slice(rank * El, (rank + 1) * El)
+    W1l, W2l = W["W1"][sl].contiguous(), W["W2"][sl].contiguous()
+    W3l = None if W["W3"] is None else W["W3"][sl].contiguous()
+    x, dy = to_device(mine["x"], shape, dev), to_device(mine["dy"], shape, dev)
+    F, d = shape.d_ff, shape.d
+    grads = (torch.empty(El, F, d, device=dev),
+             None if W3l is None else torch.empty(El, F, d, device=dev),
+             torch.empty(El, d, F, device=dev))
+    r = EPRank(shape, rank, world, device=dev, chunks=args.ep_chunks)
+    ex = DistExchange()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        step(r, ex, x, W["Wg"], bias, W1l, W3l, W2l, dy, grads)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(K):
+        starts[i].record(stream)
+        step(r, ex, x, W["Wg"], bias, W1l, W3l, W2l, dy, grads)
+        ends[i].record(stream)
+        flush.zero_()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    total_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, dev)
+    st = r.status()
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status: {moe.STATUS_NAMES.get(st, st)}")
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": job_tokens_per_s(world, shape.T, K, total_ms),
+            "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if shape.dtype == 1 else "f32",
+            "data": "synthetic",
+            "config": dict(workload_config(shape, world),
+                           parallelism=f"expert parallel x{world}, {El} experts per rank, "
+                                       f"{args.ep_chunks} exchange chunk(s)"),
+            "note": "expert-parallel mode: each step includes the host sync of the kept counts, "
+                    "the exchanges and the router-gradient all-reduce"}), flush=True)
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.ep:
+        return run_ep(args)
     return run_ours(args)
 
 
