@@ -584,9 +584,10 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   }
   if constexpr (KIND == UNDISPATCH) {
     // dx = dl Wg (the accumulator) + the token's kept routed rows of dXd (choices 0..k-1) + its
-    // shared experts' rows, summed in that fixed order.  The rows are gathered as 128-byte bulk
-    // copies (one per lane: the lane's token, one 64-column chunk, one source) into the warp's
-    // gather buffers, up to NGATH ahead; the first ones are issued before the wait for the
+    // shared experts' rows, summed in that fixed order.  Each lane gathers its token's 128 bytes
+    // (one 64-column chunk of one source row) with eight 16-byte asynchronous copies into the
+    // warp's gather buffers, up to NGATH buffers ahead, and the buffer's mbarrier completes when
+    // all 32 lanes' copies have landed; the first ones are issued before the wait for the
     // accumulator, so the gathers overlap the MMAs.
     constexpr int NG = Cfg<KIND>::NGATH;
     const int nsrc = P.gk + P.gS;
@@ -607,16 +608,14 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     auto g_issue = [&](int i) {   // the i-th gather of this tile: chunk i / nsrc, source i % nsrc
       const int ch = i / nsrc, j = i - ch * nsrc;
       const int b = gr.issued % NG;
-      uint8_t* buf = gr.base + b * GATHER_BUF_BYTES;
+      uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
       const int r = src[j];
-      const unsigned m = __ballot_sync(0xffffffffu, r >= 0);
-      fence_async_smem();   // this lane's earlier reads of its row before the copy rewrites it
-      __syncwarp();
-      if (lane == 0) mbar_expect_tx(&gr.bars[b], 128u * (uint32_t)__popc(m));
-      __syncwarp();
-      if (r >= 0)
-        bulk_g2s(buf + lane * GROW, P.gsrc + (size_t)r * P.gd + t.n * BN + ch * 64, 128u,
-                 &gr.bars[b]);
+      if (r >= 0) {
+        const __nv_bfloat16* g = P.gsrc + (size_t)r * P.gd + t.n * BN + ch * 64;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cp_async16(buf + 16 * c, g + 8 * c);
+      }
+      cp_async_arrive_noinc(&gr.bars[b]);   // every lane arrives once its own copies have landed
       ++gr.issued;
     };
     int next = 0;
@@ -822,7 +821,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     }
     mbar_init(drain, 1);
     for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
-    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 1);
+    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 32);   // one per lane
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);

@@ -29,6 +29,9 @@ namespace {
 constexpr int MAX_RSTAGES = 16;
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
 constexpr int SPLIT_MAX_EPAD = 64;            // split-K clusters reduce rows of at most 64 logits
+#ifndef MOE_ROUTER_MAX_SPLIT
+#define MOE_ROUTER_MAX_SPLIT 8                  // largest cluster a tile's contraction is split over
+#endif
 
 // Shared memory per CTA: a whole-d CTA keeps up to ~200 KB of loads in flight; the CTAs of a
 // split-K cluster stay within 112 KB so that two of them share an SM.
@@ -51,9 +54,11 @@ struct alignas(64) RouterParams {
   int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
 };
 
-__device__ __forceinline__ float ld_cluster_f32(uint32_t cluster_addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr));
   return v;
 }
 __device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
@@ -78,7 +83,9 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   const int RSTAGES = P.nstages;
   const bool split = P.n_ks > 1;
   const bool small = P.E_pad <= SPLIT_MAX_EPAD;   // rows staged in shared memory
-  const int PS = P.E_pad + 1;                     // staging row stride (floats): no bank conflicts
+  // staging row stride (floats): a multiple of 4 (16-byte rows for vector access) and an odd
+  // number of 16-byte units, so eight threads' 16-byte accesses to their rows hit distinct banks
+  const int PS = P.E_pad + 4 + ((P.E_pad / 4 + 1) % 2 == 0 ? 4 : 0);
   float* part = reinterpret_cast<float*>(smem + RSTAGES * P.stage_bytes);   // [128][PS]
   int32_t* sidx = reinterpret_cast<int32_t*>(part + (small ? 128 * PS : 0));  // [128][9]
   float* sw = reinterpret_cast<float*>(sidx + 128 * 9);                     // [128][9]
@@ -179,8 +186,13 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
           for (int i = 0; i < 16; ++i) acc[c * 16 + i] = v[i];
         }
       }
-      if (split && crank != 0)
-        for (int e = 0; e < P.E; ++e) part[row * PS + e] = acc[e];
+      if (split && crank != 0) {
+#pragma unroll
+        for (int e = 0; e < SPLIT_MAX_EPAD; e += 4)
+          if (e < P.E_pad)
+            *reinterpret_cast<float4*>(&part[row * PS + e]) =
+                make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+      }
     }
   }
   __syncwarp();
@@ -196,16 +208,37 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
         ok = ok && ld_cluster_s32(mapa_shared(smem_u32((const void*)abort_flag), r)) == 0;
     const bool live = t < P.T;
     if (small) {
+      if (ok && split) {
+        // add the other CTAs' partials in rank order, 16 logits at a time: all 16-byte DSMEM
+        // loads of a group are issued before the first add
+        const uint32_t my_row = smem_u32(&part[row * PS]);
+#pragma unroll 1
+        for (int e0 = 0; e0 < P.E_pad; e0 += 16) {
+          float4 q[7][4];
+#pragma unroll
+          for (int r = 1; r < 8; ++r)
+            if (r < P.n_ks) {
+              const uint32_t base = mapa_shared(my_row + 4u * e0, r);
+#pragma unroll
+              for (int u = 0; u < 4; ++u) q[r - 1][u] = ld_cluster_v4(base + 16u * u);
+            }
+#pragma unroll
+          for (int r = 1; r < 8; ++r)
+            if (r < P.n_ks) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                acc[e0 + 4 * u] += q[r - 1][u].x;
+                acc[e0 + 4 * u + 1] += q[r - 1][u].y;
+                acc[e0 + 4 * u + 2] += q[r - 1][u].z;
+                acc[e0 + 4 * u + 3] += q[r - 1][u].w;
+              }
+            }
+        }
+      }
       TopK8 st;
       topk_init(st);
       for (int e = 0; e < P.E; ++e) {
-        float l = 0.f;
-        if (ok) {
-          l = acc[e];
-          for (int r = 1; r < P.n_ks; ++r)   // partials of the other CTAs, in rank order
-            l += ld_cluster_f32(mapa_shared(smem_u32(&part[row * PS + e]), r));
-          l += P.bias ? P.bias[e] : 0.f;
-        }
+        const float l = ok ? acc[e] + (P.bias ? P.bias[e] : 0.f) : 0.f;
         part[row * PS + e] = l;
         topk_push(st, l, e);
       }
@@ -453,10 +486,11 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   const int nk = D.d / 64;
   int n_ks = 1;
   if (E_pad <= SPLIT_MAX_EPAD)
-    while (n_ks < 8 && n_tiles * n_ks < 2 * num_sms() && nk / (2 * n_ks) >= 2) n_ks *= 2;
+    while (n_ks < MOE_ROUTER_MAX_SPLIT && n_tiles * n_ks < 2 * num_sms() && nk / (2 * n_ks) >= 2)
+      n_ks *= 2;
   P.n_ks = n_ks;
   const int nk_cta = (nk + n_ks - 1) / n_ks;
-  const size_t stage_rows = E_pad <= SPLIT_MAX_EPAD ? (size_t)128 * (E_pad + 1) * 4 : 0;
+  const size_t stage_rows = E_pad <= SPLIT_MAX_EPAD ? (size_t)128 * (E_pad + 8) * 4 : 0;
   // alignment slack, staged rows, expert ids and weights, barriers (2 per stage + 2), TMEM slot
   const size_t fixed = 1024 + stage_rows + 2 * 128 * 9 * 4 + 2 * 8 + 16;
   const size_t budget = n_ks > 1 ? RSMEM_SPLIT : RSMEM_WHOLE;

@@ -36,16 +36,20 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="mixtral_dropless")
     ap.add_argument("--step", default="all",
-                    choices=["all", "route", "dispatch", "combine", "experts", "experts_bwd"])
+                    choices=["all", "route", "dispatch", "combine", "experts", "experts_bwd",
+                             "layer"])
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--E", type=int, default=None)
+    ap.add_argument("--F", type=int, default=None)
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     a = ap.parse_args(argv)
     shape = BY_NAME[a.workload]
-    if a.T or a.E:
+    if a.T or a.E or a.F:
         shape = shape.with_(name=shape.name + "_reduced", T=a.T or shape.T, E=a.E or shape.E,
-                            k=min(shape.k, a.E or shape.E))
+                            k=min(shape.k, a.E or shape.E), d_ff=a.F or shape.d_ff)
+    if a.step == "layer":
+        return run_layer(shape, a)
     gemm = a.step in ("experts", "experts_bwd")
     inp = make_inputs(shape, 0, with_dy=False)
     if not gemm:
@@ -124,7 +128,7 @@ def main(argv=None):
         "experts": (experts, 2.0 * rows * d * F * (g + 1)),
         "experts_bwd": (experts_bwd, 2.0 * rows * d * F * (2 * g + 2)),
     }
-    if "dispatch" in (a.step, "all") and not gemm:
+    if a.step in ("dispatch", "all") and not gemm:
         Xd = torch.empty(R, d, dtype=dt, device="cuda")   # for the dispatch runs below
     scratch_status = (lambda: moe.read_status(scratch)) if gemm else None
     for name, (fn, nbytes) in steps.items():
@@ -152,6 +156,37 @@ def main(argv=None):
         if scratch_status is not None:
             line["status"] = scratch_status()
         print(json.dumps(line), flush=True)
+
+
+def run_layer(shape, a):
+    """The whole layer, forward + backward (MoELayer), on the given shape: for captures of the
+    backward's HBM-bound kernels on a layer whose experts are shrunk (--F) to bound memory."""
+    from .layer import MoELayer
+    inp = make_inputs(shape, 0)
+    dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
+    bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).cuda()
+    layer = MoELayer(shape)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def step():
+        layer.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"])
+        layer.backward(dev["dy"], dev["x"], dev["Wg"], dev["W1"], dev["W3"], dev["W2"])
+
+    for _ in range(a.warmup):
+        step()
+        flush.zero_()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(a.iters)]
+    torch.cuda.synchronize()
+    for s_, e_ in ev:
+        s_.record()
+        step()
+        e_.record()
+        flush.zero_()
+    torch.cuda.synchronize()
+    us = 1e3 * sum(s_.elapsed_time(e_) for s_, e_ in ev) / a.iters
+    print(json.dumps({"workload": shape.name, "step": "layer", "us_per_step": us,
+                      "status": layer.status()}), flush=True)
 
 
 if __name__ == "__main__":
