@@ -83,6 +83,12 @@ constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 #ifndef MOE_GEMM_DIRECT_STORE
 #define MOE_GEMM_DIRECT_STORE 0
 #endif
+#ifndef MOE_DGRAD_H_STAGES
+#define MOE_DGRAD_H_STAGES 4   // load stages of the activation-gradient GEMM
+#endif
+#ifndef MOE_DGRAD_H_NIN
+#define MOE_DGRAD_H_NIN 4      // its epilogue input slots per warp
+#endif
 
 template <int KIND>
 struct Cfg {
@@ -94,9 +100,9 @@ struct Cfg {
       MOE_GEMM_DIRECT_STORE && (KIND == DOWN || KIND == DGRAD_X || KIND == WGRAD);
   // UNDISPATCH contracts K = E (at most 4 k blocks): two stages are plenty, and the room goes to
   // the gather buffers of its epilogue
-  static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? 5 : (KIND == DGRAD_H) ? 4
+  static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? 5 : (KIND == DGRAD_H) ? MOE_DGRAD_H_STAGES
                                        : (KIND == UNDISPATCH) ? 2 : 6;
-  static constexpr int NIN = (KIND == DGRAD_H) ? 4 : 0;   // epilogue input slots per warp
+  static constexpr int NIN = (KIND == DGRAD_H) ? MOE_DGRAD_H_NIN : 0;   // epilogue input slots per warp
   static constexpr int NGATH = (KIND == UNDISPATCH) ? 6 : 0;   // epilogue gather buffers per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NSLOT = 2;                          // output staging slots per warp
