@@ -485,11 +485,80 @@ __device__ __forceinline__ int q_sub_first(int sub, int before, int split) {
 // Warp (q, sub) covers rows 32q..32q+31 of the tile; with SPLIT > 1 warps per quarter (UP) it
 // takes the 64-column chunks q_sub_first deals to it.  Returns false if the wait for the
 // accumulator timed out.
+// The tiles of one CTA pair, for code that looks ahead to the pair's next tiles.
+struct Sched {
+  const int* tile_start;
+  int n_groups, n_tiles, n_pairs, rank;
+};
+
+// UNDISPATCH: one epilogue warp's stream of gathers, (tile, chunk, source) in the order its
+// epilogue consumes them, so that they can be issued ahead across tile boundaries.
+struct GCursor {
+  int t;          // tile (>= n_tiles: the stream has ended)
+  int ch, j;      // chunk and source inside the tile
+  int nch;        // 64-column chunks of the tile in this warp's rows (0: none)
+  int n0, row0;   // first column and first row of the warp's slab
+  int src[16];    // gathered row of each source for this lane's token, -1 when there is none
+};
+
+template <int KIND>
+__device__ __forceinline__ void gcursor_load(const Params& P, const Sched& S, int q, int lane,
+                                             GCursor& c) {
+  c.ch = 0;
+  c.j = 0;
+  c.nch = 0;
+  if (c.t >= S.n_tiles) return;
+  const Tile tl = decode<KIND>(P, S.tile_start, S.n_groups, c.t, S.rank);
+  c.row0 = tl.o_row + tl.mrow + q * 32;
+  c.n0 = tl.n * BN;
+  if (tl.live)
+    for (int ch = 0; ch < BN / 64 && c.n0 + ch * 64 < P.N; ++ch) ++c.nch;
+  const int tok = c.row0 + lane;
+  const bool live_row = tl.live && tok < P.T;
+  const int nsrc = P.gk + P.gS;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    int r = -1;
+    if (j < nsrc && live_row)
+      r = (j < P.gk) ? P.gslot[(size_t)tok * P.gk + j] : (int)((j - P.gk) * P.T_pad + tok);
+    c.src[j] = r;
+  }
+}
+
+// Issue the cursor's gather into the next buffer of the ring and advance it (past tiles whose
+// rows are not this warp's).  Each lane copies its token's 128 bytes with eight 16-byte
+// asynchronous copies; the buffer's mbarrier completes once all 32 lanes' copies have landed.
+template <int KIND>
+__device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, int q, int lane,
+                                              GCursor& c, InRing& gr) {
+  constexpr int NG = Cfg<KIND>::NGATH;
+  const int b = gr.issued % NG;
+  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
+  const int r = c.src[c.j];
+  if (r >= 0) {
+    const __nv_bfloat16* g = P.gsrc + (size_t)r * P.gd + c.n0 + c.ch * 64;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) cp_async16(buf + 16 * u, g + 8 * u);
+  }
+  cp_async_arrive_noinc(&gr.bars[b]);
+  ++gr.issued;
+  if (++c.j == P.gk + P.gS) {
+    c.j = 0;
+    if (++c.ch == c.nch) {
+      do {
+        c.t += S.n_pairs;
+        gcursor_load<KIND>(P, S, q, lane, c);
+      } while (c.t < S.n_tiles && c.nch == 0);
+    }
+  }
+}
+
 template <int KIND>
 __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, uint32_t tacc, int nk,
                                               int q, int sub, int lane,
                                               Ring<Cfg<KIND>::NSLOT>& ring,
-                                              InRing& inr, InRing& gr, int tcount, uint64_t* tfull,
+                                              InRing& inr, InRing& gr, GCursor& gc, const Sched& S,
+                                              int tcount, uint64_t* tfull,
                                               uint32_t parity, volatile int* abort_flag) {
   constexpr int SPLIT = Cfg<KIND>::SPLIT;
   const uint32_t tl = tacc + ((uint32_t)(q * 32) << 16);
@@ -590,48 +659,35 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   }
   if constexpr (KIND == UNDISPATCH) {
     // dx = dl Wg (the accumulator) + the token's kept routed rows of dXd (choices 0..k-1) + its
-    // shared experts' rows, summed in that fixed order.  Each lane gathers its token's 128 bytes
-    // (one 64-column chunk of one source row) with eight 16-byte asynchronous copies into the
-    // warp's gather buffers, up to NGATH buffers ahead, and the buffer's mbarrier completes when
-    // all 32 lanes' copies have landed; the first ones are issued before the wait for the
-    // accumulator, so the gathers overlap the MMAs.
+    // shared experts' rows, summed in that fixed order.  The rows arrive through the warp's
+    // gather stream (gcursor_issue), which runs up to NGATH buffers ahead of this consumer, across
+    // tile boundaries, so the next tile's gathers are in flight while this one finishes.
     constexpr int NG = Cfg<KIND>::NGATH;
     const int nsrc = P.gk + P.gS;
-    const int tok = row0 + lane;
-    const bool live_row = t.live && tok < P.T;
-    int src[16];   // gathered row of each source, -1 when there is none (dropped, or past T)
+    GCursor cc;   // this tile, as the consumer sees it
+    cc.t = 0;
+    {
+      cc.row0 = row0;
+      cc.n0 = t.n * BN;
+      cc.nch = 0;
+      if (t.live)
+        for (int ch = 0; ch < BN / 64 && cc.n0 + ch * 64 < P.N; ++ch) ++cc.nch;
+      const int tok = row0 + lane;
+      const bool live_row = t.live && tok < P.T;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      int r = -1;
-      if (j < nsrc && live_row)
-        r = (j < P.gk) ? P.gslot[(size_t)tok * P.gk + j] : (int)((j - P.gk) * P.T_pad + tok);
-      src[j] = r;
-    }
-    int nch = 0;
-    if (t.live)
-      for (int ch = 0; ch < BN / 64 && t.n * BN + ch * 64 < P.N; ++ch) ++nch;
-    const int total = nch * nsrc;
-    auto g_issue = [&](int i) {   // the i-th gather of this tile: chunk i / nsrc, source i % nsrc
-      const int ch = i / nsrc, j = i - ch * nsrc;
-      const int b = gr.issued % NG;
-      uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
-      const int r = src[j];
-      if (r >= 0) {
-        const __nv_bfloat16* g = P.gsrc + (size_t)r * P.gd + t.n * BN + ch * 64;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cp_async16(buf + 16 * c, g + 8 * c);
+      for (int j = 0; j < 16; ++j) {
+        int r = -1;
+        if (j < nsrc && live_row)
+          r = (j < P.gk) ? P.gslot[(size_t)tok * P.gk + j] : (int)((j - P.gk) * P.T_pad + tok);
+        cc.src[j] = r;
       }
-      cp_async_arrive_noinc(&gr.bars[b]);   // every lane arrives once its own copies have landed
-      ++gr.issued;
-    };
-    int next = 0;
-    for (; next < total && next < NG; ++next) g_issue(next);
+    }
     if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
 #pragma unroll 1
-    for (int ch = 0; ch < nch; ++ch) {
-      const int n = t.n * BN + ch * 64;
+    for (int ch = 0; ch < cc.nch; ++ch) {
+      const int n = cc.n0 + ch * 64;
       tmem_ld64(tl + ch * 64, a);
 #pragma unroll 1
       for (int j = 0; j < nsrc; ++j) {
@@ -640,7 +696,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
                        P.timeout_ns))
           return false;   // still counted as in flight: the exit path waits for it
         ++gr.consumed;
-        if (src[j] >= 0) {
+        if (cc.src[j] >= 0) {
           const uint8_t* row = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
@@ -651,7 +707,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
           }
         }
         __syncwarp();   // every lane has read this buffer before it is refilled
-        if (next < total) g_issue(next++);
+        if (gc.t < S.n_tiles) gcursor_issue<KIND>(P, S, q, lane, gc, gr);
       }
       uint8_t* slot = ring_take(ring, lane);
       slot_put_bf16(slot, lane, a);
@@ -934,11 +990,24 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
                                        mapa_shared(smem_u32(&tempty[1]), 0)};
     int acc = 0, tcount = 0;
     uint32_t acc_phase = 0;
+    const Sched sched{tile_start, n_groups, n_tiles, n_pairs, rank};
+    GCursor gc;   // UNDISPATCH: the warp's gather stream, started NGATH buffers ahead
+    gc.t = n_tiles;
+    if constexpr (KIND == UNDISPATCH) {
+      gc.t = pair;
+      gcursor_load<KIND>(P, sched, quarter, lane, gc);
+      while (gc.t < n_tiles && gc.nch == 0) {
+        gc.t += n_pairs;
+        gcursor_load<KIND>(P, sched, quarter, lane, gc);
+      }
+      for (int i = 0; i < NG && gc.t < n_tiles; ++i) gcursor_issue<KIND>(P, sched, quarter, lane, gc, gr);
+    }
     for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs, ++tcount) {
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, sub, lane,
-                               ring, inr, gr, tcount, &tfull[acc], acc_phase, abort_flag))
+                               ring, inr, gr, gc, sched, tcount, &tfull[acc], acc_phase,
+                               abort_flag))
         break;
       tc_fence_before();
       __syncwarp();

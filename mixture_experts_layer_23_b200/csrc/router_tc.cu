@@ -30,7 +30,7 @@ constexpr int MAX_RSTAGES = 16;
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
 constexpr int SPLIT_MAX_EPAD = 64;            // split-K clusters reduce rows of at most 64 logits
 #ifndef MOE_ROUTER_MAX_SPLIT
-#define MOE_ROUTER_MAX_SPLIT 8                  // largest cluster a tile's contraction is split over
+#define MOE_ROUTER_MAX_SPLIT 1                  // largest cluster a tile's contraction is split over
 #endif
 
 // Shared memory per CTA: a whole-d CTA keeps up to ~200 KB of loads in flight; the CTAs of a
