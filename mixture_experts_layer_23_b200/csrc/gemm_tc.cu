@@ -57,7 +57,10 @@ constexpr uint32_t B_BYTES = BNH * BK * 2;          // 16 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES; // per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
-constexpr int TILE_GROUP_M = 16;  // m tiles per band of the tile order (see decode)
+#ifndef MOE_TILE_GROUP_M
+#define MOE_TILE_GROUP_M 16
+#endif
+constexpr int TILE_GROUP_M = MOE_TILE_GROUP_M;  // m tiles per band of the tile order (see decode)
 // Epilogue staging: each epilogue warp owns a ring of Cfg::NSLOT 4 KB slots (32 rows x 128 B, laid out
 // in the 128-byte swizzle TMA expects); finished chunks leave through TMA tile stores.
 constexpr uint32_t SLOT_BYTES = 32 * 128;
