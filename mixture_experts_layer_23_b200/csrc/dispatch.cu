@@ -112,7 +112,6 @@ dispatch_scan_kernel(int32_t* __restrict__ blk /* in: block counts, out: exclusi
 // (16-byte vectors, read once, written to each kept slot); the last E + 1 CTAs zero the padding
 // rows and mark shared rows in row_token.
 constexpr int SC_TOK = 32;   // tokens per scatter CTA (four per warp)
-static_assert(SC_TOK % 16 == 0, "tokens go two at a time per warp");
 static_assert(DT % SC_TOK == 0, "a scatter CTA must not straddle two rank CTAs");
 
 template <typename T, bool CM>
@@ -173,14 +172,11 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
     }
     return;
   }
-  // this warp's tokens: warp, warp + 8, warp + 16, warp + 24 of the CTA's 32, two at a time so
-  // that 2 x 8 sixteen-byte loads per lane are in flight before the stores
-  int sl[SC_TOK / 8][8];
-#pragma unroll
-  for (int i = 0; i < SC_TOK / 8; ++i) {
-    const int t = blockIdx.x * SC_TOK + warp + 8 * i;
+  for (int tt = warp; tt < SC_TOK; tt += 8) {
+    const int t = blockIdx.x * SC_TOK + tt;
+    if (t >= T_) break;
     int my_slot = -1;
-    if (t < T_ && lane < k) {
+    if (lane < k) {
       const int e = topk_idx[(int64_t)t * k + lane];
       const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
       const int layer = CM ? lane : 0;
@@ -193,39 +189,16 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
       }
       slot[(int64_t)t * k + lane] = my_slot;
     }
+    int sl[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sl[i][j] = __shfl_sync(0xffffffffu, my_slot, j);
-  }
-  constexpr int U = 8;   // vectors per lane and token loaded before they are stored
+    for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    const T* src = x + (int64_t)t * d;
+#pragma unroll 8
+    for (int v = lane; v < nv; v += 32) {
+      const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
 #pragma unroll
-  for (int i = 0; i < SC_TOK / 8; i += 2) {
-    const int t0 = blockIdx.x * SC_TOK + warp + 8 * i, t1 = t0 + 8;
-    const bool ok0 = t0 < T_, ok1 = t1 < T_;
-    const T* src0 = x + (int64_t)t0 * d;
-    const T* src1 = x + (int64_t)t1 * d;
-    for (int v0 = lane; v0 < nv; v0 += 32 * U) {
-      Vec16<T> a[U], b[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v0 + 32 * u;
-        if (v < nv) {
-          if (ok0) a[u] = ld_vec_stream(src0 + (int64_t)v * VN);
-          if (ok1) b[u] = ld_vec_stream(src1 + (int64_t)v * VN);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int v = v0 + 32 * u;
-        if (v < nv) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (ok0 && j < k && sl[i][j] >= 0)
-              st_vec(Xd + (int64_t)sl[i][j] * d + (int64_t)v * VN, a[u]);
-            if (ok1 && j < k && sl[i + 1][j] >= 0)
-              st_vec(Xd + (int64_t)sl[i + 1][j] * d + (int64_t)v * VN, b[u]);
-          }
-        }
-      }
+      for (int j = 0; j < 8; ++j)
+        if (j < k && sl[j] >= 0) st_vec(Xd + (int64_t)sl[j] * d + (int64_t)v * VN, val);
     }
   }
 }
