@@ -28,13 +28,10 @@ namespace {
 
 constexpr int MAX_RSTAGES = 16;
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
-constexpr int SPLIT_MAX_EPAD = 64;            // split-K clusters reduce rows of at most 64 logits
-#ifndef MOE_ROUTER_MAX_SPLIT
-#define MOE_ROUTER_MAX_SPLIT 1                  // largest cluster a tile's contraction is split over
-#endif
+constexpr int STAGE_MAX_EPAD = 64;            // rows of at most 64 logits are staged in shared memory
 
-// Shared memory per CTA: a whole-d CTA keeps up to ~200 KB of loads in flight; the CTAs of a
-// split-K cluster stay within 112 KB so that two of them share an SM.
+// Shared memory per CTA: the router keeps up to ~200 KB of loads in flight; the router weight
+// gradient stays within 112 KB so that two of its CTAs share an SM.
 constexpr size_t RSMEM_WHOLE = 226 * 1024;
 constexpr size_t RSMEM_SPLIT = 112 * 1024;
 
@@ -50,39 +47,25 @@ struct alignas(64) RouterParams {
   int T, d, E, E_pad, k, gate_norm;
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages;
-  int n_ks;           // CTAs per cluster, each contracting d / n_ks of the 128-token tile
   int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
 };
 
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr));
-  return v;
-}
-__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
-  return v;
-}
 __device__ __forceinline__ void epi_bar() {   // the 128 epilogue threads (warps 2..5)
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-// One cluster of n_ks CTAs per 128-token tile; CTA r of the cluster contracts the k blocks
-// [r nk / n_ks, (r + 1) nk / n_ks).  With n_ks > 1 (at most 64 experts) every CTA parks its
-// partial logits in shared memory and the cluster's first CTA adds the others' partials to its
-// own in rank order (a fixed order: bit-reproducible) before the softmax and top-k.  Logits,
-// expert ids and gate weights are staged in shared memory and leave as contiguous rows.
+// One CTA per 128-token tile contracts the whole of d.  (Splitting the contraction over a cluster,
+// with the partial logits added over distributed shared memory, measured slower at every layer
+// size: 42 against 41 us at T = 16384, d = 4096, E = 8 with two CTAs per tile, and worse with more.)
+// Rows of at most 64 logits are staged in shared memory with the expert ids and gate weights, and
+// leave as contiguous rows.
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
   pdl_prologue();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const int RSTAGES = P.nstages;
-  const bool split = P.n_ks > 1;
-  const bool small = P.E_pad <= SPLIT_MAX_EPAD;   // rows staged in shared memory
+  const bool small = P.E_pad <= STAGE_MAX_EPAD;   // rows staged in shared memory
   // staging row stride (floats): a multiple of 4 (16-byte rows for vector access) and an odd
   // number of 16-byte units, so eight threads' 16-byte accesses to their rows hit distinct banks
   const int PS = P.E_pad + 4 + ((P.E_pad / 4 + 1) % 2 == 0 ? 4 : 0);
@@ -98,7 +81,6 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int crank = split ? (int)cluster_ctarank() : 0;
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int i = 0; i < RSTAGES; ++i) {
@@ -114,10 +96,8 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int m0 = (blockIdx.x / P.n_ks) * 128;
-  const int nk_all = P.d / 64;
-  const int kb0 = crank * nk_all / P.n_ks, kb1 = (crank + 1) * nk_all / P.n_ks;
-  const int nk = kb1 - kb0;
+  const int m0 = blockIdx.x * 128;
+  const int nk = P.d / 64;
   const unsigned long long budget = P.timeout_ns;
 
   uint32_t outstanding = 0, out_phase = 0;   // producer: stages loaded and not seen consumed
@@ -129,8 +109,8 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       outstanding &= ~(1u << stage);
       mbar_expect_tx(&full[stage], P.stage_bytes);
       uint8_t* sA = smem + stage * P.stage_bytes;
-      tma_load_2d(sA, &P.x_map, &full[stage], (kb0 + kb) * 64, m0);
-      tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], (kb0 + kb) * 64, 0);
+      tma_load_2d(sA, &P.x_map, &full[stage], kb * 64, m0);
+      tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], kb * 64, 0);
       outstanding |= 1u << stage;
       out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
@@ -168,7 +148,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   const int t = m0 + row;
   const bool epi = warp >= 2;
   bool have = false;                             // this warp holds its accumulator rows
-  float acc[SPLIT_MAX_EPAD];
+  float acc[STAGE_MAX_EPAD];
   if (epi) {
     // warp-uniform: the TMEM loads below need the whole warp
     have = __all_sync(0xffffffffu, wait_bounded(tfull, 0, abort_flag, budget));
@@ -178,7 +158,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     if (small) {
       const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll
-      for (int c = 0; c < SPLIT_MAX_EPAD / 16; ++c) {
+      for (int c = 0; c < STAGE_MAX_EPAD / 16; ++c) {
         if (c * 16 < P.E_pad) {
           float v[16];
           tmem_ld16(ta + (uint32_t)(c * 16), v);
@@ -186,55 +166,14 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
           for (int i = 0; i < 16; ++i) acc[c * 16 + i] = v[i];
         }
       }
-      if (split && crank != 0) {
-#pragma unroll
-        for (int e = 0; e < SPLIT_MAX_EPAD; e += 4)
-          if (e < P.E_pad)
-            *reinterpret_cast<float4*>(&part[row * PS + e]) =
-                make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
-      }
     }
   }
-  __syncwarp();
-  tc_fence_before();
-  if (split) cluster_sync();   // #1: every CTA's roles are done; partials and abort flags visible
-
-  if (epi && crank == 0) {
+  if (epi) {
     // a placeholder routing (experts 0..k-1, weight 0, logits 0) when any wait of the tile ran
     // out, so that the kernels after this one stay in bounds; the status word reports it
-    bool ok = have && !*abort_flag;
-    if (split)
-      for (int r = 1; r < P.n_ks; ++r)
-        ok = ok && ld_cluster_s32(mapa_shared(smem_u32((const void*)abort_flag), r)) == 0;
+    const bool ok = have && !*abort_flag;
     const bool live = t < P.T;
     if (small) {
-      if (ok && split) {
-        // add the other CTAs' partials in rank order, 16 logits at a time: all 16-byte DSMEM
-        // loads of a group are issued before the first add
-        const uint32_t my_row = smem_u32(&part[row * PS]);
-#pragma unroll 1
-        for (int e0 = 0; e0 < P.E_pad; e0 += 16) {
-          float4 q[7][4];
-#pragma unroll
-          for (int r = 1; r < 8; ++r)
-            if (r < P.n_ks) {
-              const uint32_t base = mapa_shared(my_row + 4u * e0, r);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) q[r - 1][u] = ld_cluster_v4(base + 16u * u);
-            }
-#pragma unroll
-          for (int r = 1; r < 8; ++r)
-            if (r < P.n_ks) {
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                acc[e0 + 4 * u] += q[r - 1][u].x;
-                acc[e0 + 4 * u + 1] += q[r - 1][u].y;
-                acc[e0 + 4 * u + 2] += q[r - 1][u].z;
-                acc[e0 + 4 * u + 3] += q[r - 1][u].w;
-              }
-            }
-        }
-      }
       TopK8 st;
       topk_init(st);
       for (int e = 0; e < P.E; ++e) {
@@ -263,7 +202,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
         P.topk_w[(size_t)m0 * P.k + i] = sw[(i / P.k) * 9 + i % P.k];
       }
     } else if (ok) {
-      // wide rows (more than 64 experts, never split): stream them out of TMEM 16 at a time
+      // wide rows (more than 64 experts): stream them out of TMEM 16 at a time
       TopK8 st;
       topk_init(st);
       float v[16];
@@ -291,7 +230,6 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     }
   }
   __syncwarp();
-  if (split) cluster_sync();   // #2: the first CTA has read the others' partials
   tc_fence_before();
   __syncthreads();             // every role has finished (the abort flag is final)
   if (*abort_flag && warp == 0 && lane == 0) {
@@ -479,22 +417,12 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   while ((int)cols < E_pad) cols <<= 1;
   P.tmem_cols = cols;
   P.stage_bytes = RA_BYTES + (uint32_t)E_pad * 128u;
-  // Split the contraction over a cluster when the token tiles alone leave the GPU short of CTAs:
-  // the smallest power-of-two split (at most 8) that brings the grid to two CTAs per SM, each
-  // keeping at least two k blocks.
   const int n_tiles = (D.T + 127) / 128;
-  const int nk = D.d / 64;
-  int n_ks = 1;
-  if (E_pad <= SPLIT_MAX_EPAD)
-    while (n_ks < MOE_ROUTER_MAX_SPLIT && n_tiles * n_ks < 2 * num_sms() && nk / (2 * n_ks) >= 2)
-      n_ks *= 2;
-  P.n_ks = n_ks;
-  const int nk_cta = (nk + n_ks - 1) / n_ks;
-  const size_t stage_rows = E_pad <= SPLIT_MAX_EPAD ? (size_t)128 * (E_pad + 8) * 4 : 0;
+  const int nk_cta = D.d / 64;
+  const size_t stage_rows = E_pad <= STAGE_MAX_EPAD ? (size_t)128 * (E_pad + 8) * 4 : 0;
   // alignment slack, staged rows, expert ids and weights, barriers (2 per stage + 2), TMEM slot
   const size_t fixed = 1024 + stage_rows + 2 * 128 * 9 * 4 + 2 * 8 + 16;
-  const size_t budget = n_ks > 1 ? RSMEM_SPLIT : RSMEM_WHOLE;
-  const size_t fit = (budget - fixed) / (P.stage_bytes + 2 * 8);
+  const size_t fit = (RSMEM_WHOLE - fixed) / (P.stage_bytes + 2 * 8);
   P.nstages = (int)std::max<size_t>(
       1, std::min<size_t>(std::min<size_t>(MAX_RSTAGES, fit), (size_t)nk_cta));
   const size_t smem = fixed + (size_t)P.nstages * (P.stage_bytes + 2 * 8);
@@ -505,7 +433,7 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
       return MOE_ERR_CUDA;
     smem_set = (int)smem;
   }
-  return launch_k(router_tc_kernel, n_tiles * n_ks, 192, smem, st, n_ks, P);
+  return launch_k(router_tc_kernel, n_tiles, 192, smem, st, 1, P);
 }
 
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
