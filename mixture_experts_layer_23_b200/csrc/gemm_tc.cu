@@ -68,10 +68,15 @@ constexpr size_t MISC_BYTES = 1536;   // barriers, TMEM slot, abort flag, tile p
 
 enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4, UNDISPATCH = 5 };
 
-// UNDISPATCH epilogue gathers: per epilogue warp, buffers of 32 rows x 64 bf16 columns, one
-// 128-byte bulk copy per row, rows 144 bytes apart (16-byte reads of a row by 8 lanes at a time hit
-// 8 distinct bank groups).
-constexpr uint32_t GROW = 144;
+// UNDISPATCH epilogue gathers: per epilogue warp, buffers of 32 rows x 64 bf16 columns.  With
+// MOE_UNDISPATCH_GATHER4 the rows arrive by TMA gathers of four rows each into the 128-byte swizzled
+// layout (rows 128 bytes apart); otherwise each lane copies its row with 16-byte asynchronous
+// copies, rows 144 bytes apart (16-byte reads of a row by 8 lanes at a time hit 8 distinct bank
+// groups).
+#ifndef MOE_UNDISPATCH_GATHER4
+#define MOE_UNDISPATCH_GATHER4 0
+#endif
+constexpr uint32_t GROW = MOE_UNDISPATCH_GATHER4 ? 128 : 144;
 constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 
 // Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
@@ -141,6 +146,7 @@ struct alignas(64) Params {
   void* out;              // the output's base and row stride (elements), for direct stores
   long long out_ld;
   // UNDISPATCH: the rows its epilogue gathers and adds
+  CUtensorMap gmap;            // dXd [rows, gd], box {64, 1}: four-row TMA gathers
   const __nv_bfloat16* gsrc;   // dXd [rows, gd]
   const int32_t* gslot;        // slot [T, gk]: routed row of each assignment, -1 if dropped
   int gk, gS, gd;              // routed choices, shared experts (rows s * T_pad + t), row length
@@ -537,14 +543,31 @@ __device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, i
                                               GCursor& c, InRing& gr) {
   constexpr int NG = Cfg<KIND>::NGATH;
   const int b = gr.issued % NG;
-  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
   const int r = c.src[c.j];
+#if MOE_UNDISPATCH_GATHER4
+  // lane i < 8 gathers the rows of lanes 4i..4i+3 (a lane without a source reads row 0, which the
+  // consumer then skips); lane 0 arms the buffer's barrier for all 32 rows
+  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES;
+  const int rr = r >= 0 ? r : 0;
+  const int src_lane = (lane & 7) * 4;
+  const int r0 = __shfl_sync(0xffffffffu, rr, src_lane), r1 = __shfl_sync(0xffffffffu, rr, src_lane + 1);
+  const int r2 = __shfl_sync(0xffffffffu, rr, src_lane + 2), r3 = __shfl_sync(0xffffffffu, rr, src_lane + 3);
+  __syncwarp();   // every lane has read this buffer's previous contents
+  if (lane == 0) {
+    fence_async_smem();
+    mbar_expect_tx(&gr.bars[b], GATHER_BUF_BYTES);
+  }
+  __syncwarp();
+  if (lane < 8) tma_gather4(buf + lane * 4 * GROW, &P.gmap, &gr.bars[b], c.n0 + c.ch * 64, r0, r1, r2, r3);
+#else
+  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
   if (r >= 0) {
     const __nv_bfloat16* g = P.gsrc + (size_t)r * P.gd + c.n0 + c.ch * 64;
 #pragma unroll
     for (int u = 0; u < 8; ++u) cp_async16(buf + 16 * u, g + 8 * u);
   }
   cp_async_arrive_noinc(&gr.bars[b]);
+#endif
   ++gr.issued;
   if (++c.j == P.gk + P.gS) {
     c.j = 0;
@@ -705,7 +728,9 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             float v[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c * 16), v);
+            // 16-byte unit c of the row (swizzled by the row index for TMA gathers)
+            const int cu = MOE_UNDISPATCH_GATHER4 ? (c ^ (lane & 7)) : c;
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(row + cu * 16), v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[8 * c + i] += v[i];
           }
@@ -887,7 +912,8 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     }
     mbar_init(drain, 1);
     for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
-    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 32);   // one per lane
+    // gather buffers: one arrival per lane (asynchronous copies) or one armed arrival (TMA gathers)
+    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], MOE_UNDISPATCH_GATHER4 ? 1 : 32);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -1251,6 +1277,11 @@ moe_status launch_undispatch_tc(const Dims& D, const __nv_bfloat16* dl16, const 
   P.N = D.d;
   P.K = (int)round_up(D.E, BK);
   P.gsrc = (const __nv_bfloat16*)dXd;
+  {
+    const uint64_t dims[2] = {(uint64_t)D.d, (uint64_t)D.R};
+    const uint32_t box[2] = {64, 1};
+    if (!make_map(&P.gmap, dXd, 2, dims, box)) return MOE_ERR_CUDA;
+  }
   P.gslot = slot;
   P.gk = D.k;
   P.gS = D.S;
