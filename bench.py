@@ -6,7 +6,9 @@
 One step = moe_layer_fwd + moe_layer_bwd over one batch of the workload (default: the largest
 layer, the Mixtral-style dropless top-2 layer, T=16384, d=4096, E=8, SwiGLU F=14336, softmax over
 the two chosen logits, bf16), inputs resident in HBM.  K steps are timed with CUDA events on the launching stream, one pair per step,
-with a 256 MiB write between steps to flush L2 (outside the timed pairs); the run is bracketed by
+with an L2 flush between steps (outside the timed pairs: a 256 MiB write, then a 256 MiB read of a
+second buffer, which evicts the written lines so that their write-back to HBM is not charged to
+the first kernel of the next step); the run is bracketed by
 a barrier and a device synchronise, and the max over ranks is taken.  value = tokens processed
 by all ranks / that time.  Several GPUs run independent replicas (the layer has no exchange step
 on one device), so scaling is weak.
@@ -38,6 +40,20 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s fwd+bwd on 1 B200; % bf16 TC peak (GEMM), % HBM BW (rest)"
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Between timed steps: write FLUSH_BYTES (twice the 126 MB L2), then read as many bytes of a
+    second buffer, so that L2 ends up holding clean lines of neither the step's inputs nor its
+    outputs (a write alone leaves L2 full of dirty lines, written back during the next step)."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        torch.amax(self.r)
 GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2"}
 
 
@@ -154,7 +170,8 @@ def workload_config(shape, world: int) -> dict:
             "capacity_factor": shape.capacity_factor, "bias": shape.bias,
             "aux_loss_coef": shape.aux_loss_coef,
             "drop_order": "choice-major" if shape.choice_major else "token",
-            "l2": "GPU arm: 256 MiB write between timed steps, outside the timed events",
+            "l2": "GPU arm: 256 MiB write + 256 MiB read of another buffer between timed "
+                  "steps, outside the timed events",
             "parallelism": f"replicas x{world}"}
 
 
@@ -374,7 +391,7 @@ def run_ours(args):
     x = to_device(inp["x"], shape, dev)
     dy = None if shape.fwd_only else to_device(inp["dy"], shape, dev)
     layer = MoELayer(shape, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -390,7 +407,7 @@ def run_ours(args):
 
     for _ in range(args.warmup):
         step()
-        flush.zero_()
+        flush()
     torch.cuda.synchronize(dev)
     st = layer.status()
     if st != moe.MOE_OK:
@@ -413,7 +430,7 @@ def run_ours(args):
         step()
         pe[i].record(stream)
         moe.set_profile_events(None, None)
-        flush.zero_()
+        flush()
     torch.cuda.synchronize(dev)
     phased_ms = sum(s.elapsed_time(e) for s, e in zip(ps, pe)) / K
     phase_ms = {}
@@ -437,7 +454,7 @@ def run_ours(args):
         starts[i].record(stream)
         step()
         ends[i].record(stream)
-        flush.zero_()
+        flush()
     launches = moe.kernel_launches() - n0
     torch.cuda.synchronize(dev)
     timed_wall_s = time.perf_counter() - t_wall
@@ -468,7 +485,7 @@ def run_ours(args):
             moe.set_profile_events(None, top_events(i))
         step()
         moe.set_profile_events(None, None)
-        flush.zero_()
+        flush()
     torch.cuda.synchronize(dev)
     top_clk = top_clocks.stop()
     barrier()
@@ -541,7 +558,7 @@ def run_ours(args):
     else:
         for _ in range(args.warmup):
             sg.replay()
-            flush.zero_()
+            flush()
         gs, ge = [mk() for _ in range(K)], [mk() for _ in range(K)]
         barrier()
         torch.cuda.synchronize(dev)
@@ -549,7 +566,7 @@ def run_ours(args):
             gs[i].record(stream)
             sg.replay()
             ge[i].record(stream)
-            flush.zero_()
+            flush()
         torch.cuda.synchronize(dev)
         barrier()
         g_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(gs, ge)))
@@ -635,7 +652,7 @@ def run_ours(args):
         else:
             for _ in range(args.warmup):
                 fused_step()
-                flush.zero_()
+                flush()
             fs, fe = [mk() for _ in range(K)], [mk() for _ in range(K)]
             barrier()
             torch.cuda.synchronize(dev)
@@ -643,7 +660,7 @@ def run_ours(args):
                 fs[i].record(stream)
                 fused_step()
                 fe[i].record(stream)
-                flush.zero_()
+                flush()
             torch.cuda.synchronize(dev)
             barrier()
             f_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(fs, fe)))
@@ -724,11 +741,11 @@ def run_ep(args):
              torch.empty(El, d, F, device=dev))
     r = EPRank(shape, rank, world, device=dev, chunks=args.ep_chunks)
     ex = DistExchange()
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
         step(r, ex, x, W["Wg"], bias, W1l, W3l, W2l, dy, grads)
-        flush.zero_()
+        flush()
     torch.cuda.synchronize(dev)
     K = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
@@ -739,7 +756,7 @@ def run_ep(args):
         starts[i].record(stream)
         step(r, ex, x, W["Wg"], bias, W1l, W3l, W2l, dy, grads)
         ends[i].record(stream)
-        flush.zero_()
+        flush()
     torch.cuda.synchronize(dev)
     dist.barrier()
     total_ms = reduce_max(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, dev)

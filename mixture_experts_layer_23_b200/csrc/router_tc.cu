@@ -6,7 +6,7 @@
 // x once from HBM: with E = 64 its 2*T*d*E FLOPs are more than the CUDA cores deliver in that
 // time, so the contraction runs on the tensor cores and everything after it stays on chip.
 //
-// One CTA per 128 tokens (192 threads): warp 0 streams x tiles [128 x 64] and the whole gate
+// One CTA per tile of at most 128 tokens (192 threads): warp 0 streams x tiles [rows x 64] and the whole gate
 // matrix slice [E_pad x 64] (E rounded up to 16, zero rows from TMA's out-of-bounds fill) through
 // a ring of up to 16 stages (as many as shared memory holds: with d <= 1024 and few experts the
 // whole token tile is in flight at once, since a CTA has only one tile to load); one lane of warp 1 issues tcgen05.mma (M = 128, N = E_pad) into a TMEM
@@ -36,7 +36,7 @@ constexpr size_t RSMEM_WHOLE = 226 * 1024;
 constexpr size_t RSMEM_SPLIT = 112 * 1024;
 
 struct alignas(64) RouterParams {
-  CUtensorMap x_map;  // x [T, d], box {64, 128}
+  CUtensorMap x_map;  // x [T, d], box {64, rows}
   CUtensorMap w_map;  // Wg [E, d], box {64, E_pad}
   const float* bias;
   float* logits;
@@ -45,6 +45,7 @@ struct alignas(64) RouterParams {
   uint32_t* status;   // may be null (no status word to report a timeout into)
   unsigned long long timeout_ns;
   int T, d, E, E_pad, k, gate_norm;
+  int rows;           // tokens per CTA (<= 128): the tiles are balanced over the SMs
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages;
   int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
@@ -54,9 +55,12 @@ __device__ __forceinline__ void epi_bar() {   // the 128 epilogue threads (warps
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
-// One CTA per 128-token tile contracts the whole of d.  (Splitting the contraction over a cluster,
-// with the partial logits added over distributed shared memory, measured slower at every layer
-// size: 42 against 41 us at T = 16384, d = 4096, E = 8 with two CTAs per tile, and worse with more.)
+// One CTA per token tile contracts the whole of d.  A tile holds `rows` <= 128 tokens, chosen on
+// the host so that the tiles come out close to a whole number of waves over the SMs (T = 16384:
+// 147 tiles of 112 tokens instead of 128 tiles of 128, which left 20 SMs idle); the MMA still
+// runs M = 128, and the accumulator lanes past `rows` (zero rows of A) are never read.
+// (Splitting the contraction over a cluster, with the partial logits added over distributed
+// shared memory, measured slower at every layer size and was dropped.)
 // Rows of at most 64 logits are staged in shared memory with the expert ids and gate weights, and
 // leave as contiguous rows.
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
@@ -92,11 +96,22 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(tmem_slot, P.tmem_cols);
+  if (P.rows < 128) {
+    // A rows [rows, 128) of every stage are never loaded: zero them once, so the MMA reads zeros
+    // there (their accumulator lanes are not read either)
+    const int tail = (128 - P.rows) * 128 / 16;   // 16-byte units per stage
+    for (int i = threadIdx.x; i < RSTAGES * tail; i += blockDim.x) {
+      const int s = i / tail, u = i - s * tail;
+      *reinterpret_cast<uint4*>(smem + s * P.stage_bytes + P.rows * 128 + u * 16) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();   // the generic-proxy zeros before the tensor core's async-proxy reads
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int m0 = blockIdx.x * 128;
+  const int m0 = blockIdx.x * P.rows;
   const int nk = P.d / 64;
   const unsigned long long budget = P.timeout_ns;
 
@@ -107,7 +122,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     for (int kb = 0; kb < nk; ++kb) {
       if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) break;
       outstanding &= ~(1u << stage);
-      mbar_expect_tx(&full[stage], P.stage_bytes);
+      mbar_expect_tx(&full[stage], (uint32_t)(P.rows + P.E_pad) * 128u);
       uint8_t* sA = smem + stage * P.stage_bytes;
       tma_load_2d(sA, &P.x_map, &full[stage], kb * 64, m0);
       tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], kb * 64, 0);
@@ -147,6 +162,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   const int row = quarter * 32 + lane;          // token row inside the tile
   const int t = m0 + row;
   const bool epi = warp >= 2;
+  const int nrow = min(P.rows, P.T - m0);       // the tile's tokens
   bool have = false;                             // this warp holds its accumulator rows
   float acc[STAGE_MAX_EPAD];
   if (epi) {
@@ -172,14 +188,24 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     // a placeholder routing (experts 0..k-1, weight 0, logits 0) when any wait of the tile ran
     // out, so that the kernels after this one stay in bounds; the status word reports it
     const bool ok = have && !*abort_flag;
-    const bool live = t < P.T;
+    const bool live = row < nrow;
     if (small) {
       TopK8 st;
       topk_init(st);
-      for (int e = 0; e < P.E; ++e) {
-        const float l = ok ? acc[e] + (P.bias ? P.bias[e] : 0.f) : 0.f;
-        part[row * PS + e] = l;
-        topk_push(st, l, e);
+      // compile-time indices keep acc in registers (a runtime index would put it in local memory)
+#pragma unroll
+      for (int c = 0; c < STAGE_MAX_EPAD / 16; ++c) {
+        if (c * 16 < P.E) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c * 16 + i;
+            if (e < P.E) {
+              const float l = ok ? acc[e] + (P.bias ? P.bias[e] : 0.f) : 0.f;
+              part[row * PS + e] = l;
+              topk_push(st, l, e);
+            }
+          }
+        }
       }
       int32_t* oi = sidx + row * 9;
       float* ow = sw + row * 9;
@@ -193,7 +219,6 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       }
       epi_bar();
       // the tile's rows are contiguous in logits, topk_idx and topk_w: coalesced stores
-      const int nrow = min(128, P.T - m0);
       const int tid = threadIdx.x - 64;
       for (int i = tid; i < nrow * P.E; i += 128)
         P.logits[(size_t)m0 * P.E + i] = part[(i / P.E) * PS + i % P.E];
@@ -397,8 +422,16 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   RouterParams P;
   memset(&P, 0, sizeof(P));
   const int E_pad = (int)round_up(D.E, 16);
-  if (!map2(&P.x_map, x, D.d, D.T, 64, 128) || !map2(&P.w_map, Wg, D.d, D.E, 64, E_pad))
+  // tokens per CTA: the fewest waves of 128-token tiles over the SMs, then tiles just large
+  // enough to cover T in that many waves (at least 16 tokens, so the per-CTA setup and the gate
+  // matrix reads stay small next to the token rows)
+  const int n_sm = num_sms();
+  const int waves = (D.T + 128 * n_sm - 1) / (128 * n_sm);
+  const int rows = (int)round_up(
+      std::max(std::min(16, D.T), std::min(128, (D.T + waves * n_sm - 1) / (waves * n_sm))), 8);
+  if (!map2(&P.x_map, x, D.d, D.T, 64, (uint32_t)rows) || !map2(&P.w_map, Wg, D.d, D.E, 64, E_pad))
     return MOE_ERR_CUDA;
+  P.rows = rows;
   P.bias = D.has_bias ? bias : nullptr;
   P.logits = logits;
   P.topk_idx = topk_idx;
@@ -417,7 +450,7 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   while ((int)cols < E_pad) cols <<= 1;
   P.tmem_cols = cols;
   P.stage_bytes = RA_BYTES + (uint32_t)E_pad * 128u;
-  const int n_tiles = (D.T + 127) / 128;
+  const int n_tiles = (D.T + rows - 1) / rows;
   const int nk_cta = D.d / 64;
   const size_t stage_rows = E_pad <= STAGE_MAX_EPAD ? (size_t)128 * (E_pad + 8) * 4 : 0;
   // alignment slack, staged rows, expert ids and weights, barriers (2 per stage + 2), TMEM slot

@@ -15,8 +15,9 @@ the device:
 steps.  The routing comes from moe_route on the workload's seeded inputs; the expert rows fed to
 the combine and the output gradients fed to the backward are random (their values do not change
 the cost).  Each timed launch is
-bracketed by CUDA events on the launching stream, with a 256 MiB write between launches to flush
-L2.  Prints one JSON line per step: average microseconds per launch, the step's algorithmic bytes
+bracketed by CUDA events on the launching stream, with an L2 flush between launches (a 256 MiB
+write, then a 256 MiB read of a second buffer, so that L2 holds no dirty lines whose write-back
+the next launch would pay for).  Prints one JSON line per step: average microseconds per launch, the step's algorithmic bytes
 and the resulting GB/s.
 """
 from __future__ import annotations
@@ -30,6 +31,18 @@ from . import moe
 from .configs import BY_NAME
 from .layer import act_dtype, to_device
 from .synth import make_inputs
+
+
+class L2Flush:
+    """256 MiB write, then 256 MiB read of another buffer: L2 ends up holding clean lines only."""
+
+    def __init__(self):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(64 << 20, dtype=torch.int32, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        torch.amax(self.r)
 
 
 def main(argv=None):
@@ -68,7 +81,7 @@ def main(argv=None):
     counts, kept = torch.empty(E, **i32), torch.empty(E, **i32)
     offsets, slot = torch.empty(E + 1, **i32), torch.empty(T, k, **i32)
     row_token = torch.empty(R, **i32)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     stream = torch.cuda.current_stream()
 
     def route():
@@ -136,7 +149,7 @@ def main(argv=None):
             continue
         for _ in range(a.warmup):
             fn()
-            flush.zero_()
+            flush()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(a.iters)]
         torch.cuda.synchronize()
@@ -144,7 +157,7 @@ def main(argv=None):
             s.record(stream)
             fn()
             e.record(stream)
-            flush.zero_()
+            flush()
         torch.cuda.synchronize()
         us = 1e3 * sum(s.elapsed_time(e) for s, e in ev) / a.iters
         line = {"workload": shape.name, "step": name, "us_per_launch": us,
@@ -166,7 +179,7 @@ def run_layer(shape, a):
     dev = {k: to_device(v, shape) for k, v in inp.items() if k != "bias"}
     bias = None if inp["bias"] is None else torch.from_numpy(inp["bias"]).cuda()
     layer = MoELayer(shape)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
 
     def step():
         layer.forward(dev["x"], dev["Wg"], bias, dev["W1"], dev["W3"], dev["W2"])
@@ -174,7 +187,7 @@ def run_layer(shape, a):
 
     for _ in range(a.warmup):
         step()
-        flush.zero_()
+        flush()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(a.iters)]
     torch.cuda.synchronize()
@@ -182,7 +195,7 @@ def run_layer(shape, a):
         s_.record()
         step()
         e_.record()
-        flush.zero_()
+        flush()
     torch.cuda.synchronize()
     us = 1e3 * sum(s_.elapsed_time(e_) for s_, e_ in ev) / a.iters
     print(json.dumps({"workload": shape.name, "step": "layer", "us_per_step": us,

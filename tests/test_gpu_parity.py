@@ -101,16 +101,19 @@ def test_edge_shapes(shape):
     _parity().full_compare(shape, seed=3)
 
 
-EDGE_SPLIT = [
-    # the router's contraction split over a cluster of 8 CTAs (two k blocks each), ragged last tile
-    LayerShape("router_split8_ragged", T=700, d=1024, E=8, k=2, d_ff=64, capacity_factor=1.0,
+EDGE_ROUTER = [
+    # router token tiles of 16 rows (44 CTAs), ragged last tile
+    LayerShape("router_ragged_tiles", T=700, d=1024, E=8, k=2, d_ff=64, capacity_factor=1.0,
                dtype=BF16, bias="normal"),
-    # one token tile split 8 ways; fewer tokens than a tile
-    LayerShape("router_split8_one_tile", T=100, d=2048, E=16, k=2, d_ff=64, capacity_factor=2.0,
-               dtype=BF16),
-    # 64 experts (split router at its widest row), 6 routed + 2 shared rows gathered per token by
-    # the un-dispatch epilogue, router weight gradient with N = 64
-    LayerShape("router_split_e64_shared", T=1111, d=512, E=64, k=6, d_ff=64, n_shared=2,
+    # fewer tokens than a 128-row tile: 16-row router tiles, the last one ragged
+    LayerShape("router_fewer_tokens_than_a_tile", T=100, d=2048, E=16, k=2, d_ff=64,
+               capacity_factor=2.0, dtype=BF16),
+    # two waves of router tiles (72 rows each, 264 CTAs), ragged last tile
+    LayerShape("router_two_waves", T=18945, d=64, E=8, k=2, d_ff=32, capacity_factor=1.25,
+               dtype=BF16, bias="normal"),
+    # 64 experts (the widest row staged in shared memory), 6 routed + 2 shared rows gathered per
+    # token by the un-dispatch epilogue, router weight gradient with N = 64
+    LayerShape("router_e64_shared_gathers", T=1111, d=512, E=64, k=6, d_ff=64, n_shared=2,
                act=SWIGLU, capacity_factor=1.25, dtype=BF16, bias="normal"),
     # 200 experts (whole-d router), k = 8 with 8 shared experts: 16 gathered rows per token;
     # router weight gradient with N = 256 and d = 192 (its second 128-column tile half outside d)
@@ -119,8 +122,8 @@ EDGE_SPLIT = [
 ]
 
 
-@pytest.mark.parametrize("shape", EDGE_SPLIT, ids=lambda s: s.name)
-def test_split_router_and_fused_backward_shapes(shape):
+@pytest.mark.parametrize("shape", EDGE_ROUTER, ids=lambda s: s.name)
+def test_router_tiles_and_fused_backward_shapes(shape):
     _parity().full_compare(shape, seed=4)
 
 
