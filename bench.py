@@ -48,12 +48,14 @@ class L2Flush:
     outputs (a write alone leaves L2 full of dirty lines, written back during the next step)."""
 
     def __init__(self, dev):
+        import torch
+        self._amax = torch.amax
         self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
         self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
     def __call__(self):
         self.w.zero_()
-        torch.amax(self.r)
+        self._amax(self.r)
 GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2"}
 
 

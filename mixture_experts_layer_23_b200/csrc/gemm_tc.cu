@@ -501,6 +501,15 @@ struct Sched {
   int n_groups, n_tiles, n_pairs, rank;
 };
 
+// a[j] for a runtime j < 16, through selects: indexing the array with j itself would move it from
+// registers to local memory, which a CTA with ~210 KB of shared memory reaches only through L2
+__device__ __forceinline__ int pick16(const int (&a)[16], int j) {
+  int r = a[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) r = (j == i) ? a[i] : r;
+  return r;
+}
+
 // UNDISPATCH: one epilogue warp's stream of gathers, (tile, chunk, source) in the order its
 // epilogue consumes them, so that they can be issued ahead across tile boundaries.
 struct GCursor {
@@ -536,14 +545,15 @@ __device__ __forceinline__ void gcursor_load(const Params& P, const Sched& S, in
 }
 
 // Issue the cursor's gather into the next buffer of the ring and advance it (past tiles whose
-// rows are not this warp's).  Each lane copies its token's 128 bytes with eight 16-byte
-// asynchronous copies; the buffer's mbarrier completes once all 32 lanes' copies have landed.
+// rows are not this warp's).  The warp copies the 32 rows' 128-byte pieces with eight 16-byte
+// asynchronous copies per lane, eight lanes to a row (each copy instruction moves four whole
+// 128-byte lines); the buffer's mbarrier completes once all 32 lanes' copies have landed.
 template <int KIND>
 __device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, int q, int lane,
                                               GCursor& c, InRing& gr) {
   constexpr int NG = Cfg<KIND>::NGATH;
   const int b = gr.issued % NG;
-  const int r = c.src[c.j];
+  const int r = pick16(c.src, c.j);
 #if MOE_UNDISPATCH_GATHER4
   // lane i < 8 gathers the rows of lanes 4i..4i+3 (a lane without a source reads row 0, which the
   // consumer then skips); lane 0 arms the buffer's barrier for all 32 rows
@@ -560,11 +570,13 @@ __device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, i
   __syncwarp();
   if (lane < 8) tma_gather4(buf + lane * 4 * GROW, &P.gmap, &gr.bars[b], c.n0 + c.ch * 64, r0, r1, r2, r3);
 #else
-  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
-  if (r >= 0) {
-    const __nv_bfloat16* g = P.gsrc + (size_t)r * P.gd + c.n0 + c.ch * 64;
+  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + (lane & 7) * 16;
+  const int col = c.n0 + c.ch * 64 + (lane & 7) * 8;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) cp_async16(buf + 16 * u, g + 8 * u);
+  for (int u = 0; u < 8; ++u) {
+    const int row = 4 * u + (lane >> 3);                 // token row of the warp's 32
+    const int rr = __shfl_sync(0xffffffffu, r, row);     // its gathered row, -1 if none
+    if (rr >= 0) cp_async16(buf + row * GROW, P.gsrc + (size_t)rr * P.gd + col);
   }
   cp_async_arrive_noinc(&gr.bars[b]);
 #endif
@@ -691,30 +703,27 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     // tile boundaries, so the next tile's gathers are in flight while this one finishes.
     constexpr int NG = Cfg<KIND>::NGATH;
     const int nsrc = P.gk + P.gS;
-    GCursor cc;   // this tile, as the consumer sees it
-    cc.t = 0;
+    // this tile as the consumer sees it: its chunks, and which of this lane's sources exist
+    const int n0 = t.n * BN;
+    int nch = 0;
+    if (t.live)
+      for (int ch = 0; ch < BN / 64 && n0 + ch * 64 < P.N; ++ch) ++nch;
+    uint32_t have_src = 0;   // bit j: source j of this lane's token is a row
     {
-      cc.row0 = row0;
-      cc.n0 = t.n * BN;
-      cc.nch = 0;
-      if (t.live)
-        for (int ch = 0; ch < BN / 64 && cc.n0 + ch * 64 < P.N; ++ch) ++cc.nch;
       const int tok = row0 + lane;
       const bool live_row = t.live && tok < P.T;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        int r = -1;
-        if (j < nsrc && live_row)
-          r = (j < P.gk) ? P.gslot[(size_t)tok * P.gk + j] : (int)((j - P.gk) * P.T_pad + tok);
-        cc.src[j] = r;
-      }
+      for (int j = 0; j < 16; ++j)
+        if (j < nsrc && live_row &&
+            (j >= P.gk || P.gslot[(size_t)tok * P.gk + j] >= 0))
+          have_src |= 1u << j;
     }
     if (!warp_wait(tfull, parity, abort_flag, P.timeout_ns)) return false;
     __syncwarp();
     tc_fence_after();
 #pragma unroll 1
-    for (int ch = 0; ch < cc.nch; ++ch) {
-      const int n = cc.n0 + ch * 64;
+    for (int ch = 0; ch < nch; ++ch) {
+      const int n = n0 + ch * 64;
       tmem_ld64(tl + ch * 64, a);
 #pragma unroll 1
       for (int j = 0; j < nsrc; ++j) {
@@ -723,7 +732,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
                        P.timeout_ns))
           return false;   // still counted as in flight: the exit path waits for it
         ++gr.consumed;
-        if (cc.src[j] >= 0) {
+        if ((have_src >> j) & 1u) {
           const uint8_t* row = gr.base + b * GATHER_BUF_BYTES + lane * GROW;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {

@@ -70,9 +70,9 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
                                              ~(uintptr_t)1023);
   const int RSTAGES = P.nstages;
   const bool small = P.E_pad <= STAGE_MAX_EPAD;   // rows staged in shared memory
-  // staging row stride (floats): a multiple of 4 (16-byte rows for vector access) and an odd
-  // number of 16-byte units, so eight threads' 16-byte accesses to their rows hit distinct banks
-  const int PS = P.E_pad + 4 + ((P.E_pad / 4 + 1) % 2 == 0 ? 4 : 0);
+  // staging row stride (floats): odd, so the 32 lanes' scalar accesses to their own rows (column
+  // e of rows 32q..32q+31) hit 32 distinct banks
+  const int PS = P.E_pad + 1;
   float* part = reinterpret_cast<float*>(smem + RSTAGES * P.stage_bytes);   // [128][PS]
   int32_t* sidx = reinterpret_cast<int32_t*>(part + (small ? 128 * PS : 0));  // [128][9]
   float* sw = reinterpret_cast<float*>(sidx + 128 * 9);                     // [128][9]
@@ -164,49 +164,36 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   const bool epi = warp >= 2;
   const int nrow = min(P.rows, P.T - m0);       // the tile's tokens
   bool have = false;                             // this warp holds its accumulator rows
-  float acc[STAGE_MAX_EPAD];
   if (epi) {
     // warp-uniform: the TMEM loads below need the whole warp
     have = __all_sync(0xffffffffu, wait_bounded(tfull, 0, abort_flag, budget));
   }
-  if (have) {
-    tc_fence_after();
-    if (small) {
-      const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll
-      for (int c = 0; c < STAGE_MAX_EPAD / 16; ++c) {
-        if (c * 16 < P.E_pad) {
-          float v[16];
-          tmem_ld16(ta + (uint32_t)(c * 16), v);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[c * 16 + i] = v[i];
-        }
-      }
-    }
-  }
+  if (have) tc_fence_after();
   if (epi) {
     // a placeholder routing (experts 0..k-1, weight 0, logits 0) when any wait of the tile ran
     // out, so that the kernels after this one stay in bounds; the status word reports it
     const bool ok = have && !*abort_flag;
     const bool live = row < nrow;
     if (small) {
-      TopK8 st;
-      topk_init(st);
-      // compile-time indices keep acc in registers (a runtime index would put it in local memory)
+      // the row's logits (+ bias) go to its staging row 16 at a time, then the serial softmax +
+      // top-k reads them back from there: a short loop body instead of E unrolled steps, whose
+      // code outgrew the instruction cache at 64 experts
+      float* prow = part + row * PS;
+      const uint32_t ta = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < P.E_pad / 16; ++c) {
+        float v[16];
+        if (have) tmem_ld16(ta + (uint32_t)(c * 16), v);
 #pragma unroll
-      for (int c = 0; c < STAGE_MAX_EPAD / 16; ++c) {
-        if (c * 16 < P.E) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = c * 16 + i;
-            if (e < P.E) {
-              const float l = ok ? acc[e] + (P.bias ? P.bias[e] : 0.f) : 0.f;
-              part[row * PS + e] = l;
-              topk_push(st, l, e);
-            }
-          }
+        for (int i = 0; i < 16; ++i) {
+          const int e = c * 16 + i;
+          if (e < P.E) prow[e] = ok ? v[i] + (P.bias ? P.bias[e] : 0.f) : 0.f;
         }
       }
+      TopK8 st;
+      topk_init(st);
+#pragma unroll 4
+      for (int e = 0; e < P.E; ++e) topk_push(st, prow[e], e);
       int32_t* oi = sidx + row * 9;
       float* ow = sw + row * 9;
       if (ok) {
