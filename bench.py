@@ -368,6 +368,26 @@ def phase_work(shape, n_kept):
     }
 
 
+def gemm_min_bytes(shape, n_kept):
+    """HBM bytes each GEMM phase cannot do without: every operand read once and every output
+    written once (kept and shared rows only, no padding).  With the FLOPs of phase_work this gives
+    each GEMM's own roofline, max(FLOPs / tensor peak, bytes / HBM bandwidth): the small layers'
+    weight gradients, for one, are bound by writing their fp32 output."""
+    b = 2 if shape.dtype == 1 else 4
+    T, d, F, S, Et = shape.T, shape.d, shape.d_ff, shape.n_shared, shape.E_tot
+    rows = n_kept + S * T
+    g = 2 if shape.act == 1 else 1
+    Xr, Fr, W = rows * d * b, rows * F * b, Et * F * d * b
+    return {
+        "expert_up": Xr + g * W + (g + 1) * Fr,          # Xd, W1 (W3) -> Gu (Gv), H
+        "expert_down": Fr + W + Xr,                      # H, W2 -> O
+        "dgrad_h": Xr + W + 2 * g * Fr,                  # dO, W2, Gu (Gv) -> dU (dV)
+        "dgrad_x": g * Fr + g * W + Xr,                  # dU (dV), W1 (W3) -> dXd
+        "wgrad_w1": g * (Fr + Xr + Et * F * d * 4),      # dU (dV), Xd -> fp32 dW1 (dW3)
+        "wgrad_w2": Xr + Fr + Et * F * d * 4,            # dO, H -> fp32 dW2
+    }
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -505,6 +525,7 @@ def run_ours(args):
     mm_peak = bf16_sus if sustained else bf16_tf
     mm_peak_name = "sustained" if sustained else "burst"
     phases = {}
+    min_bytes = gemm_min_bytes(shape, n_kept)
     for name, ms in phase_ms.items():
         bound, amount = work[name]
         if bound in ("tensor", "alu"):
@@ -513,6 +534,13 @@ def run_ours(args):
             phases[name] = {"ms": ms, "bound": bound, "achieved_tflops": ach, "frac": ach / peak}
             if bound == "tensor":
                 phases[name]["frac_burst"] = ach / bf16_tf
+                # the GEMM's own roofline: the slower of its tensor time and its HBM time
+                mb = min_bytes[name]
+                t_roof = max(amount / (peak * 1e12), mb / (hbm_gbs * 1e9))
+                phases[name].update(min_hbm_bytes=mb, roofline_ms=t_roof * 1e3,
+                                    roofline_bound="tensor" if amount / (peak * 1e12) >=
+                                    mb / (hbm_gbs * 1e9) else "hbm",
+                                    frac_roofline=t_roof * 1e3 / ms)
         else:
             ach = amount / (ms * 1e-3) / 1e9
             phases[name] = {"ms": ms, "bound": bound, "achieved_gbs": ach, "frac": ach / hbm_gbs}

@@ -125,6 +125,15 @@ ScratchLayout scratch_layout(const Dims& D) {
   S.dl16 = 0;
   if (router_bwd_tc_supported(D)) S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
   S.aux_part = take((size_t)D.n_aux * D.E * 4);
+  S.Xdt = S.dOt = S.xt = S.dyt = 0;
+  if (tc_supported(D)) {
+    S.Xdt = take(R * D.d * 2);
+    S.dOt = take(R * D.d * 2);
+    if (D.S > 0) {
+      S.xt = take((size_t)D.T_pad * D.d * 2);
+      S.dyt = take((size_t)D.T_pad * D.d * 2);
+    }
+  }
   S.total = off;
   return S;
 }
@@ -193,20 +202,37 @@ static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const
 
 // Expert FFN backward: dgrad through W2 and the activation, dgrad through W1 (and W3), then the
 // weight gradients; with phase_marks, the profiling events of backward phases 3..5 between them.
+// The expert GEMMs' backward.  s / S: the scratch area, for the tensor-core path's transposed
+// copies of Xd and dO (and of x and dy for shared experts), which its weight gradients read K-major.
 static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, const void* Xd,
                              const void* x, const int32_t* offsets, const void* W1,
                              const void* W3, const void* W2, const void* Gu, const void* Gv,
                              const void* H, void* dU, void* dV, void* dXd, float* dW1, float* dW3,
-                             float* dW2, uint32_t* status, cudaStream_t st,
+                             float* dW2, char* s, const ScratchLayout& S, cudaStream_t st,
                              bool phase_marks = false) {
+  uint32_t* status = (uint32_t*)(s + S.status);
   if (tc_supported(D)) {
     MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(3, st));
     MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(4, st));
-    MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, status, st));
+    // Xd^T and dO^T over the routed rows (padding rows are zero in both), x^T and dy^T over T_pad
+    // columns with zeros past T
+    const long long r0 = D.routed_row0, nr = D.R - D.routed_row0;
+    TransposeSpec js[4] = {
+        {Xd, s + S.Xdt, D.d, D.R, r0, r0, nr, -1, D.d},
+        {dO, s + S.dOt, D.d, D.R, r0, r0, nr, -1, D.d}};
+    int nj = 2;
+    if (D.S > 0) {
+      js[nj++] = {x, s + S.xt, D.d, D.T_pad, 0, 0, D.T_pad, D.T, D.d};
+      js[nj++] = {dy, s + S.dyt, D.d, D.T_pad, 0, 0, D.T_pad, D.T, D.d};
+    }
+    MOE_TRY(launch_transpose_bf16(js, nj, st));
+    MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, s + S.Xdt, D.S > 0 ? s + S.xt : nullptr, offsets, dW1,
+                                dW3, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(5, st));
-    MOE_TRY(launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st));
+    MOE_TRY(launch_wgrad_w2_tc(D, H, s + S.dOt, D.S > 0 ? s + S.dyt : nullptr, offsets, dW2,
+                               status, st));
     return MOE_OK;
   }
   MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, st));
@@ -460,8 +486,8 @@ moe_status moe_layer_bwd(const moe_config_t* cfg, const void* ctx, const void* d
   MOE_TRY(mark_bwd(2, st));
   MOE_TRY(expert_bwd(D, dO, dy, c + L.ctx_Xd, x, (const int32_t*)(c + L.ctx_offsets), W1, W3, W2,
                      c + L.ctx_Gu, L.ctx_Gv ? c + L.ctx_Gv : nullptr, c + L.ctx_H, s + S.dU,
-                     S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, (uint32_t*)(s + S.status),
-                     st, /*phase_marks=*/true));
+                     S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, s, S, st,
+                     /*phase_marks=*/true));
   MOE_TRY(mark_bwd(6, st));
   MOE_TRY(bwd_router_dx(D, L, S, c, s, Wg, dXd, dx, st));
   MOE_TRY(mark_bwd(7, st));
@@ -525,8 +551,7 @@ moe_status moe_expert_ffn_bwd(const moe_config_t* cfg, const void* dO, const voi
   const void* dy_ = D.S > 0 ? dy : dO;
   const void* x_ = D.S > 0 ? x : Xd;
   return expert_bwd(D, dO, dy_, Xd, x_, offsets, W1, W3, W2, Gu, Gv, H, s + S.dU,
-                    S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, (uint32_t*)(s + S.status),
-                    (cudaStream_t)stream);
+                    S.dV ? s + S.dV : nullptr, dXd, dW1, dW3, dW2, s, S, (cudaStream_t)stream);
 }
 
 moe_status moe_router_bwd(const moe_config_t* cfg, const void* ctx, const void* x, const void* Wg,

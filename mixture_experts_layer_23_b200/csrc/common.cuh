@@ -29,6 +29,11 @@ struct ScratchLayout {
   size_t dWg_part;      // [n_tchunk, E, d] float
   size_t dl16;          // [T, E8] bf16 copy of dlogits (tensor-core router backward), or 0
   size_t aux_part;      // [n_aux, E] float partial probability sums of the load-balancing loss
+  // column-major copies read K-major by the tensor-core weight gradients (0 on the CUDA-core path)
+  size_t Xdt;           // [d, R] bf16: Xd^T (routed columns)
+  size_t dOt;           // [d, R] bf16: dO^T (routed columns)
+  size_t xt;            // [d, T_pad] bf16: x^T, zero past T (shared experts only, else 0)
+  size_t dyt;           // [d, T_pad] bf16: dy^T, zero past T (shared experts only, else 0)
   size_t total;
 };
 

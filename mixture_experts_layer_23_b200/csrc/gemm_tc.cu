@@ -278,24 +278,21 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 #pragma unroll
     for (int j = 0; j < BNH / 64; ++j)
       tma_load_3d_pair(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
-  } else {  // WGRAD: K runs over the group's rows; A and B are read MN-major
+  } else {
+    // WGRAD: K runs over the group's rows.  One operand is read through its column-major copy
+    // (K-major, one 128-row box), the other straight from the token-major rows (MN-major, two
+    // 64-column boxes): with both MN-major the MMAs ran about a third slower per clock.
     if (P.which == 0) {
-      // A = dU|dV rows of the group (row space), B = Xd rows (routed) or x (shared)
+      // A = dU|dV rows of the group (row space, MN-major); B = Xd^T (routed) or x^T (shared)
 #pragma unroll
       for (int j = 0; j < BM / 64; ++j)
         tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
-#pragma unroll
-      for (int j = 0; j < BNH / 64; ++j) {
-        if (t.shared) tma_load_2d_pair(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
-        else tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
-      }
+      if (t.shared) tma_load_2d_pair(sB, &P.b_alt, bar, k0, nb);
+      else tma_load_2d_pair(sB, &P.b_main, bar, t.a_row + k0, nb);
     } else {
-      // A = dO rows (routed) or dy (shared), B = H rows of the group
-#pragma unroll
-      for (int j = 0; j < BM / 64; ++j) {
-        if (t.shared) tma_load_2d_pair(sA + j * 8192, &P.a_alt, bar, t.mrow + 64 * j, k0);
-        else tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.a_row + k0);
-      }
+      // A = dO^T (routed) or dy^T (shared), K-major; B = H rows of the group (MN-major)
+      if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
+      else tma_load_2d_pair(sA, &P.a_main, bar, t.a_row + k0, t.mrow);
 #pragma unroll
       for (int j = 0; j < BNH / 64; ++j)
         tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
@@ -947,9 +944,12 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   const uint32_t tmem_base = *tmem_slot;
   const int n_tiles = tile_start[n_groups];
   const unsigned long long budget = P.timeout_ns;
-  constexpr bool A_MN = (KIND == WGRAD);
-  constexpr bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == WGRAD || KIND == UNDISPATCH);
-  constexpr uint32_t IDESC = make_idesc(A_MN, B_MN);
+  // operand layouts: MN-major for the weights in the dgrads and, in the weight gradients, for
+  // dU|dV (dW1, dW3: P.which 0) or H (dW2), whose partner is read K-major from its transposed copy
+  const bool A_MN = (KIND == WGRAD) && P.which == 0;
+  const bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == UNDISPATCH) ||
+                    ((KIND == WGRAD) && P.which != 0);
+  const uint32_t IDESC = make_idesc(A_MN, B_MN);
 
   // producer bookkeeping, read again after every role has finished (abort drain)
   uint32_t outstanding = 0;            // stages with a load issued and not yet seen consumed
@@ -1213,14 +1213,16 @@ moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, cons
   return launch<DGRAD_X>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
 }
 
-// dW1 (and dW3) = dU^T X  -- M = F, N = d, K = the group's rows.
-moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xd,
-                               const void* x, const int32_t* offsets, float* dW1, float* dW3,
+// dW1 (and dW3) = dU^T X  -- M = F, N = d, K = the group's rows.  B comes K-major from Xdt [d][R]
+// (routed groups) or xt [d][T_pad] (shared experts).
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xdt,
+                               const void* xt, const int32_t* offsets, float* dW1, float* dW3,
                                uint32_t* status, cudaStream_t st) {
   for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
-    if (!(map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64) && map2(&P.b_main, Xd, D.d, D.R, 64, 64) &&
-          map2(&P.b_alt, x, D.d, D.T, 64, 64)))
+    if (!(map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64) &&
+          map2(&P.b_main, Xdt, D.R, D.d, 64, BNH) &&
+          (D.S == 0 || map2(&P.b_alt, xt, D.T_pad, D.d, 64, BNH))))
       return MOE_ERR_CUDA;
     if (!map3_f32(&P.o0, pass ? dW3 : dW1, D.d, D.F, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
     P.out = pass ? dW3 : dW1;
@@ -1235,12 +1237,14 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
   return MOE_OK;
 }
 
-// dW2 = dO^T H  -- M = d, N = F.
-moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, const void* dy,
+// dW2 = dO^T H  -- M = d, N = F.  A comes K-major from dOt [d][R] (routed groups) or dyt [d][T_pad]
+// (shared experts).
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dOt, const void* dyt,
                               const int32_t* offsets, float* dW2, uint32_t* status,
                               cudaStream_t st) {
   Params P = base_params(D, offsets, status);
-  if (!(map2(&P.a_main, dO, D.d, D.R, 64, 64) && map2(&P.a_alt, dy, D.d, D.T, 64, 64) &&
+  if (!(map2(&P.a_main, dOt, D.R, D.d, 64, BM) &&
+        (D.S == 0 || map2(&P.a_alt, dyt, D.T_pad, D.d, 64, BM)) &&
         map2(&P.b_main, H, D.F, D.R, 64, 64)))
     return MOE_ERR_CUDA;
   if (!map3_f32(&P.o0, dW2, D.F, D.d, D.E_tot, 32, 32)) return MOE_ERR_CUDA;

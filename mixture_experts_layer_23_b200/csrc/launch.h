@@ -63,6 +63,17 @@ moe_status launch_wgrad_w13_simt(const Dims& D, const void* dU, const void* dV, 
 moe_status launch_wgrad_w2_simt(const Dims& D, const void* H, const void* dO, const void* dy,
                                 const int32_t* offsets, float* dW2, cudaStream_t st);
 
+// Column-major copies of bf16 activations for the weight gradients: dst[c][col0 + r] =
+// src[row0 + r][c] for r < nrows, c < cols, with source rows r >= nvalid read as zeros (nvalid < 0:
+// all nrows); cols a multiple of 64, rows and destinations 16-byte aligned, the destination holds
+// round_up(nrows, 8) columns from col0.  Up to 8 jobs per launch.
+struct TransposeSpec {
+  const void* src;
+  void* dst;
+  long long src_ld, dst_ld, row0, col0, nrows, nvalid, cols;
+};
+moe_status launch_transpose_bf16(const TransposeSpec* specs, int n, cudaStream_t st);
+
 // tcgen05 router (bf16, d a multiple of 64, E <= 256); status may be null
 bool router_tc_supported(const Dims& D);
 moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const float* bias,
@@ -82,10 +93,13 @@ moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, cons
 moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
                              const void* W1, const void* W3, void* dXd, uint32_t* status,
                              cudaStream_t st);
-moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xd,
-                               const void* x, const int32_t* offsets, float* dW1, float* dW3,
+// The weight gradients read one operand through a column-major copy (launch_transpose_bf16):
+// dW1, dW3 take Xdt [d][R] (routed columns) and xt [d][T_pad] (shared experts), dW2 takes dOt
+// [d][R] and dyt [d][T_pad]; xt and dyt may be null when the layer has no shared experts.
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xdt,
+                               const void* xt, const int32_t* offsets, float* dW1, float* dW3,
                                uint32_t* status, cudaStream_t st);
-moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dO, const void* dy,
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dOt, const void* dyt,
                               const int32_t* offsets, float* dW2, uint32_t* status,
                               cudaStream_t st);
 
