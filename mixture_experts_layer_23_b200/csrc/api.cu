@@ -126,7 +126,7 @@ ScratchLayout scratch_layout(const Dims& D) {
   if (router_bwd_tc_supported(D)) S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
   S.aux_part = take((size_t)D.n_aux * D.E * 4);
   S.Xdt = S.dOt = S.xt = S.dyt = 0;
-  if (tc_supported(D)) {
+  if (wgrad_kmajor(D)) {
     S.Xdt = take(R * D.d * 2);
     S.dOt = take(R * D.d * 2);
     if (D.S > 0) {
@@ -216,6 +216,11 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
     if (phase_marks) MOE_TRY(mark_bwd(3, st));
     MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(4, st));
+    if (!wgrad_kmajor(D)) {
+      MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, status, st));
+      if (phase_marks) MOE_TRY(mark_bwd(5, st));
+      return launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st);
+    }
     // Xd^T and dO^T over the routed rows (padding rows are zero in both), x^T and dy^T over T_pad
     // columns with zeros past T
     const long long r0 = D.routed_row0, nr = D.R - D.routed_row0;

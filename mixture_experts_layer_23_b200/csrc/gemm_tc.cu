@@ -139,6 +139,7 @@ struct alignas(64) Params {
   int K;                 // row GEMMs: inner dimension (d or F)
   int act;
   int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
+  int kmajor;            // WGRAD: B (which 0) or A (which 2) read K-major from its transposed copy
   int chunk;             // > 0: the groups are fixed chunks of this many token rows (router
                          // backward) instead of the experts' row ranges
   int stall;             // failure-path test: the MMA issuer first waits on a barrier that
@@ -278,10 +279,10 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 #pragma unroll
     for (int j = 0; j < BNH / 64; ++j)
       tma_load_3d_pair(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
-  } else {
-    // WGRAD: K runs over the group's rows.  One operand is read through its column-major copy
-    // (K-major, one 128-row box), the other straight from the token-major rows (MN-major, two
-    // 64-column boxes): with both MN-major the MMAs ran about a third slower per clock.
+  } else if (P.kmajor) {
+    // WGRAD, K over the group's rows, one operand read through its column-major copy (K-major,
+    // one 128-row box), the other straight from the token-major rows (MN-major, two 64-column
+    // boxes): with both MN-major the MMAs ran about a third slower per clock
     if (P.which == 0) {
       // A = dU|dV rows of the group (row space, MN-major); B = Xd^T (routed) or x^T (shared)
 #pragma unroll
@@ -293,6 +294,28 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
       // A = dO^T (routed) or dy^T (shared), K-major; B = H rows of the group (MN-major)
       if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
       else tma_load_2d_pair(sA, &P.a_main, bar, t.a_row + k0, t.mrow);
+#pragma unroll
+      for (int j = 0; j < BNH / 64; ++j)
+        tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
+    }
+  } else {  // WGRAD, both operands straight from the token-major rows (MN-major)
+    if (P.which == 0) {
+      // A = dU|dV rows of the group (row space), B = Xd rows (routed) or x (shared)
+#pragma unroll
+      for (int j = 0; j < BM / 64; ++j)
+        tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
+#pragma unroll
+      for (int j = 0; j < BNH / 64; ++j) {
+        if (t.shared) tma_load_2d_pair(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
+        else tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
+      }
+    } else {
+      // A = dO rows (routed) or dy (shared), B = H rows of the group
+#pragma unroll
+      for (int j = 0; j < BM / 64; ++j) {
+        if (t.shared) tma_load_2d_pair(sA + j * 8192, &P.a_alt, bar, t.mrow + 64 * j, k0);
+        else tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.a_row + k0);
+      }
 #pragma unroll
       for (int j = 0; j < BNH / 64; ++j)
         tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
@@ -944,11 +967,12 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   const uint32_t tmem_base = *tmem_slot;
   const int n_tiles = tile_start[n_groups];
   const unsigned long long budget = P.timeout_ns;
-  // operand layouts: MN-major for the weights in the dgrads and, in the weight gradients, for
-  // dU|dV (dW1, dW3: P.which 0) or H (dW2), whose partner is read K-major from its transposed copy
-  const bool A_MN = (KIND == WGRAD) && P.which == 0;
+  // operand layouts: MN-major for the weights in the dgrads; in the weight gradients, both
+  // operands MN-major, or (P.kmajor) dU|dV (dW1, dW3: P.which 0) or H (dW2) MN-major and the
+  // partner read K-major from its transposed copy
+  const bool A_MN = (KIND == WGRAD) && (P.which == 0 || !P.kmajor);
   const bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == UNDISPATCH) ||
-                    ((KIND == WGRAD) && P.which != 0);
+                    ((KIND == WGRAD) && (P.which != 0 || !P.kmajor));
   const uint32_t IDESC = make_idesc(A_MN, B_MN);
 
   // producer bookkeeping, read again after every role has finished (abort drain)
@@ -1147,6 +1171,15 @@ bool tc_supported(const Dims& D) {
          tc::encoder() != nullptr;
 }
 
+// Weight gradients with one operand read K-major from a transposed copy: worth its copies (two
+// [rows, d] arrays read and written) only when the experts take long batches.  Measured: the
+// Mixtral-style layer (T k / E = 4096 rows per expert) gains 1.2 ms of its 30.6 ms step; the
+// DeepSeek-style (1536), BERT- and GPT-2-style (512) layers lost 0.1-0.25 ms, their weight
+// gradients being short or bound by writing their fp32 output.
+bool wgrad_kmajor(const Dims& D) {
+  return tc_supported(D) && (long long)D.T * D.k >= 2048LL * D.E;
+}
+
 
 using namespace tc;
 
@@ -1213,17 +1246,23 @@ moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, cons
   return launch<DGRAD_X>(P, row_tiles_bound(D, (D.d + BN - 1) / BN), st);
 }
 
-// dW1 (and dW3) = dU^T X  -- M = F, N = d, K = the group's rows.  B comes K-major from Xdt [d][R]
-// (routed groups) or xt [d][T_pad] (shared experts).
-moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xdt,
-                               const void* xt, const int32_t* offsets, float* dW1, float* dW3,
+// dW1 (and dW3) = dU^T X  -- M = F, N = d, K = the group's rows.  With wgrad_kmajor(D), B comes
+// K-major from Xdt [d][R] (routed groups) or xt [d][T_pad] (shared experts); otherwise Xd and x
+// are read MN-major as they are.
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* X,
+                               const void* xs, const int32_t* offsets, float* dW1, float* dW3,
                                uint32_t* status, cudaStream_t st) {
+  const bool km = wgrad_kmajor(D);
   for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
-    if (!(map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64) &&
-          map2(&P.b_main, Xdt, D.R, D.d, 64, BNH) &&
-          (D.S == 0 || map2(&P.b_alt, xt, D.T_pad, D.d, 64, BNH))))
-      return MOE_ERR_CUDA;
+    P.kmajor = km ? 1 : 0;
+    bool ok = map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64);
+    if (km)
+      ok = ok && map2(&P.b_main, X, D.R, D.d, 64, BNH) &&
+           (D.S == 0 || map2(&P.b_alt, xs, D.T_pad, D.d, 64, BNH));
+    else
+      ok = ok && map2(&P.b_main, X, D.d, D.R, 64, 64) && map2(&P.b_alt, xs, D.d, D.T, 64, 64);
+    if (!ok) return MOE_ERR_CUDA;
     if (!map3_f32(&P.o0, pass ? dW3 : dW1, D.d, D.F, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
     P.out = pass ? dW3 : dW1;
     P.out_ld = D.d;
@@ -1237,16 +1276,21 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
   return MOE_OK;
 }
 
-// dW2 = dO^T H  -- M = d, N = F.  A comes K-major from dOt [d][R] (routed groups) or dyt [d][T_pad]
-// (shared experts).
-moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dOt, const void* dyt,
+// dW2 = dO^T H  -- M = d, N = F.  With wgrad_kmajor(D), A comes K-major from dOt [d][R] (routed
+// groups) or dyt [d][T_pad] (shared experts); otherwise dO and dy are read MN-major as they are.
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* G, const void* gs,
                               const int32_t* offsets, float* dW2, uint32_t* status,
                               cudaStream_t st) {
+  const bool km = wgrad_kmajor(D);
   Params P = base_params(D, offsets, status);
-  if (!(map2(&P.a_main, dOt, D.R, D.d, 64, BM) &&
-        (D.S == 0 || map2(&P.a_alt, dyt, D.T_pad, D.d, 64, BM)) &&
-        map2(&P.b_main, H, D.F, D.R, 64, 64)))
-    return MOE_ERR_CUDA;
+  P.kmajor = km ? 1 : 0;
+  bool ok = map2(&P.b_main, H, D.F, D.R, 64, 64);
+  if (km)
+    ok = ok && map2(&P.a_main, G, D.R, D.d, 64, BM) &&
+         (D.S == 0 || map2(&P.a_alt, gs, D.T_pad, D.d, 64, BM));
+  else
+    ok = ok && map2(&P.a_main, G, D.d, D.R, 64, 64) && map2(&P.a_alt, gs, D.d, D.T, 64, 64);
+  if (!ok) return MOE_ERR_CUDA;
   if (!map3_f32(&P.o0, dW2, D.F, D.d, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
   P.out = dW2;
   P.out_ld = D.F;

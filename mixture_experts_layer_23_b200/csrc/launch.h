@@ -93,13 +93,15 @@ moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, cons
 moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
                              const void* W1, const void* W3, void* dXd, uint32_t* status,
                              cudaStream_t st);
-// The weight gradients read one operand through a column-major copy (launch_transpose_bf16):
-// dW1, dW3 take Xdt [d][R] (routed columns) and xt [d][T_pad] (shared experts), dW2 takes dOt
-// [d][R] and dyt [d][T_pad]; xt and dyt may be null when the layer has no shared experts.
-moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* Xdt,
-                               const void* xt, const int32_t* offsets, float* dW1, float* dW3,
+// The weight gradients.  With wgrad_kmajor(D) they read one operand through a column-major copy
+// (launch_transpose_bf16): X / xs are Xdt [d][R] (routed columns) / xt [d][T_pad] (shared experts)
+// and G / gs are dOt [d][R] / dyt [d][T_pad], xs and gs null without shared experts; otherwise X,
+// xs, G, gs are Xd, x, dO, dy themselves (all valid pointers).
+bool wgrad_kmajor(const Dims& D);
+moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* X,
+                               const void* xs, const int32_t* offsets, float* dW1, float* dW3,
                                uint32_t* status, cudaStream_t st);
-moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* dOt, const void* dyt,
+moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* G, const void* gs,
                               const int32_t* offsets, float* dW2, uint32_t* status,
                               cudaStream_t st);
 

@@ -122,6 +122,22 @@ EDGE_ROUTER = [
 ]
 
 
+# layers with at least 2048 routed rows per expert on average, whose weight gradients read Xd^T and
+# dO^T (and x^T, dy^T for shared experts) K-major from transposed copies: a shared expert with a
+# ragged token count (T_pad columns, zeros past T), and a GELU top-1 layer
+EDGE_WGRAD = [
+    LayerShape("kmajor_wgrad_shared_ragged", T=2500, d=128, E=2, k=2, d_ff=192, n_shared=1,
+               act=SWIGLU, capacity_factor=1.25, dtype=BF16, bias="normal"),
+    LayerShape("kmajor_wgrad_gelu_top1", T=4200, d=192, E=2, k=1, d_ff=128, act=GELU,
+               capacity_factor=None, dtype=BF16),
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_WGRAD, ids=lambda s: s.name)
+def test_kmajor_weight_gradient_shapes(shape):
+    _parity().full_compare(shape, seed=5)
+
+
 @pytest.mark.parametrize("shape", EDGE_ROUTER, ids=lambda s: s.name)
 def test_router_tiles_and_fused_backward_shapes(shape):
     _parity().full_compare(shape, seed=4)
