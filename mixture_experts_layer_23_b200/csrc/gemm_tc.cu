@@ -68,15 +68,16 @@ constexpr size_t MISC_BYTES = 1536;   // barriers, TMEM slot, abort flag, tile p
 
 enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4, UNDISPATCH = 5 };
 
-// UNDISPATCH epilogue gathers: per epilogue warp, buffers of 32 rows x 64 bf16 columns.  With
-// MOE_UNDISPATCH_GATHER4 the rows arrive by TMA gathers of four rows each into the 128-byte swizzled
-// layout (rows 128 bytes apart); otherwise each lane copies its row with 16-byte asynchronous
-// copies, rows 144 bytes apart (16-byte reads of a row by 8 lanes at a time hit 8 distinct bank
-// groups).
-#ifndef MOE_UNDISPATCH_GATHER4
-#define MOE_UNDISPATCH_GATHER4 0
+// UNDISPATCH epilogue gathers: per epilogue warp, buffers of 32 rows x 64 bf16 columns, rows 144
+// bytes apart (16-byte reads of a row by 8 lanes at a time hit 8 distinct bank groups), filled by
+// 16-byte asynchronous copies.  (TMA gathers of four rows each into the 128-byte swizzled layout
+// measured slower: 213 against 191 us on the Mixtral-style layer, 256 against 202 us on the
+// DeepSeek-style layer.)  MOE_UNDISPATCH_SPLIT = 2 gives the kind 8 epilogue warps, two per TMEM
+// lane quarter taking alternate 64-column chunks, with 3 gather buffers each and one load stage.
+#ifndef MOE_UNDISPATCH_SPLIT
+#define MOE_UNDISPATCH_SPLIT 1
 #endif
-constexpr uint32_t GROW = MOE_UNDISPATCH_GATHER4 ? 128 : 144;
+constexpr uint32_t GROW = 144;
 constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 
 // Per-kind balance of epilogue warps against pipeline stages (shared memory holds both).  The
@@ -101,7 +102,7 @@ constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 
 template <int KIND>
 struct Cfg {
-  static constexpr int EPI_WARPS = (KIND == UP) ? 8 : 4;
+  static constexpr int EPI_WARPS = (KIND == UP) ? 8 : (KIND == UNDISPATCH) ? 4 * MOE_UNDISPATCH_SPLIT : 4;
   static constexpr int SPLIT = EPI_WARPS / 4;   // epilogue warps per TMEM lane quarter
   // plain-output kinds may store straight from registers, which frees the staging ring for a
   // seventh stage of loads in flight
@@ -110,9 +111,9 @@ struct Cfg {
   // UNDISPATCH contracts K = E (at most 4 k blocks): two stages are plenty, and the room goes to
   // the gather buffers of its epilogue
   static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? 5 : (KIND == DGRAD_H) ? MOE_DGRAD_H_STAGES
-                                       : (KIND == UNDISPATCH) ? 2 : 6;
+                                       : (KIND == UNDISPATCH) ? (MOE_UNDISPATCH_SPLIT > 1 ? 1 : 2) : 6;
   static constexpr int NIN = (KIND == DGRAD_H) ? MOE_DGRAD_H_NIN : 0;   // epilogue input slots per warp
-  static constexpr int NGATH = (KIND == UNDISPATCH) ? 6 : 0;   // epilogue gather buffers per warp
+  static constexpr int NGATH = (KIND == UNDISPATCH) ? (MOE_UNDISPATCH_SPLIT > 1 ? 3 : 6) : 0;   // gather buffers per warp
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int NSLOT = 2;                          // output staging slots per warp
   static constexpr uint32_t RING_BYTES = DIRECT ? 0 : EPI_WARPS * NSLOT * SLOT_BYTES;
@@ -147,7 +148,6 @@ struct alignas(64) Params {
   void* out;              // the output's base and row stride (elements), for direct stores
   long long out_ld;
   // UNDISPATCH: the rows its epilogue gathers and adds
-  CUtensorMap gmap;            // dXd [rows, gd], box {64, 1}: four-row TMA gathers
   const __nv_bfloat16* gsrc;   // dXd [rows, gd]
   const int32_t* gslot;        // slot [T, gk]: routed row of each assignment, -1 if dropped
   int gk, gS, gd;              // routed choices, shared experts (rows s * T_pad + t), row length
@@ -535,6 +535,7 @@ __device__ __forceinline__ int pick16(const int (&a)[16], int j) {
 struct GCursor {
   int t;          // tile (>= n_tiles: the stream has ended)
   int ch, j;      // chunk and source inside the tile
+  int sub;        // the warp's chunks of a tile are sub, sub + SPLIT, ...
   int nch;        // 64-column chunks of the tile in this warp's rows (0: none)
   int n0, row0;   // first column and first row of the warp's slab
   int src[16];    // gathered row of each source for this lane's token, -1 when there is none
@@ -543,7 +544,7 @@ struct GCursor {
 template <int KIND>
 __device__ __forceinline__ void gcursor_load(const Params& P, const Sched& S, int q, int lane,
                                              GCursor& c) {
-  c.ch = 0;
+  c.ch = c.sub;
   c.j = 0;
   c.nch = 0;
   if (c.t >= S.n_tiles) return;
@@ -574,22 +575,6 @@ __device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, i
   constexpr int NG = Cfg<KIND>::NGATH;
   const int b = gr.issued % NG;
   const int r = pick16(c.src, c.j);
-#if MOE_UNDISPATCH_GATHER4
-  // lane i < 8 gathers the rows of lanes 4i..4i+3 (a lane without a source reads row 0, which the
-  // consumer then skips); lane 0 arms the buffer's barrier for all 32 rows
-  uint8_t* buf = gr.base + b * GATHER_BUF_BYTES;
-  const int rr = r >= 0 ? r : 0;
-  const int src_lane = (lane & 7) * 4;
-  const int r0 = __shfl_sync(0xffffffffu, rr, src_lane), r1 = __shfl_sync(0xffffffffu, rr, src_lane + 1);
-  const int r2 = __shfl_sync(0xffffffffu, rr, src_lane + 2), r3 = __shfl_sync(0xffffffffu, rr, src_lane + 3);
-  __syncwarp();   // every lane has read this buffer's previous contents
-  if (lane == 0) {
-    fence_async_smem();
-    mbar_expect_tx(&gr.bars[b], GATHER_BUF_BYTES);
-  }
-  __syncwarp();
-  if (lane < 8) tma_gather4(buf + lane * 4 * GROW, &P.gmap, &gr.bars[b], c.n0 + c.ch * 64, r0, r1, r2, r3);
-#else
   uint8_t* buf = gr.base + b * GATHER_BUF_BYTES + (lane & 7) * 16;
   const int col = c.n0 + c.ch * 64 + (lane & 7) * 8;
 #pragma unroll
@@ -599,15 +584,15 @@ __device__ __forceinline__ void gcursor_issue(const Params& P, const Sched& S, i
     if (rr >= 0) cp_async16(buf + row * GROW, P.gsrc + (size_t)rr * P.gd + col);
   }
   cp_async_arrive_noinc(&gr.bars[b]);
-#endif
   ++gr.issued;
   if (++c.j == P.gk + P.gS) {
     c.j = 0;
-    if (++c.ch == c.nch) {
+    c.ch += Cfg<KIND>::SPLIT;
+    if (c.ch >= c.nch) {
       do {
         c.t += S.n_pairs;
         gcursor_load<KIND>(P, S, q, lane, c);
-      } while (c.t < S.n_tiles && c.nch == 0);
+      } while (c.t < S.n_tiles && c.ch >= c.nch);
     }
   }
 }
@@ -742,7 +727,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
     __syncwarp();
     tc_fence_after();
 #pragma unroll 1
-    for (int ch = 0; ch < nch; ++ch) {
+    for (int ch = sub; ch < nch; ch += SPLIT) {
       const int n = n0 + ch * 64;
       tmem_ld64(tl + ch * 64, a);
 #pragma unroll 1
@@ -757,9 +742,7 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             float v[8];
-            // 16-byte unit c of the row (swizzled by the row index for TMA gathers)
-            const int cu = MOE_UNDISPATCH_GATHER4 ? (c ^ (lane & 7)) : c;
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(row + cu * 16), v);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(row + c * 16), v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) a[8 * c + i] += v[i];
           }
@@ -942,7 +925,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     mbar_init(drain, 1);
     for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
     // gather buffers: one arrival per lane (asynchronous copies) or one armed arrival (TMA gathers)
-    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], MOE_UNDISPATCH_GATHER4 ? 1 : 32);
+    for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 32);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -1056,10 +1039,11 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     const Sched sched{tile_start, n_groups, n_tiles, n_pairs, rank};
     GCursor gc;   // UNDISPATCH: the warp's gather stream, started NGATH buffers ahead
     gc.t = n_tiles;
+    gc.sub = sub;
     if constexpr (KIND == UNDISPATCH) {
       gc.t = pair;
       gcursor_load<KIND>(P, sched, quarter, lane, gc);
-      while (gc.t < n_tiles && gc.nch == 0) {
+      while (gc.t < n_tiles && gc.ch >= gc.nch) {
         gc.t += n_pairs;
         gcursor_load<KIND>(P, sched, quarter, lane, gc);
       }
@@ -1334,11 +1318,6 @@ moe_status launch_undispatch_tc(const Dims& D, const __nv_bfloat16* dl16, const 
   P.N = D.d;
   P.K = (int)round_up(D.E, BK);
   P.gsrc = (const __nv_bfloat16*)dXd;
-  {
-    const uint64_t dims[2] = {(uint64_t)D.d, (uint64_t)D.R};
-    const uint32_t box[2] = {64, 1};
-    if (!make_map(&P.gmap, dXd, 2, dims, box)) return MOE_ERR_CUDA;
-  }
   P.gslot = slot;
   P.gk = D.k;
   P.gS = D.S;

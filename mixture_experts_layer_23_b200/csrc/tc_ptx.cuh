@@ -85,17 +85,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// TMA gather of four rows (row indices r0..r3) of one box column range starting at column c0,
-// into 4 consecutive 128-byte rows of shared memory (the map's box is one row high).
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int c0,
-                                            int r0, int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // 16-byte asynchronous copy global -> shared through the load/store path (both addresses 16-byte
 // aligned), and the arrive-on of an mbarrier once all of this thread's earlier such copies have
 // completed (the arrival counts against the barrier's expected count).
