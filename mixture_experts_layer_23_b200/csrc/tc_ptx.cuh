@@ -85,6 +85,14 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Untiled bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this CTA's
+// shared memory to global memory, tracked by the thread's bulk groups (bulk_commit / bulk_wait*).
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared through the load/store path (both addresses 16-byte
 // aligned), and the arrive-on of an mbarrier once all of this thread's earlier such copies have
 // completed (the arrival counts against the barrier's expected count).
