@@ -352,7 +352,8 @@ moe_status moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* t
   MOE_TRY(check_ptrs({x, topk_idx, counts, kept, offsets, slot, row_token, Xd, scratch}));
   const ScratchLayout S = scratch_layout(D);
   return launch_dispatch(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
-                         (int32_t*)((char*)scratch + S.blk_counts), (cudaStream_t)stream);
+                         (int32_t*)((char*)scratch + S.blk_counts),
+                         (uint32_t*)((char*)scratch + S.status), (cudaStream_t)stream);
 }
 
 moe_status moe_expert_ffn(const moe_config_t* cfg, const void* Xd, const void* x,
@@ -408,7 +409,7 @@ moe_status moe_layer_fwd(const moe_config_t* cfg, const void* x, const void* Wg,
   MOE_TRY(launch_route(D, x, Wg, bias, logits, idx, w, (uint32_t*)(s + S.status), st));
   MOE_TRY(mark_fwd(1, st));
   MOE_TRY(launch_dispatch(D, x, idx, counts, kept, offsets, slot, row_token, Xd,
-                          (int32_t*)(s + S.blk_counts), st));
+                          (int32_t*)(s + S.blk_counts), (uint32_t*)(s + S.status), st));
   if (D.aux_coef > 0.f)
     MOE_TRY(launch_aux_loss(D, logits, counts, (float*)(s + S.aux_part), (float*)(c + L.ctx_aux_loss),
                             st));

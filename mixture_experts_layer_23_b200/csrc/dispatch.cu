@@ -24,6 +24,8 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tc_host.h"
+#include "tc_ptx.cuh"
 
 namespace moe {
 namespace {
@@ -114,14 +116,126 @@ dispatch_scan_kernel(int32_t* __restrict__ blk /* in: block counts, out: exclusi
 constexpr int SC_TOK = 32;   // tokens per scatter CTA (four per warp)
 static_assert(DT % SC_TOK == 0, "a scatter CTA must not straddle two rank CTAs");
 
+// BULK: rows move through shared memory by bulk copies (one warp lane issues them): each warp
+// keeps SC_NB row buffers, loading token i + SC_NB while token i's row is stored to its slots.
+#ifndef MOE_DISPATCH_BULK
+#define MOE_DISPATCH_BULK 0
+#endif
+constexpr int SC_NB = 2;
+
+// The slot of this lane's assignment (lanes < k) of token t: its rank CTA's base + its rank inside
+// that CTA, kept if below C; writes slot[] and row_token[].  Returns -1 for dropped assignments.
+template <bool CM>
+__device__ __forceinline__ int finalise_slot(const int32_t* __restrict__ topk_idx,
+                                             const int32_t* __restrict__ blk_base,
+                                             const int32_t* s_off, int t, int E, int k, int64_t C,
+                                             int my_blk, int32_t* __restrict__ slot,
+                                             int32_t* __restrict__ row_token, int lane) {
+  int my_slot = -1;
+  if (lane < k) {
+    const int L = CM ? k : 1;
+    const int e = topk_idx[(int64_t)t * k + lane];
+    const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
+    const int layer = CM ? lane : 0;
+    const int pos = valid ? blk_base[((int64_t)my_blk * L + layer) * E + e] +
+                                slot[(int64_t)t * k + lane]
+                          : 0;
+    if (valid && (int64_t)pos < C) {
+      my_slot = s_off[e] + pos;
+      row_token[my_slot] = t;
+    }
+    slot[(int64_t)t * k + lane] = my_slot;
+  }
+  return my_slot;
+}
+
+// Bulk-copy form of the row copies: warp w takes tokens w, w + 8, w + 16, w + 24 of the CTA.  Lane 0
+// loads each token's row into one of the warp's SC_NB shared-memory buffers (an mbarrier per
+// buffer), stores it to each kept slot, and reloads the buffer for the token SC_NB later once those
+// stores have read it.  Every wait is bounded: when one runs out the warp stops, lets its copies in
+// flight land, and the status word (if any) reports MOE_STATUS_TIMEOUT.
 template <typename T, bool CM>
+__device__ __forceinline__ void scatter_rows_bulk(
+    const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
+    const int32_t* __restrict__ blk_base, const int32_t* s_off, int T_, int d, int E, int k,
+    int64_t C, int my_blk, int32_t* __restrict__ slot, int32_t* __restrict__ row_token,
+    T* __restrict__ Xd, uint32_t* __restrict__ status, unsigned long long budget) {
+  extern __shared__ __align__(128) uint8_t sc_rows[];   // [8 warps][SC_NB][row bytes], barriers
+  __shared__ int sc_abort;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t rb = (uint32_t)d * (uint32_t)sizeof(T);
+  uint8_t* buf = sc_rows + (size_t)warp * SC_NB * rb;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sc_rows + (size_t)8 * SC_NB * rb) + warp * SC_NB;
+  if (threadIdx.x == 0) sc_abort = 0;
+  if (lane == 0) {
+    for (int b = 0; b < SC_NB; ++b) tc::mbar_init(&bars[b], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  volatile int* abort_flag = &sc_abort;
+  const int t0 = blockIdx.x * SC_TOK + warp;
+  int n = 0;   // this warp's tokens: t0 + 8 i, i < n
+  while (n < SC_TOK / 8 && t0 + 8 * n < T_) ++n;
+  int pend[SC_NB];   // token (index i) whose load into buffer b is in flight, -1 if none
+#pragma unroll
+  for (int b = 0; b < SC_NB; ++b) pend[b] = -1;
+  if (lane == 0)
+    for (int i = 0; i < n && i < SC_NB; ++i) {
+      tc::mbar_expect_tx(&bars[i], rb);
+      tc::bulk_g2s(buf + (size_t)i * rb, x + (int64_t)(t0 + 8 * i) * d, rb, &bars[i]);
+      pend[i] = i;
+    }
+  bool ok = true;
+  for (int i = 0; i < n; ++i) {
+    const int t = t0 + 8 * i;
+    const int my_slot = finalise_slot<CM>(topk_idx, blk_base, s_off, t, E, k, C, my_blk, slot,
+                                          row_token, lane);
+    int sl[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    if (lane == 0 && ok) {
+      const int b = i % SC_NB;
+      if (!tc::wait_bounded(&bars[b], (uint32_t)(i / SC_NB) & 1u, abort_flag, budget)) {
+        ok = false;
+      } else {
+        pend[b] = -1;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < k && sl[j] >= 0) tc::bulk_s2g(Xd + (int64_t)sl[j] * d, buf + (size_t)b * rb, rb);
+        tc::bulk_commit();
+        if (i + SC_NB < n) {
+          tc::bulk_wait_read<0>();   // this buffer's stores have read it
+          tc::mbar_expect_tx(&bars[b], rb);
+          tc::bulk_g2s(buf + (size_t)b * rb, x + (int64_t)(t + 8 * SC_NB) * d, rb, &bars[b]);
+          pend[b] = i + SC_NB;
+        }
+      }
+    }
+    __syncwarp();
+  }
+  if (lane == 0) {
+    // loads still in flight after an abort land before the CTA exits (bounded), then every store
+    // has completed
+#pragma unroll
+    for (int b = 0; b < SC_NB; ++b)
+      if (pend[b] >= 0) {
+        volatile int never = 0;
+        tc::wait_bounded(&bars[b], (uint32_t)(pend[b] / SC_NB) & 1u, &never, 20000000ull);
+      }
+    tc::bulk_wait<0>();
+    if (!ok && status) atomicOr(status, MOE_STATUS_TIMEOUT);
+  }
+}
+
+template <typename T, bool CM, bool BULK>
 __global__ void __launch_bounds__(256)
 dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
                         const int32_t* __restrict__ blk_base, const int32_t* __restrict__ kept,
                         int T_, int d, int E, int k, int64_t C, int routed_row0, int n_tok_blocks,
                         int shared_rows, int32_t* __restrict__ offsets_out,
                         int32_t* __restrict__ slot /* in: local rank, out: slot */,
-                        int32_t* __restrict__ row_token, T* __restrict__ Xd) {
+                        int32_t* __restrict__ row_token, T* __restrict__ Xd,
+                        uint32_t* __restrict__ status, unsigned long long budget) {
   pdl_prologue();
   __shared__ int32_t s_kept[256];
   __shared__ int32_t s_off[257];
@@ -130,7 +244,6 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool tok_cta = (int)blockIdx.x < n_tok_blocks;
   const int my_blk = tok_cta ? (int)(blockIdx.x * SC_TOK / DT) : 0;
-  const int L = CM ? k : 1;
   for (int e = threadIdx.x; e < E; e += 256) {
     const int kp = kept[e];
     s_kept[e] = kp;
@@ -172,33 +285,26 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
     }
     return;
   }
-  for (int tt = warp; tt < SC_TOK; tt += 8) {
-    const int t = blockIdx.x * SC_TOK + tt;
-    if (t >= T_) break;
-    int my_slot = -1;
-    if (lane < k) {
-      const int e = topk_idx[(int64_t)t * k + lane];
-      const bool valid = (unsigned)e < (unsigned)E;  // an out-of-range id is never kept
-      const int layer = CM ? lane : 0;
-      const int pos = valid ? blk_base[((int64_t)my_blk * L + layer) * E + e] +
-                                  slot[(int64_t)t * k + lane]
-                            : 0;
-      if (valid && (int64_t)pos < C) {
-        my_slot = s_off[e] + pos;
-        row_token[my_slot] = t;
-      }
-      slot[(int64_t)t * k + lane] = my_slot;
-    }
-    int sl[8];
+  if constexpr (BULK) {
+    scatter_rows_bulk<T, CM>(x, topk_idx, blk_base, s_off, T_, d, E, k, C, my_blk, slot,
+                             row_token, Xd, status, budget);
+  } else {
+    for (int tt = warp; tt < SC_TOK; tt += 8) {
+      const int t = blockIdx.x * SC_TOK + tt;
+      if (t >= T_) break;
+      const int my_slot = finalise_slot<CM>(topk_idx, blk_base, s_off, t, E, k, C, my_blk, slot,
+                                            row_token, lane);
+      int sl[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
-    const T* src = x + (int64_t)t * d;
+      for (int j = 0; j < 8; ++j) sl[j] = __shfl_sync(0xffffffffu, my_slot, j);
+      const T* src = x + (int64_t)t * d;
 #pragma unroll 8
-    for (int v = lane; v < nv; v += 32) {
-      const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
+      for (int v = lane; v < nv; v += 32) {
+        const Vec16<T> val = ld_vec_stream(src + (int64_t)v * VN);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < k && sl[j] >= 0) st_vec(Xd + (int64_t)sl[j] * d + (int64_t)v * VN, val);
+        for (int j = 0; j < 8; ++j)
+          if (j < k && sl[j] >= 0) st_vec(Xd + (int64_t)sl[j] * d + (int64_t)v * VN, val);
+      }
     }
   }
 }
@@ -208,34 +314,47 @@ dispatch_scatter_kernel(const T* __restrict__ x, const int32_t* __restrict__ top
 template <typename T, bool CM>
 static moe_status dispatch_t(const Dims& D, const void* x, const int32_t* topk_idx,
                              int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot,
-                             int32_t* row_token, void* Xd, int32_t* blk_counts, cudaStream_t st) {
+                             int32_t* row_token, void* Xd, int32_t* blk_counts, uint32_t* status,
+                             cudaStream_t st) {
   MOE_TRY_S(launch_k(dispatch_rank_kernel<CM>, D.n_blk, 256, 0, st, 1, topk_idx, D.T, D.E, D.k,
                      blk_counts, slot));
   MOE_TRY_S(launch_k(dispatch_scan_kernel, (D.E + 7) / 8, 256, 0, st, 1, blk_counts, D.n_blk, D.E,
                      D.n_layers, D.C, counts, kept));
   const int n_tok_blocks = (D.T + SC_TOK - 1) / SC_TOK;
   const int grid = n_tok_blocks + D.E + 1;
-  return launch_k(dispatch_scatter_kernel<T, CM>, grid, 256, 0, st, 1, (const T*)x, topk_idx,
-                  (const int32_t*)blk_counts, (const int32_t*)kept, D.T, D.d, D.E, D.k, D.C,
-                  (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, offsets, slot, row_token,
-                  (T*)Xd);
+  constexpr bool BULK = MOE_DISPATCH_BULK != 0;
+  size_t smem = 0;
+  if (BULK) {
+    smem = (size_t)8 * SC_NB * D.d * sizeof(T) + 8 * SC_NB * 8;
+    static size_t smem_set = 48 * 1024;
+    if (smem > smem_set) {
+      if (cudaFuncSetAttribute(dispatch_scatter_kernel<T, CM, BULK>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      smem_set = smem;
+    }
+  }
+  return launch_k(dispatch_scatter_kernel<T, CM, BULK>, grid, 256, smem, st, 1, (const T*)x,
+                  topk_idx, (const int32_t*)blk_counts, (const int32_t*)kept, D.T, D.d, D.E, D.k,
+                  D.C, (int)D.routed_row0, n_tok_blocks, (int)D.routed_row0, offsets, slot,
+                  row_token, (T*)Xd, status, tc::wait_budget_ns());
 }
 
 moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
                            int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
-                           void* Xd, int32_t* blk_counts, cudaStream_t st) {
+                           void* Xd, int32_t* blk_counts, uint32_t* status, cudaStream_t st) {
   if (D.dtype == MOE_DTYPE_BF16) {
     if (D.choice_major)
       return dispatch_t<__nv_bfloat16, true>(D, x, topk_idx, counts, kept, offsets, slot,
-                                             row_token, Xd, blk_counts, st);
+                                             row_token, Xd, blk_counts, status, st);
     return dispatch_t<__nv_bfloat16, false>(D, x, topk_idx, counts, kept, offsets, slot,
-                                            row_token, Xd, blk_counts, st);
+                                            row_token, Xd, blk_counts, status, st);
   }
   if (D.choice_major)
     return dispatch_t<float, true>(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
-                                   blk_counts, st);
+                                   blk_counts, status, st);
   return dispatch_t<float, false>(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd,
-                                  blk_counts, st);
+                                  blk_counts, status, st);
 }
 
 // ----------------------------------------------------------------------------- no-allocation form
@@ -313,5 +432,5 @@ extern "C" moe_status moe_dispatch_noalloc(const moe_config_t* cfg, const void* 
   const moe_status h = moe::noalloc_histogram(&hist);
   if (h != MOE_OK) return h;
   return moe::launch_dispatch(D, x, topk_idx, counts, kept, offsets, slot, row_token, Xd, hist,
-                              (cudaStream_t)stream);
+                              nullptr, (cudaStream_t)stream);
 }

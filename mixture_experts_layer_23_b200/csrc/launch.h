@@ -13,9 +13,10 @@ moe_status launch_router_warp(const Dims& D, const void* x, const void* Wg, cons
                               float* logits, int32_t* topk_idx, float* topk_w, cudaStream_t st);
 moe_status launch_topk_from_logits(const Dims& D, const float* logits, int32_t* topk_idx,
                                    float* topk_w, cudaStream_t st);
+// status: the scratch status word, or null (moe_dispatch_noalloc)
 moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx, int32_t* counts,
                            int32_t* kept, int32_t* offsets, int32_t* slot, int32_t* row_token,
-                           void* Xd, int32_t* blk_counts, cudaStream_t st);
+                           void* Xd, int32_t* blk_counts, uint32_t* status, cudaStream_t st);
 moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
                           void* y, cudaStream_t st);
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
