@@ -72,10 +72,13 @@ enum Kind { UP = 0, DOWN = 1, DGRAD_H = 2, DGRAD_X = 3, WGRAD = 4, UNDISPATCH = 
 // bytes apart (16-byte reads of a row by 8 lanes at a time hit 8 distinct bank groups), filled by
 // 16-byte asynchronous copies.  (TMA gathers of four rows each into the 128-byte swizzled layout
 // measured slower: 213 against 191 us on the Mixtral-style layer, 256 against 202 us on the
-// DeepSeek-style layer.)  MOE_UNDISPATCH_SPLIT = 2 gives the kind 8 epilogue warps, two per TMEM
-// lane quarter taking alternate 64-column chunks, with 3 gather buffers each and one load stage.
+// DeepSeek-style layer.)  The kind has 8 epilogue warps (MOE_UNDISPATCH_SPLIT = 2), two per TMEM
+// lane quarter taking alternate 64-column chunks, with 3 gather buffers each and one load stage:
+// 190 -> 155 us on the Mixtral-style layer and 205 -> 150 us on the DeepSeek-style layer against 4
+// warps with 6 buffers each (MOE_UNDISPATCH_SPLIT = 1), whose single warp per SM sub-partition
+// could not keep its gathers in flight.
 #ifndef MOE_UNDISPATCH_SPLIT
-#define MOE_UNDISPATCH_SPLIT 1
+#define MOE_UNDISPATCH_SPLIT 2
 #endif
 constexpr uint32_t GROW = 144;
 constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;

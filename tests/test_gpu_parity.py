@@ -122,6 +122,21 @@ EDGE_ROUTER = [
 ]
 
 
+# rows too long for the dispatch's shared-memory row buffers (8 warps x 2 rows of 13 KB), which
+# take the 16-byte register copies instead of bulk copies
+EDGE_LONG_ROWS = [
+    LayerShape("dispatch_long_rows_bf16", T=300, d=6656, E=4, k=2, d_ff=64, capacity_factor=1.25,
+               dtype=BF16, bias="normal"),
+    LayerShape("dispatch_long_rows_fp32", T=200, d=3328, E=4, k=2, d_ff=32, capacity_factor=1.0,
+               dtype=FP32),
+]
+
+
+@pytest.mark.parametrize("shape", EDGE_LONG_ROWS, ids=lambda s: s.name)
+def test_dispatch_long_rows(shape):
+    _parity().full_compare(shape, seed=6)
+
+
 # layers with at least 2048 routed rows per expert on average, whose weight gradients read Xd^T and
 # dO^T (and x^T, dy^T for shared experts) K-major from transposed copies: a shared expert with a
 # ragged token count (T_pad columns, zeros past T), and a GELU top-1 layer
