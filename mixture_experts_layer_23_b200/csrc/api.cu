@@ -129,6 +129,7 @@ ScratchLayout scratch_layout(const Dims& D) {
     S.rw_count = take((size_t)(D.d + 127) / 128 * 4);
   }
   S.aux_part = take((size_t)D.n_aux * D.E * 4);
+  S.wg_sched = take(16);
   S.Xdt = S.dOt = S.xt = S.dyt = 0;
   if (wgrad_kmajor(D)) {
     S.Xdt = take(R * D.d * 2);
@@ -218,12 +219,13 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
   if (tc_supported(D)) {
     MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(3, st));
-    MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, status, st));
+    int* wg_sched = (int*)(s + S.wg_sched);   // zeroed by the input-gradient launch
+    MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, wg_sched, 4, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(4, st));
     if (!wgrad_kmajor(D)) {
-      MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, status, st));
+      MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, Xd, x, offsets, dW1, dW3, wg_sched, status, st));
       if (phase_marks) MOE_TRY(mark_bwd(5, st));
-      return launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, status, st);
+      return launch_wgrad_w2_tc(D, H, dO, dy, offsets, dW2, wg_sched + 2, status, st);
     }
     // Xd^T and dO^T over the routed rows (padding rows are zero in both), x^T and dy^T over T_pad
     // columns with zeros past T
@@ -238,10 +240,10 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
     }
     MOE_TRY(launch_transpose_bf16(js, nj, st));
     MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, s + S.Xdt, D.S > 0 ? s + S.xt : nullptr, offsets, dW1,
-                                dW3, status, st));
+                                dW3, wg_sched, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(5, st));
     MOE_TRY(launch_wgrad_w2_tc(D, H, s + S.dOt, D.S > 0 ? s + S.dyt : nullptr, offsets, dW2,
-                               status, st));
+                               wg_sched + 2, status, st));
     return MOE_OK;
   }
   MOE_TRY(launch_dgrad_h_simt(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, st));

@@ -122,11 +122,14 @@ struct Cfg {
   static constexpr uint32_t RING_BYTES = DIRECT ? 0 : EPI_WARPS * NSLOT * SLOT_BYTES;
   static constexpr uint32_t IN_BYTES = EPI_WARPS * NIN * SLOT_BYTES;
   static constexpr uint32_t GATH_BYTES = EPI_WARPS * NGATH * GATHER_BUF_BYTES;
-  static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN + EPI_WARPS * NGATH;
+  // WGRAD takes its tiles from a queue (longest first, claimed by the pair that is free first): its
+  // tiles' K is the group's row count, which differs tenfold between shared and routed experts
+  static constexpr int QD = (KIND == WGRAD) ? 8 : 0;         // tile-queue slots
+  static constexpr int NBARS = 2 * STAGES + 5 + EPI_WARPS * NIN + EPI_WARPS * NGATH + 2 * QD;
   static constexpr size_t SMEM_BYTES =
       1024 + STAGES * STAGE_BYTES + RING_BYTES + IN_BYTES + GATH_BYTES + MISC_BYTES;
   static_assert(SMEM_BYTES <= 232448, "over the 227 KB per-CTA shared memory limit");
-  static_assert(8 * NBARS + 16 + 4 * (MAX_GROUPS + 1) <= MISC_BYTES, "misc too small");
+  static_assert(8 * NBARS + 16 + 4 * (MAX_GROUPS + 1) + 4 * QD <= MISC_BYTES, "misc too small");
 };
 
 struct alignas(64) Params {
@@ -148,6 +151,10 @@ struct alignas(64) Params {
                          // backward) instead of the experts' row ranges
   int stall;             // failure-path test: the MMA issuer first waits on a barrier that
                          // nothing arrives on, so the wait runs out and the CTA aborts
+  int dynamic;           // WGRAD: tiles from the queue, shared experts' groups first
+  int* sched;            // dynamic: the launch's tile counter (zero before the launch)
+  int* zero;             // set zero[0..zero_n) to 0 first (the next launches' tile counters)
+  int zero_n;
   void* out;              // the output's base and row stride (elements), for direct stores
   long long out_ld;
   // UNDISPATCH: the rows its epilogue gathers and adds
@@ -211,17 +218,25 @@ __device__ __forceinline__ void group_rows(const Params& P, int g, int& a_row, i
   }
 }
 
+// The group at position v of the tile order: groups in index order, or (dynamic) the shared
+// experts' groups first, whose K = T_pad is the longest, then the routed ones.
+__device__ __forceinline__ int group_at(const Params& P, int v) {
+  if (!P.dynamic || P.S == 0) return v;
+  return v < P.S ? P.E + v : v - P.S;
+}
+
 template <int KIND>
 __device__ __forceinline__ Tile decode(const Params& P, const int* tile_start, int n_groups, int t,
                                        int rank) {
-  int lo = 0, hi = n_groups - 1;  // last g with tile_start[g] <= t
+  int lo = 0, hi = n_groups - 1;  // last position v with tile_start[v] <= t
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if (tile_start[mid] <= t) lo = mid; else hi = mid - 1;
   }
   Tile T;
-  T.g = lo;
-  group_rows(P, lo, T.a_row, T.o_row, T.rows, T.shared);
+  const int g = group_at(P, lo);
+  T.g = g;
+  group_rows(P, g, T.a_row, T.o_row, T.rows, T.shared);
   // Tile order inside the group: bands of TILE_GROUP_M m tiles, each walked m-fastest across all
   // n tiles.  The CTA pairs run consecutive tile indices at the same time, so one wave of pairs
   // touches about TILE_GROUP_M A slices and (pairs / TILE_GROUP_M) B slices, which stay in L2;
@@ -872,6 +887,87 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
   return true;
 }
 
+// ----------------------------------------------------------------------------- tile queue
+
+// The static tile sequence of a pair: pair, pair + n_pairs, ... (-1 past the last tile).
+__device__ __forceinline__ int static_next(int it, int t, int pair, int n_pairs, int n_tiles) {
+  const int n = it == 0 ? pair : t + n_pairs;
+  return n < n_tiles ? n : -1;
+}
+//
+// With P.dynamic (WGRAD) the pair's tiles come from a queue instead of the static sequence pair,
+// pair + n_pairs, ...: the leader's producer takes tile `pair` first and then claims tiles from the
+// launch's counter (n_pairs + atomicAdd), and publishes each in slot pos % QD of both CTAs' queues;
+// the leader's MMA issuer and epilogue warps and the second CTA's producer and epilogue warps read
+// the slots in order and free them on the leader's q_empty.  -1 ends the sequence.  So the pair
+// that is free first takes the next tile, and the longest tiles (the shared experts' groups, first
+// in the tile order) are spread over the pairs before the short ones fill in.
+struct TileQueue {
+  int* tile;                 // this CTA's slots
+  uint64_t* full;            // this CTA's q_full
+  uint64_t* empty;           // this CTA's q_empty (the leader's are the ones used)
+  uint32_t own_tile, own_full, peer_tile, peer_full, leader_empty;   // shared::cluster addresses
+  int pos;                   // tiles taken so far
+};
+
+__device__ __forceinline__ TileQueue make_queue(int* tile, uint64_t* full, uint64_t* empty,
+                                                int rank) {
+  TileQueue q;
+  q.tile = tile;
+  q.full = full;
+  q.empty = empty;
+  q.own_tile = mapa_shared(smem_u32(tile), rank);
+  q.own_full = mapa_shared(smem_u32(full), rank);
+  q.peer_tile = mapa_shared(smem_u32(tile), rank ^ 1);
+  q.peer_full = mapa_shared(smem_u32(full), rank ^ 1);
+  q.leader_empty = mapa_shared(smem_u32(empty), 0);
+  q.pos = 0;
+  return q;
+}
+
+// the leader's producer: publish `t` in the next slot of both CTAs' queues
+template <int QD>
+__device__ __forceinline__ bool q_publish(TileQueue& q, int t, volatile int* abort_flag,
+                                          unsigned long long budget) {
+  const int s = q.pos % QD;
+  if (!wait_bounded_cluster(&q.empty[s], ((uint32_t)(q.pos / QD) & 1u) ^ 1u, abort_flag, budget))
+    return false;
+  st_cluster_u32(q.own_tile + 4 * s, t);
+  st_cluster_u32(q.peer_tile + 4 * s, t);
+  mbar_arrive_cluster(q.own_full + 8 * s);
+  mbar_arrive_cluster(q.peer_full + 8 * s);
+  ++q.pos;
+  return true;
+}
+
+// a single reading thread: the next tile (-1: none), or false if the wait ran out
+template <int QD>
+__device__ __forceinline__ bool q_take(TileQueue& q, int& t, volatile int* abort_flag,
+                                       unsigned long long budget) {
+  const int s = q.pos % QD;
+  if (!wait_bounded_cluster(&q.full[s], (uint32_t)(q.pos / QD) & 1u, abort_flag, budget))
+    return false;
+  t = *reinterpret_cast<volatile int*>(&q.tile[s]);
+  mbar_arrive_cluster(q.leader_empty + 8 * s);
+  ++q.pos;
+  return true;
+}
+
+// a reading warp (every lane gets the same answer; lane 0 frees the slot)
+template <int QD>
+__device__ __forceinline__ bool q_take_warp(TileQueue& q, int& t, int lane, volatile int* abort_flag,
+                                            unsigned long long budget) {
+  const int s = q.pos % QD;
+  if (!__all_sync(0xffffffffu, wait_bounded_cluster(&q.full[s], (uint32_t)(q.pos / QD) & 1u,
+                                                    abort_flag, budget)))
+    return false;
+  t = *reinterpret_cast<volatile int*>(&q.tile[s]);
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(q.leader_empty + 8 * s);
+  ++q.pos;
+  return true;
+}
+
 // ----------------------------------------------------------------------------- kernel
 
 template <int KIND>
@@ -898,21 +994,26 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   uint64_t* drain = tempty + 2;          // [1]
   uint64_t* in_bars = drain + 1;         // [EPI_WARPS * NIN]
   uint64_t* g_bars = in_bars + NUM_EPI_WARPS * NIN;   // [EPI_WARPS * NG]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(g_bars + NUM_EPI_WARPS * NG);
+  constexpr int QD = Cfg<KIND>::QD;
+  uint64_t* q_full = g_bars + NUM_EPI_WARPS * NG;      // [QD] tile-queue slot written
+  uint64_t* q_empty = q_full + QD;                     // [QD] slot read by all (the leader's used)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_empty + QD);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tile_start = reinterpret_cast<int*>(tmem_slot + 4);   // [MAX_GROUPS + 1]
+  int* q_tile = tile_start + MAX_GROUPS + 1;                 // [QD]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = (int)cluster_ctarank();   // 0 = leader of the pair
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int n_groups = P.E + P.S;
 
-  // per-group tile counts, then an exclusive prefix (warp 0)
-  for (int g = threadIdx.x; g < n_groups; g += NUM_THREADS) {
+  if (P.zero && blockIdx.x == 0 && (int)threadIdx.x < P.zero_n) P.zero[threadIdx.x] = 0;
+  // per-group tile counts in tile order, then an exclusive prefix (warp 0)
+  for (int v = threadIdx.x; v < n_groups; v += NUM_THREADS) {
     int a_row, o_row, rows;
     bool sh;
-    group_rows(P, g, a_row, o_row, rows, sh);
-    tile_start[g + 1] = group_tiles<KIND>(P, rows);
+    group_rows(P, group_at(P, v), a_row, o_row, rows, sh);
+    tile_start[v + 1] = group_tiles<KIND>(P, rows);
   }
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -929,6 +1030,12 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     for (int i = 0; i < NUM_EPI_WARPS * NIN; ++i) mbar_init(&in_bars[i], 1);
     // gather buffers: one arrival per lane (asynchronous copies) or one armed arrival (TMA gathers)
     for (int i = 0; i < NUM_EPI_WARPS * NG; ++i) mbar_init(&g_bars[i], 32);
+    // tile queue: written by the leader's producer (one arrival in each CTA), read by the leader's
+    // MMA issuer and epilogue warps and by the second CTA's producer and epilogue warps
+    for (int i = 0; i < QD; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 2 + 2 * NUM_EPI_WARPS);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -964,11 +1071,31 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   // producer bookkeeping, read again after every role has finished (abort drain)
   uint32_t outstanding = 0;            // stages with a load issued and not yet seen consumed
   uint32_t out_phase = 0;              // bit s: phase parity of stage s's last issued load
+  const bool dyn = QD > 0 && P.dynamic;
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer (both CTAs)
+    // ---------------- TMA producer (both CTAs; with the tile queue, the leader's publishes)
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+    TileQueue q = make_queue(q_tile, q_full, q_empty, rank);
+    int t = -1, t_next = pair < n_tiles ? pair : -1;   // the leader claims one tile ahead
+    for (int it = 0; !*abort_flag; ++it) {
+      if constexpr (QD > 0) {
+        if (dyn && rank == 0) {
+          t = t_next;
+          if (!q_publish<QD>(q, t, abort_flag, budget)) break;
+          if (t >= 0) {
+            const int c = n_pairs + atomicAdd(P.sched, 1);
+            t_next = c < n_tiles ? c : -1;
+          }
+        } else if (dyn) {
+          if (!q_take<QD>(q, t, abort_flag, budget)) break;
+        } else {
+          t = static_next(it, t, pair, n_pairs, n_tiles);
+        }
+      } else {
+        t = static_next(it, t, pair, n_pairs, n_tiles);
+      }
+      if (t < 0) break;
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       bool ok = true;
@@ -997,7 +1124,19 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
     // test hook: `drain` gets no arrival before an abort, so this wait runs out after `budget`
     // and raises the abort flag before any MMA is issued
     if (P.stall) wait_bounded(drain, 0u, abort_flag, budget);
-    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs) {
+    TileQueue q = make_queue(q_tile, q_full, q_empty, rank);
+    int t = -1;
+    for (int it = 0; !*abort_flag; ++it) {
+      if constexpr (QD > 0) {
+        if (dyn) {
+          if (!q_take<QD>(q, t, abort_flag, budget)) break;
+        } else {
+          t = static_next(it, t, pair, n_pairs, n_tiles);
+        }
+      } else {
+        t = static_next(it, t, pair, n_pairs, n_tiles);
+      }
+      if (t < 0) break;
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       if (!wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, budget)) break;
@@ -1052,7 +1191,19 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       }
       for (int i = 0; i < NG && gc.t < n_tiles; ++i) gcursor_issue<KIND>(P, sched, quarter, lane, gc, gr);
     }
-    for (int t = pair; t < n_tiles && !*abort_flag; t += n_pairs, ++tcount) {
+    TileQueue q = make_queue(q_tile, q_full, q_empty, rank);
+    int t = -1;
+    for (int it = 0; !*abort_flag; ++it, ++tcount) {
+      if constexpr (QD > 0) {
+        if (dyn) {
+          if (!q_take_warp<QD>(q, t, lane, abort_flag, budget)) break;
+        } else {
+          t = static_next(it, t, pair, n_pairs, n_tiles);
+        }
+      } else {
+        t = static_next(it, t, pair, n_pairs, n_tiles);
+      }
+      if (t < 0) break;
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
       if (!epilogue_tile<KIND>(P, tl, tmem_base + (uint32_t)(acc * BN), nk, quarter, sub, lane,
@@ -1218,9 +1369,11 @@ moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, cons
 }
 
 moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
-                             const void* W1, const void* W3, void* dXd, uint32_t* status,
-                             cudaStream_t st) {
+                             const void* W1, const void* W3, void* dXd, int* zero, int zero_n,
+                             uint32_t* status, cudaStream_t st) {
   Params P = base_params(D, offsets, status);
+  P.zero = zero;
+  P.zero_n = zero_n;
   bool ok = map2(&P.a_main, dU, D.F, D.R, 64, BM) && map3(&P.b_main, W1, D.d, D.F, D.E_tot, 64, 64);
   if (D.act == MOE_ACT_SWIGLU)
     ok = ok && map2(&P.a_alt, dV, D.F, D.R, 64, BM) && map3(&P.b_alt, W3, D.d, D.F, D.E_tot, 64, 64);
@@ -1238,11 +1391,13 @@ moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, cons
 // are read MN-major as they are.
 moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* X,
                                const void* xs, const int32_t* offsets, float* dW1, float* dW3,
-                               uint32_t* status, cudaStream_t st) {
+                               int* sched, uint32_t* status, cudaStream_t st) {
   const bool km = wgrad_kmajor(D);
   for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
     P.kmajor = km ? 1 : 0;
+    P.dynamic = 1;
+    P.sched = sched + pass;
     bool ok = map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64);
     if (km)
       ok = ok && map2(&P.b_main, X, D.R, D.d, 64, BNH) &&
@@ -1266,11 +1421,13 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
 // dW2 = dO^T H  -- M = d, N = F.  With wgrad_kmajor(D), A comes K-major from dOt [d][R] (routed
 // groups) or dyt [d][T_pad] (shared experts); otherwise dO and dy are read MN-major as they are.
 moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* G, const void* gs,
-                              const int32_t* offsets, float* dW2, uint32_t* status,
+                              const int32_t* offsets, float* dW2, int* sched, uint32_t* status,
                               cudaStream_t st) {
   const bool km = wgrad_kmajor(D);
   Params P = base_params(D, offsets, status);
   P.kmajor = km ? 1 : 0;
+  P.dynamic = 1;
+  P.sched = sched;
   bool ok = map2(&P.b_main, H, D.F, D.R, 64, 64);
   if (km)
     ok = ok && map2(&P.a_main, G, D.R, D.d, 64, BM) &&

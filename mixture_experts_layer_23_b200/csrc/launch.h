@@ -93,19 +93,21 @@ moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* of
 moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, const int32_t* offsets,
                              const void* W2, const void* U, const void* V, void* dU, void* dV,
                              uint32_t* status, cudaStream_t st);
+// zero[0..zero_n): the weight gradients' tile counters, reset by this launch (it always runs first)
 moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
-                             const void* W1, const void* W3, void* dXd, uint32_t* status,
-                             cudaStream_t st);
+                             const void* W1, const void* W3, void* dXd, int* zero, int zero_n,
+                             uint32_t* status, cudaStream_t st);
 // The weight gradients.  With wgrad_kmajor(D) they read one operand through a column-major copy
 // (launch_transpose_bf16): X / xs are Xdt [d][R] (routed columns) / xt [d][T_pad] (shared experts)
 // and G / gs are dOt [d][R] / dyt [d][T_pad], xs and gs null without shared experts; otherwise X,
 // xs, G, gs are Xd, x, dO, dy themselves (all valid pointers).
 bool wgrad_kmajor(const Dims& D);
+// sched: zeroed tile counters, one per launch (w13: dW1 at [0], dW3 at [1]; w2: [0])
 moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, const void* X,
                                const void* xs, const int32_t* offsets, float* dW1, float* dW3,
-                               uint32_t* status, cudaStream_t st);
+                               int* sched, uint32_t* status, cudaStream_t st);
 moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* G, const void* gs,
-                              const int32_t* offsets, float* dW2, uint32_t* status,
+                              const int32_t* offsets, float* dW2, int* sched, uint32_t* status,
                               cudaStream_t st);
 
 }  // namespace moe

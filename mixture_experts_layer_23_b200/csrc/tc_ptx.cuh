@@ -246,6 +246,10 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 // arrive (release, cluster scope) on an mbarrier given by its shared::cluster address
+// 32-bit store into the shared memory of a CTA of the cluster (shared::cluster address)
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
