@@ -244,8 +244,7 @@ moe_status moe_expert_ffn_bwd(const moe_config_t* cfg, const void* dO, const voi
                               const void* Gv, const void* H, void* dXd, float* dW1, float* dW3,
                               float* dW2, void* scratch, moe_stream_t stream);
 
-/* Steps 1-2 backward on the token side, after moe_combine_bwd on the same scratch (which also
- * resets the arrival counters the tensor-core dWg keeps in scratch):
+/* Steps 1-2 backward on the token side, after moe_combine_bwd on the same scratch:
  * dWg [E,d] = dlogits^T x (float, overwritten) and dx [T,d] = dlogits Wg + the sum of each
  * token's kept rows of dXd and its shared experts' rows (fixed-order sums, no float atomics). */
 moe_status moe_router_bwd(const moe_config_t* cfg, const void* ctx, const void* x, const void* Wg,

@@ -123,11 +123,7 @@ ScratchLayout scratch_layout(const Dims& D) {
   S.dlogits = take(T * D.E * 4);
   S.dWg_part = take((size_t)D.n_tchunk * D.E * D.d * 4);
   S.dl16 = 0;
-  S.rw_count = 0;
-  if (router_bwd_tc_supported(D)) {
-    S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
-    S.rw_count = take((size_t)(D.d + 127) / 128 * 4);
-  }
+  if (router_bwd_tc_supported(D)) S.dl16 = take(T * (size_t)round_up(D.E, 8) * 2);
   S.aux_part = take((size_t)D.n_aux * D.E * 4);
   S.wg_sched = take(16);
   S.Xdt = S.dOt = S.xt = S.dyt = 0;
@@ -443,9 +439,7 @@ static moe_status bwd_combine(const Dims& D, const moe_layout_t& L, const Scratc
                             (const float*)(c + L.ctx_topk_w), (const int32_t*)(c + L.ctx_topk_idx),
                             (const float*)(c + L.ctx_logits), (const int32_t*)(c + L.ctx_kept),
                             (const int32_t*)(c + L.ctx_offsets), (const int32_t*)(c + L.ctx_counts),
-                            (float*)(s + S.dg), (float*)(s + S.dlogits), dl16, dO,
-                            S.rw_count ? (int32_t*)(s + S.rw_count) : nullptr,
-                            S.rw_count ? (D.d + 127) / 128 : 0, st);
+                            (float*)(s + S.dg), (float*)(s + S.dlogits), dl16, dO, st);
 }
 
 // Router weight gradient dWg = dl^T x (tensor cores over token chunks for bf16 with d % 64 == 0,
@@ -453,9 +447,12 @@ static moe_status bwd_combine(const Dims& D, const moe_layout_t& L, const Scratc
 static moe_status bwd_router_wgrad(const Dims& D, const ScratchLayout& S, char* s, const void* x,
                                    float* dWg, cudaStream_t st) {
   float* part = (float*)(s + S.dWg_part);
-  if (S.dl16)   // the chunk partials' sum is folded into the kernel (counters zeroed by bwd_combine)
-    return launch_router_wgrad_tc(D, (const __nv_bfloat16*)(s + S.dl16), x, part, dWg,
-                                  (int*)(s + S.rw_count), (uint32_t*)(s + S.status), st);
+  if (S.dl16) {
+    int n_chunks = 0;
+    MOE_TRY(launch_router_wgrad_tc(D, (const __nv_bfloat16*)(s + S.dl16), x, part, &n_chunks,
+                                   (uint32_t*)(s + S.status), st));
+    return launch_router_wgrad_reduce(D, part, n_chunks, dWg, st);
+  }
   return launch_router_wgrad(D, (const float*)(s + S.dlogits), x, part, dWg, st);
 }
 

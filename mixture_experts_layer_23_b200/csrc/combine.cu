@@ -202,10 +202,8 @@ combine_bwd_kernel(const T* __restrict__ dy, const T* __restrict__ O,
                    const int32_t* __restrict__ counts, float aux_scale, float inv_Tk, int T_,
                    int d, int E, int k, int gate_norm, int n_tok_blocks, float* __restrict__ dg,
                    float* __restrict__ dlogits, __nv_bfloat16* __restrict__ dl16, int E8,
-                   T* __restrict__ dO, int32_t* __restrict__ zero, int n_zero) {
+                   T* __restrict__ dO) {
   pdl_prologue();
-  // the arrival counters of the router weight gradient launched after this kernel
-  if (blockIdx.x == 0 && (int)threadIdx.x < n_zero) zero[threadIdx.x] = 0;
   constexpr int VN = Vec16<T>::N;
   constexpr int U = KS >= 8 ? 1 : 8 / KS;
   const int lane = threadIdx.x & 31;
@@ -318,33 +316,30 @@ static moe_status combine_bwd_t(const Dims& D, const void* dy, const void* O, co
                                 const float* topk_w, const int32_t* topk_idx,
                                 const float* logits, const int32_t* kept, const int32_t* offsets,
                                 const int32_t* counts, float* dg, float* dlogits,
-                                __nv_bfloat16* dl16, void* dO, int32_t* zero, int n_zero,
-                                cudaStream_t st) {
+                                __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
   const int n_tok_blocks = (D.T + 7) / 8;
   return launch_k(combine_bwd_kernel<T, KS>, n_tok_blocks + D.E, 256, 0, st, 1, (const T*)dy,
                   (const T*)O, slot, topk_w, topk_idx, logits, kept, offsets, counts,
                   D.aux_coef > 0.f ? D.aux_coef * (float)D.E / (float)D.T : 0.f,
                   1.f / ((float)D.T * (float)D.k), D.T, D.d, D.E, D.k,
-                  D.gate_norm, n_tok_blocks, dg, dlogits, dl16, (int)round_up(D.E, 8), (T*)dO,
-                  zero, n_zero);
+                  D.gate_norm, n_tok_blocks, dg, dlogits, dl16, (int)round_up(D.E, 8), (T*)dO);
 }
 template <typename T>
 static moe_status combine_bwd_ks(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                                  const float* topk_w, const int32_t* topk_idx,
                                  const float* logits, const int32_t* kept,
                                  const int32_t* offsets, const int32_t* counts, float* dg,
-                                 float* dlogits, __nv_bfloat16* dl16, void* dO, int32_t* zero,
-                                 int n_zero, cudaStream_t st) {
+                                 float* dlogits, __nv_bfloat16* dl16, void* dO, cudaStream_t st) {
   switch (pow2_at_least(D.k)) {
     case 1: case 2:
       return combine_bwd_t<T, 2>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
-                                 counts, dg, dlogits, dl16, dO, zero, n_zero, st);
+                                 counts, dg, dlogits, dl16, dO, st);
     case 4:
       return combine_bwd_t<T, 4>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
-                                 counts, dg, dlogits, dl16, dO, zero, n_zero, st);
+                                 counts, dg, dlogits, dl16, dO, st);
     default:
       return combine_bwd_t<T, 8>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
-                                 counts, dg, dlogits, dl16, dO, zero, n_zero, st);
+                                 counts, dg, dlogits, dl16, dO, st);
   }
 }
 
@@ -352,13 +347,12 @@ moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, cons
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
                               const int32_t* kept, const int32_t* offsets, const int32_t* counts,
                               float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
-                              int32_t* zero, int n_zero, cudaStream_t st) {
-  if (n_zero < 0 || n_zero > 256) return MOE_ERR_INVALID_ARG;
+                              cudaStream_t st) {
   if (D.dtype == MOE_DTYPE_BF16)
     return combine_bwd_ks<__nv_bfloat16>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets,
-                                         counts, dg, dlogits, dl16, dO, zero, n_zero, st);
+                                         counts, dg, dlogits, dl16, dO, st);
   return combine_bwd_ks<float>(D, dy, O, slot, topk_w, topk_idx, logits, kept, offsets, counts, dg,
-                               dlogits, dl16, dO, zero, n_zero, st);
+                               dlogits, dl16, dO, st);
 }
 
 }  // namespace moe

@@ -28,7 +28,6 @@ struct ScratchLayout {
   size_t dlogits;       // [T, E] float
   size_t dWg_part;      // [n_tchunk, E, d] float
   size_t dl16;          // [T, E8] bf16 copy of dlogits (tensor-core router backward), or 0
-  size_t rw_count;      // [ceil(d / 128)] int32 arrival counters of the tensor-core dWg (with dl16)
   size_t wg_sched;      // [4] int32 tile counters of the tensor-core weight gradients (dW1, dW3, dW2)
   size_t aux_part;      // [n_aux, E] float partial probability sums of the load-balancing loss
   // column-major copies read K-major by the tensor-core weight gradients (0 on the CUDA-core path)

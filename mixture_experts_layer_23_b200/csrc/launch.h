@@ -19,12 +19,11 @@ moe_status launch_dispatch(const Dims& D, const void* x, const int32_t* topk_idx
                            void* Xd, int32_t* blk_counts, uint32_t* status, cudaStream_t st);
 moe_status launch_combine(const Dims& D, const void* O, const int32_t* slot, const float* topk_w,
                           void* y, cudaStream_t st);
-// zero[0..n_zero) (n_zero <= 256) are set to 0 first: the arrival counters of the tensor-core dWg
 moe_status launch_combine_bwd(const Dims& D, const void* dy, const void* O, const int32_t* slot,
                               const float* topk_w, const int32_t* topk_idx, const float* logits,
                               const int32_t* kept, const int32_t* offsets, const int32_t* counts,
                               float* dg, float* dlogits, __nv_bfloat16* dl16, void* dO,
-                              int32_t* zero, int n_zero, cudaStream_t st);
+                              cudaStream_t st);
 // Router backward on the tensor cores (bf16, d a multiple of 64): dWg partials over token
 // chunks and their fixed-order sum; dl Wg with the un-dispatch gather fused into its epilogue.
 bool router_bwd_tc_supported(const Dims& D);
@@ -37,11 +36,10 @@ moe_status launch_fused_small_fwd(const Dims& D, const void* x, const void* Wg, 
 // Load-balancing loss (forward): loss[0] from the logits and the pre-drop counts.
 moe_status launch_aux_loss(const Dims& D, const float* logits, const int32_t* counts, float* part,
                            float* loss, cudaStream_t st);
-// dWg from chunk partials in `part`, summed in chunk order by the last CTA of each 128-column tile;
-// count: ceil(d / 128) counters, zero on entry (left zero)
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
-                                  float* part, float* dWg, int* count, uint32_t* status,
-                                  cudaStream_t st);
+                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st);
+moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,
+                                      cudaStream_t st);
 moe_status launch_undispatch_tc(const Dims& D, const __nv_bfloat16* dl16, const void* Wg,
                                 const void* dXd, const int32_t* slot, void* dx, uint32_t* status,
                                 cudaStream_t st);

@@ -282,6 +282,13 @@ undispatch_warp_kernel(const float* __restrict__ dl, const T* __restrict__ Wg,
 
 }  // namespace
 
+moe_status launch_router_wgrad_reduce(const Dims& D, const float* part, int n_chunks, float* dWg,
+                                      cudaStream_t st) {
+  const int64_t n = (int64_t)D.E * D.d;
+  return launch_k(router_wgrad_reduce_kernel, (int)((n + 255) / 256), 256, 0, st, 1, part,
+                  n_chunks, n, dWg);
+}
+
 bool undispatch_warp_supported(const Dims& D) {
   const int esz = D.dtype == MOE_DTYPE_BF16 ? 2 : 4;
   return D.E <= 32 && D.k + D.S <= 16 && (size_t)D.E * D.d * esz <= (size_t)96 * 1024;

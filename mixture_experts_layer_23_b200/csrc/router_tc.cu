@@ -267,17 +267,15 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 // every expert at once (N = E rounded up to 64, dl16 read MN-major, one 64-expert swizzle atom per
 // 64 experts).  The MMA work is then 2 d N T flops, a few percent of the time it takes to read x,
 // and x is read exactly once.  Each CTA writes its chunk's partial dWg[e][d] in fp32 (a warp's lanes
-// hold 32 consecutive columns: coalesced); the last CTA of each 128-column tile to finish (an
-// arrival counter per tile) adds the chunks' partials in chunk order into dWg, so no second launch
-// reduces them.  The chunks are sized so that all CTAs fit in one wave at two per SM.
+// hold 32 consecutive columns: coalesced); router_wgrad_reduce adds the chunks in order.  The chunks
+// are sized so that all CTAs fit in one wave at two per SM.  (Folding the sum into this kernel, the
+// last CTA of each 128-column tile adding every chunk's partial, measured slower: on the
+// DeepSeek-style layer that CTA's E x 128 x chunks loads took 136 against 30 us for both launches.)
 
 struct alignas(64) RWParams {
   CUtensorMap x_map;   // x [T, d], box {64 (d), 64 (tokens)}
   CUtensorMap l_map;   // dl16 [T, E8], box {64 (experts), 64 (tokens)}
   float* part;         // [n_chunks][E][d]
-  float* dWg;          // [E][d]: the chunks' sum, written by the last CTA of each column tile
-  int* count;          // [n_dt] CTAs of each column tile done (zero on entry; left zero)
-  int n_chunks;
   uint32_t* status;
   unsigned long long timeout_ns;
   int T, d, E, N, chunk, n_dt;
@@ -384,30 +382,6 @@ __global__ void __launch_bounds__(192, 1) router_wgrad_tc_kernel(const __grid_co
   __syncwarp();
   tc_fence_before();
   __syncthreads();   // every role has finished (the abort flag is final)
-  // The last CTA of this column tile to finish adds the chunks' partials in chunk order (the same
-  // fixed order whichever CTA is last: bit-reproducible) and resets the tile's counter.  An aborted
-  // CTA does not count itself, so after a timeout dWg is left unwritten (the status reports it).
-  __shared__ int last;
-  if (threadIdx.x == 0) {
-    last = 0;
-    if (!*abort_flag) {
-      __threadfence();   // this CTA's partial is visible before its arrival is counted
-      last = atomicAdd(&P.count[dt], 1) == P.n_chunks - 1;
-    }
-  }
-  __syncthreads();
-  if (last) {
-    __threadfence();
-    for (int i = threadIdx.x; i < P.E * 128; i += blockDim.x) {
-      const int e = i / 128, col = d0 + i % 128;
-      if (col >= P.d) continue;
-      float acc = 0.f;
-      for (int cc = 0; cc < P.n_chunks; ++cc)
-        acc += __ldcg(P.part + ((size_t)cc * P.E + e) * P.d + col);
-      P.dWg[(size_t)e * P.d + col] = acc;
-    }
-    if (threadIdx.x == 0) P.count[dt] = 0;
-  }
   if (*abort_flag && warp == 0 && lane == 0) {
     // TMA loads of an aborted CTA may still be in flight: let them land before it exits
     for (int s = 0; s < RSTAGES; ++s)
@@ -486,8 +460,7 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
 }
 
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,
-                                  float* part, float* dWg, int* count, uint32_t* status,
-                                  cudaStream_t st) {
+                                  float* part, int* n_chunks, uint32_t* status, cudaStream_t st) {
   using namespace tc;
   RWParams P;
   memset(&P, 0, sizeof(P));
@@ -526,9 +499,7 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
       return MOE_ERR_CUDA;
     smem_set = (int)smem;
   }
-  P.n_chunks = nc;
-  P.dWg = dWg;
-  P.count = count;
+  *n_chunks = nc;
   return launch_k(router_wgrad_tc_kernel, P.n_dt * nc, 192, smem, st, 1, P);
 }
 
