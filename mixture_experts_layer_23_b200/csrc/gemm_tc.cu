@@ -1318,6 +1318,13 @@ bool wgrad_kmajor(const Dims& D) {
   return tc_supported(D) && (long long)D.T * D.k >= 2048LL * D.E;
 }
 
+// Weight-gradient tiles from the queue (claimed by the pair free first, longest first) only when the
+// layer has shared experts, whose tiles are T_pad rows long against the routed experts' share of
+// T k: measured on the DeepSeek-style layer (K 16384 against ~1000) 1430 -> 1348 us for dW1|dW3 and
+// 729 -> 685 us for dW2; with tiles of equal length the queue's per-tile hand-offs cost more than they
+// balance (GPT-2-style layer 57 -> 65 us, BERT-style 165 -> 182 us).
+static bool wgrad_queue(const Dims& D) { return D.S > 0; }
+
 
 using namespace tc;
 
@@ -1396,7 +1403,7 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
   for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
     P.kmajor = km ? 1 : 0;
-    P.dynamic = 1;
+    P.dynamic = wgrad_queue(D) ? 1 : 0;
     P.sched = sched + pass;
     bool ok = map2(&P.a_main, pass ? dV : dU, D.F, D.R, 64, 64);
     if (km)
@@ -1426,7 +1433,7 @@ moe_status launch_wgrad_w2_tc(const Dims& D, const void* H, const void* G, const
   const bool km = wgrad_kmajor(D);
   Params P = base_params(D, offsets, status);
   P.kmajor = km ? 1 : 0;
-  P.dynamic = 1;
+  P.dynamic = wgrad_queue(D) ? 1 : 0;
   P.sched = sched;
   bool ok = map2(&P.b_main, H, D.F, D.R, 64, 64);
   if (km)
