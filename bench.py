@@ -59,11 +59,40 @@ class L2Flush:
 GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wgrad_w2"}
 
 
-# DRAM traffic of a kernel from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of
-# one launch), keyed by workload and phase.  It stands only for the kernel sources it was taken on:
-# the SHA-256 of those files is stored with it and the bench reports null once they have changed.
+# DRAM traffic of a phase from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of the
+# phase's launches in one step, averaged over the run's steps), keyed by workload and phase.  It
+# stands only for the kernel sources it was taken on: the SHA-256 of those files is stored with it
+# and the bench reports null once they have changed.  The large layers' figures come from the
+# one-pass launch lists of `python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline`
+# (profiles/launches_mixtral_dropless.md, profiles/launches_deepseek_v2.md).
 GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "act_fast.cuh", "common.cuh"]
+WGRAD_SOURCES = GEMM_SOURCES + ["transpose.cu"]
 NCU_TRAFFIC = {
+    # weight-gradient phase: transpose64_kernel + the dW1 and dW3 launches
+    ("mixtral_dropless", "wgrad_w1"): {
+        "bytes": 14112258790,
+        "sources": WGRAD_SOURCES,
+        "sha256": "98cdd15fa617bcadbbb4272181c9334631035f10d7b3f6ba1f2ea70ee655fa9a",
+        "profile": "profiles/launches_mixtral_dropless.md",
+    },
+    ("mixtral_dropless", "expert_up"): {
+        "bytes": 9424231654,
+        "sources": GEMM_SOURCES,
+        "sha256": "3681793c7edf6f65cf0352cbd2526b66350fe704a497e2bd12d5d9f7b2ea969b",
+        "profile": "profiles/launches_mixtral_dropless.md",
+    },
+    ("deepseek_v2", "wgrad_w1"): {   # the dW1 and dW3 launches (no transposes on this layer)
+        "bytes": 2873133107,
+        "sources": WGRAD_SOURCES,
+        "sha256": "98cdd15fa617bcadbbb4272181c9334631035f10d7b3f6ba1f2ea70ee655fa9a",
+        "profile": "profiles/launches_deepseek_v2.md",
+    },
+    ("deepseek_v2", "expert_up"): {
+        "bytes": 2028915302,
+        "sources": GEMM_SOURCES,
+        "sha256": "3681793c7edf6f65cf0352cbd2526b66350fe704a497e2bd12d5d9f7b2ea969b",
+        "profile": "profiles/launches_deepseek_v2.md",
+    },
     # one launch of the up-projection GEMM captured with the command given in
     # profiles/expert_up_gpt2_gshard.md (ncu --set full --clock-control none, one kernel):
     # dram__bytes_read.sum 89.732096 MB + dram__bytes_write.sum 60.708352 MB
