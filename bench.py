@@ -63,8 +63,9 @@ GEMM_PHASES = {"expert_up", "expert_down", "dgrad_h", "dgrad_x", "wgrad_w1", "wg
 # phase's launches in one step, averaged over the run's steps), keyed by workload and phase.  It
 # stands only for the kernel sources it was taken on: the SHA-256 of those files is stored with it
 # and the bench reports null once they have changed.  The large layers' figures come from the
-# one-pass launch lists of `python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline`
-# (profiles/launches_mixtral_dropless.md, profiles/launches_deepseek_v2.md).
+# one-pass launch lists (gpu__time_duration.sum and the two DRAM byte counters) of
+# `python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline`; "profile" names the
+# summary of the capture under profiles/.
 GEMM_SOURCES = ["gemm_tc.cu", "tc_ptx.cuh", "act_fast.cuh", "common.cuh"]
 WGRAD_SOURCES = GEMM_SOURCES + ["transpose.cu"]
 NCU_TRAFFIC = {
@@ -93,8 +94,8 @@ NCU_TRAFFIC = {
         "sha256": "3681793c7edf6f65cf0352cbd2526b66350fe704a497e2bd12d5d9f7b2ea969b",
         "profile": "profiles/launches_deepseek_v2.md",
     },
-    # one launch of the up-projection GEMM captured with the command given in
-    # profiles/expert_up_gpt2_gshard.md (ncu --set full --clock-control none, one kernel):
+    # one launch of the up-projection GEMM (ncu --set full --clock-control none, one kernel, on
+    # `python bench.py --workload gpt2_gshard --steps 1 --warmup 1 --no-cpu-baseline`):
     # dram__bytes_read.sum 89.732096 MB + dram__bytes_write.sum 60.708352 MB
     ("gpt2_gshard", "expert_up"): {
         "bytes": 150440448,
