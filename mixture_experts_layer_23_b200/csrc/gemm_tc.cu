@@ -57,6 +57,9 @@ constexpr uint32_t B_BYTES = BNH * BK * 2;          // 16 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES; // per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int MAX_GROUPS = 264;
+#ifndef MOE_HALF_N_EDGE
+#define MOE_HALF_N_EDGE 1   // N = 128 MMAs for tiles with at most 128 valid columns (see half_n)
+#endif
 #ifndef MOE_TILE_GROUP_M
 #define MOE_TILE_GROUP_M 16
 #endif
@@ -263,6 +266,16 @@ __device__ __forceinline__ int k_blocks(const Params& P, const Tile& t) {
   return P.K / BK;
 }
 
+// A tile whose valid columns fit in half of BN (the last N tile of, for example, F = 1408) runs
+// N = 128 MMAs with each CTA staging 64 rows of B, instead of a full 256-column tile half of which
+// is zero.  Only kinds whose B is read MN-major in 64-row boxes.
+template <int KIND>
+__device__ __forceinline__ bool half_n(const Params& P, const Tile& t) {
+  const bool kinds = KIND == DGRAD_H || KIND == DGRAD_X ||
+                     (KIND == WGRAD && !(P.kmajor && P.which == 0));
+  return MOE_HALF_N_EDGE && kinds && P.N - t.n * BN <= BNH;
+}
+
 // ----------------------------------------------------------------------------- producer
 //
 // Each CTA loads its own half: A rows [mrow, mrow + 128) and B rows [nb, nb + 128) with
@@ -274,7 +287,9 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
                                             uint8_t* sA, uint8_t* sB, uint32_t bar) {
   const bool swiglu = P.act == MOE_ACT_SWIGLU;
   const int k0 = kb * BK;
-  const int nb = t.n * BN + rank * BNH;
+  const bool hn = half_n<KIND>(P, t);
+  const int nb = t.n * BN + rank * (hn ? BNH / 2 : BNH);
+  const int nbj = hn ? 1 : BNH / 64;   // 64-row B boxes of an MN-major B
   if (KIND == UP) {
     if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
     else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
@@ -286,16 +301,14 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
   } else if (KIND == DGRAD_H) {
     if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
     else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
-#pragma unroll
-    for (int j = 0; j < BNH / 64; ++j)
+    for (int j = 0; j < nbj; ++j)
       tma_load_3d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, k0, t.g);
   } else if (KIND == DGRAD_X || KIND == UNDISPATCH) {
     const int nkF = P.K / BK;
     const bool second = kb >= nkF;
     const int kk = (second ? kb - nkF : kb) * BK;
     tma_load_2d_pair(sA, second ? &P.a_alt : &P.a_main, bar, kk, t.o_row + t.mrow);
-#pragma unroll
-    for (int j = 0; j < BNH / 64; ++j)
+    for (int j = 0; j < nbj; ++j)
       tma_load_3d_pair(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
   } else if (P.kmajor) {
     // WGRAD, K over the group's rows, one operand read through its column-major copy (K-major,
@@ -312,8 +325,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
       // A = dO^T (routed) or dy^T (shared), K-major; B = H rows of the group (MN-major)
       if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
       else tma_load_2d_pair(sA, &P.a_main, bar, t.a_row + k0, t.mrow);
-#pragma unroll
-      for (int j = 0; j < BNH / 64; ++j)
+      for (int j = 0; j < nbj; ++j)
         tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
     }
   } else {  // WGRAD, both operands straight from the token-major rows (MN-major)
@@ -322,8 +334,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 #pragma unroll
       for (int j = 0; j < BM / 64; ++j)
         tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
-#pragma unroll
-      for (int j = 0; j < BNH / 64; ++j) {
+      for (int j = 0; j < nbj; ++j) {
         if (t.shared) tma_load_2d_pair(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
         else tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
       }
@@ -334,8 +345,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
         if (t.shared) tma_load_2d_pair(sA + j * 8192, &P.a_alt, bar, t.mrow + 64 * j, k0);
         else tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.a_row + k0);
       }
-#pragma unroll
-      for (int j = 0; j < BNH / 64; ++j)
+      for (int j = 0; j < nbj; ++j)
         tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
     }
   }
@@ -1070,6 +1080,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
   const bool B_MN = (KIND == DGRAD_H || KIND == DGRAD_X || KIND == UNDISPATCH) ||
                     ((KIND == WGRAD) && (P.which != 0 || !P.kmajor));
   const uint32_t IDESC = make_idesc(A_MN, B_MN);
+  const uint32_t IDESC_HALF = idesc_bf16(BMP, BN / 2, A_MN, B_MN);   // N = 128 edge tiles
 
   // producer bookkeeping, read again after every role has finished (abort drain)
   uint32_t outstanding = 0;            // stages with a load issued and not yet seen consumed
@@ -1101,11 +1112,12 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       if (t < 0) break;
       const Tile tl = decode<KIND>(P, tile_start, n_groups, t, rank);
       const int nk = k_blocks<KIND>(P, tl);
+      const bool hn = half_n<KIND>(P, tl);
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) { ok = false; break; }
         outstanding &= ~(1u << stage);
-        if (rank == 0) mbar_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        if (rank == 0) mbar_expect_tx(&full[stage], hn ? 2 * (A_BYTES + B_BYTES / 2) : 2 * STAGE_BYTES);
         uint8_t* sA = tiles + stage * STAGE_BYTES;
         issue_loads<KIND>(P, tl, kb, rank, sA, sA + A_BYTES, mapa_shared(smem_u32(&full[stage]), 0));
         outstanding |= 1u << stage;
@@ -1145,6 +1157,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
       if (!wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, abort_flag, budget)) break;
       tc_fence_after();
       const uint32_t dtm = tmem_base + (uint32_t)(acc * BN);
+      const uint32_t idesc = half_n<KIND>(P, tl) ? IDESC_HALF : IDESC;
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb) {
         if (!wait_bounded(&full[stage], phase, abort_flag, budget)) { ok = false; break; }
@@ -1155,7 +1168,7 @@ grouped_gemm_kernel(const __grid_constant__ Params P) {
         for (int k = 0; k < BK / 16; ++k) {
           const uint64_t ad = sw128_desc(sa + k * a_step, a_lbo, 1024);
           const uint64_t bd = sw128_desc(sb + k * b_step, b_lbo, 1024);
-          umma_bf16_pair(dtm, ad, bd, IDESC, (kb > 0 || k > 0) ? 1u : 0u);
+          umma_bf16_pair(dtm, ad, bd, idesc, (kb > 0 || k > 0) ? 1u : 0u);
         }
         issued_any = true;
         umma_commit_pair(&empty[stage], 0x3);   // frees this stage in both CTAs
