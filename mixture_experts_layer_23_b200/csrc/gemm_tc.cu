@@ -1377,8 +1377,10 @@ moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* of
 
 moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, const int32_t* offsets,
                              const void* W2, const void* U, const void* V, void* dU, void* dV,
-                             uint32_t* status, cudaStream_t st) {
+                             int* zero, int zero_n, uint32_t* status, cudaStream_t st) {
   Params P = base_params(D, offsets, status);
+  P.zero = zero;
+  P.zero_n = zero_n;
   if (!(map2(&P.a_main, dO, D.d, D.R, 64, BM) && map2(&P.a_alt, dy, D.d, D.T, 64, BM) &&
         map3(&P.b_main, W2, D.F, D.d, D.E_tot, 64, 64)))
     return MOE_ERR_CUDA;
