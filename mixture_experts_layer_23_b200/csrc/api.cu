@@ -5,8 +5,6 @@
 #include <stdio.h>
 #include <string.h>
 
-#include <mutex>
-
 #include "launch.h"
 #include "tc_host.h"
 
@@ -203,35 +201,6 @@ static moe_status expert_fwd(const Dims& D, const void* Xd, const void* x, const
   return launch_expert_down_simt(D, H, offsets, W2, O, st);
 }
 
-// Side streams of the concurrent expert backward, created once per device and kept for the
-// process (with the fork and join events); null if they cannot be created.
-#ifndef MOE_BWD_CONCURRENT
-#define MOE_BWD_CONCURRENT 0
-#endif
-struct SideStreams {
-  cudaStream_t s[2];
-  cudaEvent_t fork, join[2];
-};
-static SideStreams* side_streams() {
-  constexpr int kMaxDevices = 64;
-  static SideStreams side[kMaxDevices];
-  static bool made[kMaxDevices] = {};
-  static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!made[dev]) {
-    SideStreams& z = side[dev];
-    for (int i = 0; i < 2; ++i) {
-      if (cudaStreamCreateWithFlags(&z.s[i], cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-      if (cudaEventCreateWithFlags(&z.join[i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
-    }
-    if (cudaEventCreateWithFlags(&z.fork, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-    made[dev] = true;
-  }
-  return &side[dev];
-}
-
 // Expert FFN backward: dgrad through W2 and the activation, dgrad through W1 (and W3), then the
 // weight gradients; with phase_marks, the profiling events of backward phases 3..5 between them.
 // The expert GEMMs' backward.  s / S: the scratch area, for the tensor-core path's transposed
@@ -245,43 +214,6 @@ static moe_status expert_bwd(const Dims& D, const void* dO, const void* dy, cons
   uint32_t* status = (uint32_t*)(s + S.status);
   if (tc_supported(D)) {
     int* wg_sched = (int*)(s + S.wg_sched);   // the weight gradients' tile counters
-    SideStreams* side = (MOE_BWD_CONCURRENT && !phase_marks) ? side_streams() : nullptr;
-    if (side) {
-      // after the activation gradient (which zeroes the counters) the input gradient and the two
-      // weight gradients are independent: they run on three streams, so each one's last partial
-      // wave overlaps the others
-      MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, wg_sched, 4, status, st));
-      const void *X = Xd, *xs = x, *G = dO, *gs = dy;
-      if (wgrad_kmajor(D)) {
-        const long long r0 = D.routed_row0, nr = D.R - D.routed_row0;
-        TransposeSpec js[4] = {
-            {Xd, s + S.Xdt, D.d, D.R, r0, r0, nr, -1, D.d},
-            {dO, s + S.dOt, D.d, D.R, r0, r0, nr, -1, D.d}};
-        int nj = 2;
-        if (D.S > 0) {
-          js[nj++] = {x, s + S.xt, D.d, D.T_pad, 0, 0, D.T_pad, D.T, D.d};
-          js[nj++] = {dy, s + S.dyt, D.d, D.T_pad, 0, 0, D.T_pad, D.T, D.d};
-        }
-        MOE_TRY(launch_transpose_bf16(js, nj, st));
-        X = s + S.Xdt;
-        xs = D.S > 0 ? s + S.xt : nullptr;
-        G = s + S.dOt;
-        gs = D.S > 0 ? s + S.dyt : nullptr;
-      }
-      if (cudaEventRecord(side->fork, st) != cudaSuccess ||
-          cudaStreamWaitEvent(side->s[0], side->fork, 0) != cudaSuccess ||
-          cudaStreamWaitEvent(side->s[1], side->fork, 0) != cudaSuccess)
-        return MOE_ERR_CUDA;
-      MOE_TRY(launch_wgrad_w13_tc(D, dU, dV, X, xs, offsets, dW1, dW3, wg_sched, status,
-                                  side->s[0]));
-      MOE_TRY(launch_wgrad_w2_tc(D, H, G, gs, offsets, dW2, wg_sched + 2, status, side->s[1]));
-      MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, nullptr, 0, status, st));
-      for (int i = 0; i < 2; ++i)
-        if (cudaEventRecord(side->join[i], side->s[i]) != cudaSuccess ||
-            cudaStreamWaitEvent(st, side->join[i], 0) != cudaSuccess)
-          return MOE_ERR_CUDA;
-      return MOE_OK;
-    }
     MOE_TRY(launch_dgrad_h_tc(D, dO, dy, offsets, W2, Gu, Gv, dU, dV, nullptr, 0, status, st));
     if (phase_marks) MOE_TRY(mark_bwd(3, st));
     MOE_TRY(launch_dgrad_x_tc(D, dU, dV, offsets, W1, W3, dXd, wg_sched, 4, status, st));

@@ -91,8 +91,8 @@ moe_status launch_expert_down_tc(const Dims& D, const void* H, const int32_t* of
 moe_status launch_dgrad_h_tc(const Dims& D, const void* dO, const void* dy, const int32_t* offsets,
                              const void* W2, const void* U, const void* V, void* dU, void* dV,
                              int* zero, int zero_n, uint32_t* status, cudaStream_t st);
-// zero[0..zero_n): the weight gradients' tile counters, reset by the launch that runs before them
-// (the input gradient, or the activation gradient when the three run concurrently)
+// zero[0..zero_n): the weight gradients' tile counters, reset by the input gradient that runs
+// before them
 moe_status launch_dgrad_x_tc(const Dims& D, const void* dU, const void* dV, const int32_t* offsets,
                              const void* W1, const void* W3, void* dXd, int* zero, int zero_n,
                              uint32_t* status, cudaStream_t st);
