@@ -150,6 +150,7 @@ struct alignas(64) Params {
   int act;
   int which;             // WGRAD: 0 -> A = dU|dV (row space), B = Xd|x;  2 -> A = dO|dy, B = H
   int kmajor;            // WGRAD: B (which 0) or A (which 2) read K-major from its transposed copy
+  int wtrans;            // WGRAD: the tiles are of the weight gradient's transpose (stored transposed)
   int chunk;             // > 0: the groups are fixed chunks of this many token rows (router
                          // backward) instead of the experts' row ranges
   int stall;             // failure-path test: the MMA issuer first waits on a barrier that
@@ -659,6 +660,16 @@ __device__ __forceinline__ bool epilogue_tile(const Params& P, const Tile& t, ui
       }
       if constexpr (Cfg<KIND>::DIRECT) {
         st_row_f32(P.out, P.out_ld, (long long)t.g * P.Mw + m_row0 + lane, n, a);
+      } else if (P.wtrans) {
+        // the accumulator holds the transpose of the weight gradient's tile (rows = its columns):
+        // lane l writes its 32 values down column l of the 32 x 32 box, in the 128-byte swizzle
+        // the TMA store reads (16-byte unit u of row r at unit u ^ (r % 8): conflict-free)
+        uint8_t* slot = ring_take(ring, lane);
+#pragma unroll
+        for (int f = 0; f < 32; ++f)
+          *reinterpret_cast<float*>(slot + f * 128 + ((((lane >> 2) ^ (f & 7)) << 4)) +
+                                    (lane & 3) * 4) = a[f];
+        ring_store_3d(&P.o0, slot, m_row0, n, t.g, lane);
       } else {
         uint8_t* slot = ring_take(ring, lane);
         slot_put_f32(slot, lane, a);
@@ -1418,7 +1429,34 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
                                const void* xs, const int32_t* offsets, float* dW1, float* dW3,
                                int* sched, uint32_t* status, cudaStream_t st) {
   const bool km = wgrad_kmajor(D);
-  for (int pass = 0; pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
+  // dW1^T = X^T dU when F ends in a partial N tile of at most 128 columns and d fills its M tiles:
+  // the dW2 form (A = X, B = dU|dV), edge tiles of N = 128, tiles stored transposed.  In the direct
+  // orientation the last M tile of F = 1408 would be half empty (the pair computing 256 rows for 128).
+  const bool swap = !MOE_GEMM_DIRECT_STORE && D.F % BMP != 0 && D.F % BMP <= BNH && D.d % BMP == 0;
+  for (int pass = 0; swap && pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
+    Params P = base_params(D, offsets, status);
+    P.kmajor = km ? 1 : 0;
+    P.dynamic = wgrad_queue(D) ? 1 : 0;
+    P.sched = sched + pass;
+    P.wtrans = 1;
+    bool ok = map2(&P.b_main, pass ? dV : dU, D.F, D.R, 64, 64);
+    if (km)
+      ok = ok && map2(&P.a_main, X, D.R, D.d, 64, BM) &&
+           (D.S == 0 || map2(&P.a_alt, xs, D.T_pad, D.d, 64, BM));
+    else
+      ok = ok && map2(&P.a_main, X, D.d, D.R, 64, 64) && map2(&P.a_alt, xs, D.d, D.T, 64, 64);
+    if (!ok) return MOE_ERR_CUDA;
+    if (!map3_f32(&P.o0, pass ? dW3 : dW1, D.d, D.F, D.E_tot, 32, 32)) return MOE_ERR_CUDA;
+    P.out = pass ? dW3 : dW1;
+    P.out_ld = D.d;
+    P.Mw = D.d;
+    P.N = D.F;
+    P.which = 2;   // the dW2 form: A's rows are the expert's routed rows, B's the row space
+    const int tiles = D.E_tot * ((D.d + BMP - 1) / BMP) * ((D.F + BN - 1) / BN);
+    const moe_status s = launch<WGRAD>(P, tiles, st);
+    if (s != MOE_OK) return s;
+  }
+  for (int pass = 0; !swap && pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
     P.kmajor = km ? 1 : 0;
     P.dynamic = wgrad_queue(D) ? 1 : 0;

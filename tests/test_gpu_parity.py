@@ -145,6 +145,13 @@ EDGE_WGRAD = [
                act=SWIGLU, capacity_factor=1.25, dtype=BF16, bias="normal"),
     LayerShape("kmajor_wgrad_gelu_top1", T=4200, d=192, E=2, k=1, d_ff=128, act=GELU,
                capacity_factor=None, dtype=BF16),
+    # F ending in a partial tile of at most 128 columns with d a multiple of 256: dW1 and dW3 are
+    # computed transposed (stored through the transposing epilogue) with N = 128 edge tiles; with
+    # the K-major operand and a shared expert, and without
+    LayerShape("transposed_dw1_kmajor_shared", T=2100, d=256, E=2, k=2, d_ff=320, n_shared=1,
+               act=SWIGLU, capacity_factor=1.25, dtype=BF16, bias="normal"),
+    LayerShape("transposed_dw1_gelu", T=300, d=512, E=4, k=2, d_ff=64, act=GELU,
+               capacity_factor=1.0, dtype=BF16),
 ]
 
 
