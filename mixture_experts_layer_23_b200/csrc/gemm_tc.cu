@@ -60,6 +60,9 @@ constexpr int MAX_GROUPS = 264;
 #ifndef MOE_HALF_N_EDGE
 #define MOE_HALF_N_EDGE 1   // N = 128 MMAs for tiles with at most 128 valid columns (see half_n)
 #endif
+#ifndef MOE_WGRAD_TRANSPOSED_W13
+#define MOE_WGRAD_TRANSPOSED_W13 1   // dW1, dW3 computed transposed when F ends in a short tile
+#endif
 #ifndef MOE_TILE_GROUP_M
 #define MOE_TILE_GROUP_M 16
 #endif
@@ -1432,7 +1435,7 @@ moe_status launch_wgrad_w13_tc(const Dims& D, const void* dU, const void* dV, co
   // dW1^T = X^T dU when F ends in a partial N tile of at most 128 columns and d fills its M tiles:
   // the dW2 form (A = X, B = dU|dV), edge tiles of N = 128, tiles stored transposed.  In the direct
   // orientation the last M tile of F = 1408 would be half empty (the pair computing 256 rows for 128).
-  const bool swap = !MOE_GEMM_DIRECT_STORE && D.F % BMP != 0 && D.F % BMP <= BNH && D.d % BMP == 0;
+  const bool swap = MOE_WGRAD_TRANSPOSED_W13 && !MOE_GEMM_DIRECT_STORE && D.F % BMP != 0 && D.F % BMP <= BNH && D.d % BMP == 0;
   for (int pass = 0; swap && pass < (D.act == MOE_ACT_SWIGLU ? 2 : 1); ++pass) {
     Params P = base_params(D, offsets, status);
     P.kmajor = km ? 1 : 0;

@@ -27,6 +27,9 @@ namespace tc {
 namespace {
 
 constexpr int MAX_RSTAGES = 16;
+#ifndef MOE_ROUTER_ISSUE_GROUP
+#define MOE_ROUTER_ISSUE_GROUP 1
+#endif
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
 constexpr int STAGE_MAX_EPAD = 64;            // rows of at most 64 logits are staged in shared memory
 
@@ -119,16 +122,30 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   if (warp == 0 && lane == 0) {
     int stage = 0;
     uint32_t phase = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, budget)) break;
-      outstanding &= ~(1u << stage);
-      mbar_expect_tx(&full[stage], (uint32_t)(P.rows + P.E_pad) * 128u);
-      uint8_t* sA = smem + stage * P.stage_bytes;
-      tma_load_2d(sA, &P.x_map, &full[stage], kb * 64, m0);
-      tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], kb * 64, 0);
-      outstanding |= 1u << stage;
-      out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
-      if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
+    // loads leave in groups of G consecutive k blocks: the producer waits until G stages are free,
+    // then issues them back to back, so that the G 128-byte pieces of each token row reach the
+    // memory system together
+    const int G = min(MOE_ROUTER_ISSUE_GROUP, RSTAGES);
+    bool ok = true;
+    for (int kb0 = 0; ok && kb0 < nk; kb0 += G) {
+      const int gn = min(G, nk - kb0);
+      int s = stage;
+      uint32_t ph = phase;
+      for (int j = 0; j < gn; ++j) {
+        if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, budget)) { ok = false; break; }
+        outstanding &= ~(1u << s);
+        if (++s == RSTAGES) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      for (int kb = kb0; kb < kb0 + gn; ++kb) {
+        mbar_expect_tx(&full[stage], (uint32_t)(P.rows + P.E_pad) * 128u);
+        uint8_t* sA = smem + stage * P.stage_bytes;
+        tma_load_2d(sA, &P.x_map, &full[stage], kb * 64, m0);
+        tma_load_2d(sA + RA_BYTES, &P.w_map, &full[stage], kb * 64, 0);
+        outstanding |= 1u << stage;
+        out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
+        if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
+      }
     }
   } else if (warp == 1 && lane == 0) {
     int stage = 0;
