@@ -73,8 +73,16 @@ fused_small_fwd_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
     topk_init(st);
 #pragma unroll
     for (int e = 0; e < FS_MAX_E; ++e)
-      if (e < E) topk_push(st, lg[e] + (bias ? bias[e] : 0.f), e);
-    topk_finish(st, k, gate_norm, sidx + (size_t)t * k, sw + (size_t)t * k);
+      if (e < E) {
+        lg[e] += bias ? bias[e] : 0.f;
+        topk_push(st, lg[e], e);
+      }
+    float den = 0.f;
+    if (gate_norm == 0)
+#pragma unroll
+      for (int e = 0; e < FS_MAX_E; ++e)
+        if (e < E) den += softmax_term(st, lg[e]);
+    topk_finish(st, k, gate_norm, den, sidx + (size_t)t * k, sw + (size_t)t * k);
   }
   if (tid < FS_MAX_E) run[tid] = 0;
   __syncthreads();

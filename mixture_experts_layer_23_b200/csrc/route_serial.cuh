@@ -12,36 +12,32 @@
 
 namespace moe {
 
-struct TopK8 {
-  float v[8];  // best logits so far, descending; ties keep the earlier (lower) expert first
-  int e[8];
-  float m;     // running max of all logits (online softmax)
-  float s;     // running sum of exp(logit - m)
+// The KS best logits so far (KS >= k; the first k entries do not depend on KS, so a caller that
+// knows k at compile time keeps only that many slots and shortens every insertion).
+template <int KS>
+struct TopK {
+  float v[KS];  // descending; ties keep the earlier (lower) expert first
+  int e[KS];
 };
+using TopK8 = TopK<8>;
 
-__device__ __forceinline__ void topk_init(TopK8& t) {
+template <int KS>
+__device__ __forceinline__ void topk_init(TopK<KS>& t) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < KS; ++j) {
     t.v[j] = -INFINITY;
     t.e[j] = 0x7fffffff;
   }
-  t.m = -INFINITY;
-  t.s = 0.f;
 }
 
 // Feed logit v of expert e; experts must arrive in increasing index order.
-__device__ __forceinline__ void topk_push(TopK8& t, float v, int e) {
-  if (v > t.m) {
-    t.s = t.s * expf(t.m - v) + 1.f;
-    t.m = v;
-  } else {
-    t.s += expf(v - t.m);
-  }
-  if (v > t.v[7]) {
+template <int KS>
+__device__ __forceinline__ void topk_push(TopK<KS>& t, float v, int e) {
+  if (v > t.v[KS - 1]) {
     // insert at the first slot holding a strictly smaller logit (an equal, earlier expert stays
     // ahead) and shift the tail down by one; walking from the end reads only unmodified slots
 #pragma unroll
-    for (int j = 7; j > 0; --j) {
+    for (int j = KS - 1; j > 0; --j) {
       if (v > t.v[j - 1]) {
         t.v[j] = t.v[j - 1];
         t.e[j] = t.e[j - 1];
@@ -57,25 +53,38 @@ __device__ __forceinline__ void topk_push(TopK8& t, float v, int e) {
   }
 }
 
-__device__ __forceinline__ void topk_finish(const TopK8& t, int k, int gate_norm,
+// The softmax over all E logits is taken in two passes: the top-k pass above finds the largest
+// logit (t.v[0]), and a second pass adds exp(l - t.v[0]) over the logits in increasing expert
+// order.  The exponentials of that pass do not depend on one another, so they overlap; an online
+// softmax inside the top-k pass would put one exponential per expert on a serial chain.
+template <int KS>
+__device__ __forceinline__ float softmax_term(const TopK<KS>& t, float l) {
+  return expf(l - t.v[0]);
+}
+
+// Gate weights of the k best experts.  gate_norm 0: softmax over all E logits, `den` being the
+// sum of softmax_term over them (in increasing expert order); gate_norm 1: softmax over the k
+// chosen logits only (`den` unused).
+template <int KS>
+__device__ __forceinline__ void topk_finish(const TopK<KS>& t, int k, int gate_norm, float den,
                                             int32_t* __restrict__ idx_out,
                                             float* __restrict__ w_out) {
   if (gate_norm == 0) {
-    const float inv = 1.f / t.s;
+    const float inv = 1.f / den;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < KS; ++j)
       if (j < k) {
         idx_out[j] = t.e[j];
-        w_out[j] = expf(t.v[j] - t.m) * inv;
+        w_out[j] = expf(t.v[j] - t.v[0]) * inv;
       }
   } else {
     float z = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < KS; ++j)
       if (j < k) z += expf(t.v[j] - t.v[0]);
     const float inv = 1.f / z;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
+    for (int j = 0; j < KS; ++j)
       if (j < k) {
         idx_out[j] = t.e[j];
         w_out[j] = expf(t.v[j] - t.v[0]) * inv;

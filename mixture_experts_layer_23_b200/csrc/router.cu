@@ -82,7 +82,10 @@ router_fwd_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
     TopK8 st;
     topk_init(st);
     for (int e = 0; e < E; ++e) topk_push(st, ls[tid * (E + 1) + e], e);
-    topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
+    float den = 0.f;
+    if (gate_norm == 0)
+      for (int e = 0; e < E; ++e) den += softmax_term(st, ls[tid * (E + 1) + e]);
+    topk_finish(st, k, gate_norm, den, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
   }
 }
 
@@ -96,7 +99,10 @@ __global__ void topk_from_logits_kernel(const float* __restrict__ logits, int T_
   TopK8 st;
   topk_init(st);
   for (int e = 0; e < E; ++e) topk_push(st, row[e], e);
-  topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
+  float den = 0.f;
+  if (gate_norm == 0)
+    for (int e = 0; e < E; ++e) den += softmax_term(st, row[e]);
+  topk_finish(st, k, gate_norm, den, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
 }
 
 // Few experts: one warp per token.  The CTA stages the whole gate matrix Wg [E, d] in shared
@@ -175,7 +181,14 @@ router_warp_kernel(const T* __restrict__ x, const T* __restrict__ Wg,
       const float v = __shfl_sync(0xffffffffu, lg, e << SH);
       if (lane == 0) topk_push(st, v, e);
     }
-    if (lane == 0) topk_finish(st, k, gate_norm, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
+    float den = 0.f;
+    if (gate_norm == 0)
+      for (int e = 0; e < E; ++e) {
+        const float v = __shfl_sync(0xffffffffu, lg, e << SH);
+        if (lane == 0) den += softmax_term(st, v);
+      }
+    if (lane == 0)
+      topk_finish(st, k, gate_norm, den, topk_idx + (int64_t)t * k, topk_w + (int64_t)t * k);
   }
 }
 

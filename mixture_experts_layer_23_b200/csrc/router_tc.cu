@@ -6,12 +6,13 @@
 // x once from HBM: with E = 64 its 2*T*d*E FLOPs are more than the CUDA cores deliver in that
 // time, so the contraction runs on the tensor cores and everything after it stays on chip.
 //
-// One CTA per tile of at most 128 tokens (192 threads): warp 0 streams x tiles [rows x 64] and the whole gate
-// matrix slice [E_pad x 64] (E rounded up to 16, zero rows from TMA's out-of-bounds fill) through
-// a ring of up to 16 stages (as many as shared memory holds: with d <= 1024 and few experts the
-// whole token tile is in flight at once, since a CTA has only one tile to load); one lane of warp 1 issues tcgen05.mma (M = 128, N = E_pad) into a TMEM
-// accumulator; warps 2..5 read it back with tcgen05.ld, so each thread holds the E logits of one
-// token, adds the bias, writes the logits and runs the serial softmax + top-k of route_serial.cuh.
+// One CTA per tile of at most 128 tokens (192 threads).  Warp 0 streams x tiles [rows x 64] and the
+// gate matrix slice [E_pad x 64] (E rounded up to 16, zero rows from TMA's out-of-bounds fill)
+// through a ring of up to 16 stages: as many as shared memory holds, so with d <= 1024 and few
+// experts the whole token tile is in flight at once (a CTA has only one tile to load).  One lane of
+// warp 1 issues tcgen05.mma (M = 128, N = E_pad) into a TMEM accumulator.  Warps 2..5 read it back
+// with tcgen05.ld, one token per thread, add the bias, write the logits and run the softmax + top-k
+// of route_serial.cuh (k slots per token, the softmax denominator in a second pass).
 #include <string.h>
 
 #include <algorithm>
@@ -27,8 +28,12 @@ namespace tc {
 namespace {
 
 constexpr int MAX_RSTAGES = 16;
+// x loads leave in groups of this many consecutive k blocks (see the producer loop).  Measured with
+// the router alone, L2 flushed between launches: groups of 2 took 4-6 % off every bf16 layer size
+// (Mixtral-style 35.6 -> 33.6 us, DeepSeek-style 37.4 -> 35.7 us); groups of 4 and 8 were slower
+// than 2, since the producer then holds back more free stages.
 #ifndef MOE_ROUTER_ISSUE_GROUP
-#define MOE_ROUTER_ISSUE_GROUP 1
+#define MOE_ROUTER_ISSUE_GROUP 2
 #endif
 constexpr uint32_t RA_BYTES = 128 * 64 * 2;  // x tile
 constexpr int STAGE_MAX_EPAD = 64;            // rows of at most 64 logits are staged in shared memory
@@ -51,11 +56,23 @@ struct alignas(64) RouterParams {
   int rows;           // tokens per CTA (<= 128): the tiles are balanced over the SMs
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages;
+  uint32_t region;    // bytes before the barriers: the load ring, which the staged rows reuse
   int stall;          // failure-path test: the MMA issuer first waits on a barrier nothing arrives on
 };
 
 __device__ __forceinline__ void epi_bar() {   // the 128 epilogue threads (warps 2..5)
   asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// the same barrier, returning whether `v` holds in every epilogue thread
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
 }
 
 // One CTA per token tile contracts the whole of d.  A tile holds `rows` <= 128 tokens, chosen on
@@ -66,6 +83,8 @@ __device__ __forceinline__ void epi_bar() {   // the 128 epilogue threads (warps
 // shared memory, measured slower at every layer size and was dropped.)
 // Rows of at most 64 logits are staged in shared memory with the expert ids and gate weights, and
 // leave as contiguous rows.
+// KS: top-k slots kept per token (>= k), so the insertion work per expert scales with k, not 8.
+template <int KS>
 __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant__ RouterParams P) {
   pdl_prologue();
   extern __shared__ uint8_t smem_raw[];
@@ -76,10 +95,13 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
   // staging row stride (floats): odd, so the 32 lanes' scalar accesses to their own rows (column
   // e of rows 32q..32q+31) hit 32 distinct banks
   const int PS = P.E_pad + 1;
-  float* part = reinterpret_cast<float*>(smem + RSTAGES * P.stage_bytes);   // [128][PS]
+  // The staged rows reuse the load ring: they are written only once every MMA of the tile, the
+  // ring's last reader, has completed (so no load is in flight either), which leaves the whole
+  // ring to loads in flight until then.
+  float* part = reinterpret_cast<float*>(smem);                             // [128][PS]
   int32_t* sidx = reinterpret_cast<int32_t*>(part + (small ? 128 * PS : 0));  // [128][9]
   float* sw = reinterpret_cast<float*>(sidx + 128 * 9);                     // [128][9]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sw + 128 * 9);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P.region);
   uint64_t* full = bars;
   uint64_t* empty = bars + RSTAGES;
   uint64_t* tfull = bars + 2 * RSTAGES;
@@ -191,7 +213,18 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     // out, so that the kernels after this one stay in bounds; the status word reports it
     const bool ok = have && !*abort_flag;
     const bool live = row < nrow;
-    if (small) {
+    // staging only when every epilogue thread saw the tile complete: otherwise loads may still be
+    // landing in the ring, and the placeholders go straight to global memory
+    const bool staged = small && epi_bar_and(ok);
+    if (small && !staged) {
+      if (live) {
+        for (int e = 0; e < P.E; ++e) P.logits[(size_t)t * P.E + e] = 0.f;
+        for (int j = 0; j < P.k; ++j) {
+          P.topk_idx[(size_t)t * P.k + j] = j;
+          P.topk_w[(size_t)t * P.k + j] = 0.f;
+        }
+      }
+    } else if (small) {
       // the row's logits (+ bias) go to its staging row 16 at a time, then the serial softmax +
       // top-k reads them back from there: a short loop body instead of E unrolled steps, whose
       // code outgrew the instruction cache at 64 experts
@@ -200,27 +233,23 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 #pragma unroll 1
       for (int c = 0; c < P.E_pad / 16; ++c) {
         float v[16];
-        if (have) tmem_ld16(ta + (uint32_t)(c * 16), v);
+        tmem_ld16(ta + (uint32_t)(c * 16), v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int e = c * 16 + i;
-          if (e < P.E) prow[e] = ok ? v[i] + (P.bias ? P.bias[e] : 0.f) : 0.f;
+          if (e < P.E) prow[e] = v[i] + (P.bias ? P.bias[e] : 0.f);
         }
       }
-      TopK8 st;
+      TopK<KS> st;
       topk_init(st);
 #pragma unroll 4
       for (int e = 0; e < P.E; ++e) topk_push(st, prow[e], e);
-      int32_t* oi = sidx + row * 9;
-      float* ow = sw + row * 9;
-      if (ok) {
-        topk_finish(st, P.k, P.gate_norm, oi, ow);
-      } else {
-        for (int j = 0; j < P.k; ++j) {
-          oi[j] = j;
-          ow[j] = 0.f;
-        }
+      float den = 0.f;
+      if (P.gate_norm == 0) {
+#pragma unroll 8
+        for (int e = 0; e < P.E; ++e) den += softmax_term(st, prow[e]);
       }
+      topk_finish(st, P.k, P.gate_norm, den, sidx + row * 9, sw + row * 9);
       epi_bar();
       // the tile's rows are contiguous in logits, topk_idx and topk_w: coalesced stores
       const int tid = threadIdx.x - 64;
@@ -232,7 +261,7 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
       }
     } else if (ok) {
       // wide rows (more than 64 experts): stream them out of TMEM 16 at a time
-      TopK8 st;
+      TopK<KS> st;
       topk_init(st);
       float v[16];
       for (int c = 0; c < P.E_pad / 16; ++c) {
@@ -247,8 +276,19 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
           }
         }
       }
+      float den = 0.f;
+      if (P.gate_norm == 0) {   // second pass over the accumulator for the softmax denominator
+        for (int c = 0; c < P.E_pad / 16; ++c) {
+          tmem_ld16(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(c * 16), v);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = c * 16 + i;
+            if (e < P.E) den += softmax_term(st, v[i] + (P.bias ? P.bias[e] : 0.f));
+          }
+        }
+      }
       if (live)
-        topk_finish(st, P.k, P.gate_norm, P.topk_idx + (size_t)t * P.k,
+        topk_finish(st, P.k, P.gate_norm, den, P.topk_idx + (size_t)t * P.k,
                     P.topk_w + (size_t)t * P.k);
     } else if (live) {
       for (int e = 0; e < P.E; ++e) P.logits[(size_t)t * P.E + e] = 0.f;
@@ -422,6 +462,19 @@ bool router_tc_supported(const Dims& D) {
   return D.dtype == MOE_DTYPE_BF16 && D.d % 64 == 0 && D.E <= 256 && tc::encoder() != nullptr;
 }
 
+template <int KS>
+static moe_status launch_router_ks(const tc::RouterParams& P, int n_tiles, size_t smem,
+                                   cudaStream_t st) {
+  static int smem_set = 0;
+  if ((int)smem > smem_set) {
+    if (cudaFuncSetAttribute(tc::router_tc_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    smem_set = (int)smem;
+  }
+  return launch_k(tc::router_tc_kernel<KS>, n_tiles, 192, smem, st, 1, P);
+}
+
 moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const float* bias,
                             float* logits, int32_t* topk_idx, float* topk_w, uint32_t* status,
                             cudaStream_t st) {
@@ -461,19 +514,19 @@ moe_status launch_router_tc(const Dims& D, const void* x, const void* Wg, const 
   const int nk_cta = D.d / 64;
   const size_t stage_rows = E_pad <= STAGE_MAX_EPAD ? (size_t)128 * (E_pad + 8) * 4 : 0;
   // alignment slack, staged rows, expert ids and weights, barriers (2 per stage + 2), TMEM slot
-  const size_t fixed = 1024 + stage_rows + 2 * 128 * 9 * 4 + 2 * 8 + 16;
+  // alignment slack, barriers (2 per stage + 2), TMEM slot and abort flag; the staged rows, expert
+  // ids and weights reuse the ring
+  const size_t fixed = 1024 + 2 * 8 + 16;
   const size_t fit = (RSMEM_WHOLE - fixed) / (P.stage_bytes + 2 * 8);
   P.nstages = (int)std::max<size_t>(
       1, std::min<size_t>(std::min<size_t>(MAX_RSTAGES, fit), (size_t)nk_cta));
-  const size_t smem = fixed + (size_t)P.nstages * (P.stage_bytes + 2 * 8);
-  static int smem_set = 0;
-  if ((int)smem > smem_set) {
-    if (cudaFuncSetAttribute(router_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    smem_set = (int)smem;
-  }
-  return launch_k(router_tc_kernel, n_tiles, 192, smem, st, 1, P);
+  const size_t staged = stage_rows + 2 * 128 * 9 * 4;
+  P.region = (uint32_t)round_up(std::max<size_t>((size_t)P.nstages * P.stage_bytes, staged), 8);
+  const size_t smem = fixed + P.region + (size_t)P.nstages * 2 * 8;
+  return P.k <= 2   ? launch_router_ks<2>(P, n_tiles, smem, st)
+         : P.k <= 4 ? launch_router_ks<4>(P, n_tiles, smem, st)
+         : P.k <= 6 ? launch_router_ks<6>(P, n_tiles, smem, st)
+                    : launch_router_ks<8>(P, n_tiles, smem, st);
 }
 
 moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, const void* x,

@@ -18,9 +18,11 @@ int main() {
     moe::TopK8 st;
     moe::topk_init(st);
     for (int e = 0; e < E; ++e) moe::topk_push(st, row[e], e);
+    float den = 0.f;   // second pass: softmax denominator over all E logits, in expert order
+    for (int e = 0; e < E; ++e) den += moe::softmax_term(st, row[e]);
     int idx[8];
     float w[8];
-    moe::topk_finish(st, k, gate_norm, idx, w);
+    moe::topk_finish(st, k, gate_norm, den, idx, w);
     for (int j = 0; j < k; ++j) printf("%d ", idx[j]);
     for (int j = 0; j < k; ++j) printf("%.9g ", w[j]);
     printf("\n");
