@@ -71,27 +71,27 @@ WGRAD_SOURCES = GEMM_SOURCES + ["transpose.cu"]
 NCU_TRAFFIC = {
     # weight-gradient phase: transpose64_kernel + the dW1 and dW3 launches
     ("mixtral_dropless", "wgrad_w1"): {
-        "bytes": 14112258790,
+        "bytes": 11645794125,
         "sources": WGRAD_SOURCES,
-        "sha256": "98cdd15fa617bcadbbb4272181c9334631035f10d7b3f6ba1f2ea70ee655fa9a",
+        "sha256": "41af3019e08d24fe8bc6539984b7815221925c99b270a4f2674fe0be4055d772",
         "profile": "profiles/launches_mixtral_dropless.md",
     },
     ("mixtral_dropless", "expert_up"): {
-        "bytes": 9424231654,
+        "bytes": 7161878170,
         "sources": GEMM_SOURCES,
-        "sha256": "3681793c7edf6f65cf0352cbd2526b66350fe704a497e2bd12d5d9f7b2ea969b",
+        "sha256": "fdd434ed07ec0e71eacdb4758d6cdff948328d40a3df7d97dc54e0675abdafe8",
         "profile": "profiles/launches_mixtral_dropless.md",
     },
     ("deepseek_v2", "wgrad_w1"): {   # the dW1 and dW3 launches (no transposes on this layer)
-        "bytes": 2873133107,
+        "bytes": 2878450816,
         "sources": WGRAD_SOURCES,
-        "sha256": "98cdd15fa617bcadbbb4272181c9334631035f10d7b3f6ba1f2ea70ee655fa9a",
+        "sha256": "41af3019e08d24fe8bc6539984b7815221925c99b270a4f2674fe0be4055d772",
         "profile": "profiles/launches_deepseek_v2.md",
     },
     ("deepseek_v2", "expert_up"): {
-        "bytes": 2028915302,
+        "bytes": 2036857626,
         "sources": GEMM_SOURCES,
-        "sha256": "3681793c7edf6f65cf0352cbd2526b66350fe704a497e2bd12d5d9f7b2ea969b",
+        "sha256": "fdd434ed07ec0e71eacdb4758d6cdff948328d40a3df7d97dc54e0675abdafe8",
         "profile": "profiles/launches_deepseek_v2.md",
     },
     # one launch of the up-projection GEMM (ncu --set full --clock-control none, one kernel, on
