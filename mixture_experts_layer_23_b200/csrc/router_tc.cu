@@ -121,17 +121,9 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) tmem_alloc(tmem_slot, P.tmem_cols);
-  if (P.rows < 128) {
-    // A rows [rows, 128) of every stage are never loaded: zero them once, so the MMA reads zeros
-    // there (their accumulator lanes are not read either)
-    const int tail = (128 - P.rows) * 128 / 16;   // 16-byte units per stage
-    for (int i = threadIdx.x; i < RSTAGES * tail; i += blockDim.x) {
-      const int s = i / tail, u = i - s * tail;
-      *reinterpret_cast<uint4*>(smem + s * P.stage_bytes + P.rows * 128 + u * 16) =
-          make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_async_smem();   // the generic-proxy zeros before the tensor core's async-proxy reads
-  }
+  // A rows [rows, 128) of the stages are never loaded and hold whatever shared memory held: each
+  // accumulator lane depends only on its own A row, and lanes past the tile's tokens are not stored.
+  // (Zeroing them cost 3.6 us per launch on the GPT-2-style layer, 32-token tiles.)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
