@@ -269,10 +269,16 @@ def calibrate_sample(shape, inp, target_s):
 def cpu_baseline(shape, inp, target_s):
     prepare_oracle_weights(shape, inp)
     n, _ = calibrate_sample(shape, inp, target_s)
-    t = oracle_step(shape, inp, n)
-    return {"value": n / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {n} of {shape.T} tokens, one float64 forward+backward of the same "
-                      f"layer (capacity recomputed for {n} tokens), {t:.1f} s"}
+    # a layer whose step cost is mostly the weight gradients (fixed in n) reaches the target with
+    # repeated steps on the sample rather than a larger one (at most four)
+    t, reps = oracle_step(shape, inp, n), 1
+    while t < 0.8 * target_s and reps < 4:
+        t += oracle_step(shape, inp, n)
+        reps += 1
+    steps = f"{reps} float64 forward+backward steps" if reps > 1 else "one float64 forward+backward"
+    return {"value": n * reps / t, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {n} of {shape.T} tokens, {steps} of the same layer (capacity "
+                      f"recomputed for {n} tokens), {t:.1f} s"}
 
 
 def run_reference(args):
