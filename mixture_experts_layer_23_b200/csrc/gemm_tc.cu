@@ -102,6 +102,12 @@ constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 #ifndef MOE_GEMM_DIRECT_STORE
 #define MOE_GEMM_DIRECT_STORE 0
 #endif
+#ifndef MOE_UP_STAGES
+#define MOE_UP_STAGES 5        // load stages of the up-projection GEMM
+#endif
+#ifndef MOE_UP_EPI_WARPS
+#define MOE_UP_EPI_WARPS 8     // its epilogue warps (4 or 8)
+#endif
 #ifndef MOE_DGRAD_H_STAGES
 #define MOE_DGRAD_H_STAGES 5   // load stages of the activation-gradient GEMM
 #endif
@@ -111,7 +117,7 @@ constexpr uint32_t GATHER_BUF_BYTES = 32 * GROW;
 
 template <int KIND>
 struct Cfg {
-  static constexpr int EPI_WARPS = (KIND == UP) ? 8 : (KIND == UNDISPATCH) ? 4 * MOE_UNDISPATCH_SPLIT : 4;
+  static constexpr int EPI_WARPS = (KIND == UP) ? MOE_UP_EPI_WARPS : (KIND == UNDISPATCH) ? 4 * MOE_UNDISPATCH_SPLIT : 4;
   static constexpr int SPLIT = EPI_WARPS / 4;   // epilogue warps per TMEM lane quarter
   // plain-output kinds may store straight from registers, which frees the staging ring for a
   // seventh stage of loads in flight
@@ -119,7 +125,7 @@ struct Cfg {
       MOE_GEMM_DIRECT_STORE && (KIND == DOWN || KIND == DGRAD_X || KIND == WGRAD);
   // UNDISPATCH contracts K = E (at most 4 k blocks): two stages are plenty, and the room goes to
   // the gather buffers of its epilogue
-  static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? 5 : (KIND == DGRAD_H) ? MOE_DGRAD_H_STAGES
+  static constexpr int STAGES = DIRECT ? 7 : (KIND == UP) ? MOE_UP_STAGES : (KIND == DGRAD_H) ? MOE_DGRAD_H_STAGES
                                        : (KIND == UNDISPATCH) ? (MOE_UNDISPATCH_SPLIT > 1 ? 1 : 2) : 6;
   static constexpr int NIN = (KIND == DGRAD_H) ? MOE_DGRAD_H_NIN : 0;   // epilogue input slots per warp
   static constexpr int NGATH = (KIND == UNDISPATCH) ? (MOE_UNDISPATCH_SPLIT > 1 ? 3 : 6) : 0;   // gather buffers per warp
