@@ -71,37 +71,34 @@ WGRAD_SOURCES = GEMM_SOURCES + ["transpose.cu"]
 NCU_TRAFFIC = {
     # weight-gradient phase: transpose64_kernel + the dW1 and dW3 launches
     ("mixtral_dropless", "wgrad_w1"): {
-        "bytes": 11645794125,
+        "bytes": 15686405478,
         "sources": WGRAD_SOURCES,
-        "sha256": "41af3019e08d24fe8bc6539984b7815221925c99b270a4f2674fe0be4055d772",
+        "sha256": "bdf5917b14f1a7688c880b17a52e5d21bea257f7a01a57c65a5477a036629f53",
         "profile": "profiles/launches_mixtral_dropless.md",
     },
     ("mixtral_dropless", "expert_up"): {
-        "bytes": 7161878170,
+        "bytes": 11330623053,
         "sources": GEMM_SOURCES,
-        "sha256": "fdd434ed07ec0e71eacdb4758d6cdff948328d40a3df7d97dc54e0675abdafe8",
+        "sha256": "9935fc610e25e1760dc0152fe0942080d209f33a55c7ce35a6db03ea2ef1e2e3",
         "profile": "profiles/launches_mixtral_dropless.md",
     },
     ("deepseek_v2", "wgrad_w1"): {   # the dW1 and dW3 launches (no transposes on this layer)
-        "bytes": 2878450816,
+        "bytes": 2882665472,
         "sources": WGRAD_SOURCES,
-        "sha256": "41af3019e08d24fe8bc6539984b7815221925c99b270a4f2674fe0be4055d772",
+        "sha256": "bdf5917b14f1a7688c880b17a52e5d21bea257f7a01a57c65a5477a036629f53",
         "profile": "profiles/launches_deepseek_v2.md",
     },
     ("deepseek_v2", "expert_up"): {
-        "bytes": 2036857626,
+        "bytes": 2031581773,
         "sources": GEMM_SOURCES,
-        "sha256": "fdd434ed07ec0e71eacdb4758d6cdff948328d40a3df7d97dc54e0675abdafe8",
+        "sha256": "9935fc610e25e1760dc0152fe0942080d209f33a55c7ce35a6db03ea2ef1e2e3",
         "profile": "profiles/launches_deepseek_v2.md",
     },
-    # one launch of the up-projection GEMM (ncu --set full --clock-control none, one kernel, on
-    # `python bench.py --workload gpt2_gshard --steps 1 --warmup 1 --no-cpu-baseline`):
-    # dram__bytes_read.sum 89.732096 MB + dram__bytes_write.sum 60.708352 MB
     ("gpt2_gshard", "expert_up"): {
-        "bytes": 150440448,
+        "bytes": 146722355,
         "sources": GEMM_SOURCES,
-        "sha256": "b7412286015775b8673a67b6a41166523ba9cc5be06084b44510b77b574f82bb",
-        "profile": "profiles/expert_up_gpt2_gshard.md",
+        "sha256": "9935fc610e25e1760dc0152fe0942080d209f33a55c7ce35a6db03ea2ef1e2e3",
+        "profile": "profiles/launches_gpt2_gshard.md",
     },
 }
 
