@@ -67,3 +67,23 @@ def test_reference_arm_runs_on_rank_zero_only():
     line = json.loads(r.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_cpu_baseline_repeats_a_short_sample(monkeypatch):
+    """The oracle baseline repeats its sample's step (at most four times) until it has run for about
+    the target time, and reports tokens over the summed time of all the repetitions."""
+    sys.path.insert(0, ROOT)
+    import bench
+    steps = []
+    monkeypatch.setattr(bench, "prepare_oracle_weights", lambda shape, inp: None)
+    monkeypatch.setattr(bench, "calibrate_sample", lambda shape, inp, target: (200, 3.0))
+    monkeypatch.setattr(bench, "oracle_step", lambda shape, inp, n: steps.append(n) or 3.0)
+    shape = type("Shape", (), {"T": 16384})()
+    out = bench.cpu_baseline(shape, None, 12.0)
+    assert steps == [200] * 4
+    assert out["value"] == pytest.approx(200 * 4 / 12.0)
+    assert "4 float64 forward+backward steps" in out["sample"]
+    steps.clear()
+    monkeypatch.setattr(bench, "oracle_step", lambda shape, inp, n: steps.append(n) or 20.0)
+    out = bench.cpu_baseline(shape, None, 12.0)
+    assert steps == [200] and out["value"] == pytest.approx(10.0)
