@@ -292,29 +292,6 @@ __device__ __forceinline__ bool half_n(const Params& P, const Tile& t) {
 // nb = n0 + 128 * rank (for the SwiGLU up-projection: CTA 0 loads W1 rows, CTA 1 the same rows of
 // W3, which makes accumulator columns 0..127 U and 128..255 V).  bar: the leader's full barrier.
 
-// B loads.  The tile order walks a band of 16 m tiles across the n tiles, so the pairs of one wave
-// share about 5 B slices between 16 tiles each and about 16 A slices between 5 tiles each; with
-// MOE_GEMM_B_EVICT_LAST the B lines are kept in L2 ahead of the A lines.
-#ifndef MOE_GEMM_B_EVICT_LAST
-#define MOE_GEMM_B_EVICT_LAST 1
-#endif
-__device__ __forceinline__ void load_b2(void* dst, const CUtensorMap* map, uint32_t bar, int c0,
-                                        int c1) {
-#if MOE_GEMM_B_EVICT_LAST
-  tma_load_2d_pair(dst, map, bar, c0, c1, l2_policy_evict_last());
-#else
-  tma_load_2d_pair(dst, map, bar, c0, c1);
-#endif
-}
-__device__ __forceinline__ void load_b3(void* dst, const CUtensorMap* map, uint32_t bar, int c0,
-                                        int c1, int c2) {
-#if MOE_GEMM_B_EVICT_LAST
-  tma_load_3d_pair(dst, map, bar, c0, c1, c2, l2_policy_evict_last());
-#else
-  tma_load_3d_pair(dst, map, bar, c0, c1, c2);
-#endif
-}
-
 template <int KIND>
 __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int kb, int rank,
                                             uint8_t* sA, uint8_t* sB, uint32_t bar) {
@@ -326,23 +303,23 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
   if (KIND == UP) {
     if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
     else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
-    if (swiglu) load_b3(sB, rank ? &P.b_alt : &P.b_main, bar, k0, t.n * BNH, t.g);
-    else load_b3(sB, &P.b_main, bar, k0, nb, t.g);
+    if (swiglu) tma_load_3d_pair(sB, rank ? &P.b_alt : &P.b_main, bar, k0, t.n * BNH, t.g);
+    else tma_load_3d_pair(sB, &P.b_main, bar, k0, nb, t.g);
   } else if (KIND == DOWN) {
     tma_load_2d_pair(sA, &P.a_main, bar, k0, t.o_row + t.mrow);
-    load_b3(sB, &P.b_main, bar, k0, nb, t.g);
+    tma_load_3d_pair(sB, &P.b_main, bar, k0, nb, t.g);
   } else if (KIND == DGRAD_H) {
     if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
     else tma_load_2d_pair(sA, &P.a_main, bar, k0, t.a_row + t.mrow);
     for (int j = 0; j < nbj; ++j)
-      load_b3(sB + j * 8192, &P.b_main, bar, nb + 64 * j, k0, t.g);
+      tma_load_3d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, k0, t.g);
   } else if (KIND == DGRAD_X || KIND == UNDISPATCH) {
     const int nkF = P.K / BK;
     const bool second = kb >= nkF;
     const int kk = (second ? kb - nkF : kb) * BK;
     tma_load_2d_pair(sA, second ? &P.a_alt : &P.a_main, bar, kk, t.o_row + t.mrow);
     for (int j = 0; j < nbj; ++j)
-      load_b3(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
+      tma_load_3d_pair(sB + j * 8192, second ? &P.b_alt : &P.b_main, bar, nb + 64 * j, kk, t.g);
   } else if (P.kmajor) {
     // WGRAD, K over the group's rows, one operand read through its column-major copy (K-major,
     // one 128-row box), the other straight from the token-major rows (MN-major, two 64-column
@@ -352,14 +329,14 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
 #pragma unroll
       for (int j = 0; j < BM / 64; ++j)
         tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
-      if (t.shared) load_b2(sB, &P.b_alt, bar, k0, nb);
-      else load_b2(sB, &P.b_main, bar, t.a_row + k0, nb);
+      if (t.shared) tma_load_2d_pair(sB, &P.b_alt, bar, k0, nb);
+      else tma_load_2d_pair(sB, &P.b_main, bar, t.a_row + k0, nb);
     } else {
       // A = dO^T (routed) or dy^T (shared), K-major; B = H rows of the group (MN-major)
       if (t.shared) tma_load_2d_pair(sA, &P.a_alt, bar, k0, t.mrow);
       else tma_load_2d_pair(sA, &P.a_main, bar, t.a_row + k0, t.mrow);
       for (int j = 0; j < nbj; ++j)
-        load_b2(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
+        tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
     }
   } else {  // WGRAD, both operands straight from the token-major rows (MN-major)
     if (P.which == 0) {
@@ -368,8 +345,8 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
       for (int j = 0; j < BM / 64; ++j)
         tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.o_row + k0);
       for (int j = 0; j < nbj; ++j) {
-        if (t.shared) load_b2(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
-        else load_b2(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
+        if (t.shared) tma_load_2d_pair(sB + j * 8192, &P.b_alt, bar, nb + 64 * j, k0);
+        else tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.a_row + k0);
       }
     } else {
       // A = dO rows (routed) or dy (shared), B = H rows of the group
@@ -379,7 +356,7 @@ __device__ __forceinline__ void issue_loads(const Params& P, const Tile& t, int 
         else tma_load_2d_pair(sA + j * 8192, &P.a_main, bar, t.mrow + 64 * j, t.a_row + k0);
       }
       for (int j = 0; j < nbj; ++j)
-        load_b2(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
+        tma_load_2d_pair(sB + j * 8192, &P.b_main, bar, nb + 64 * j, t.o_row + k0);
     }
   }
 }
