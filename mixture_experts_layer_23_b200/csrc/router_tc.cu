@@ -323,14 +323,28 @@ __global__ void __launch_bounds__(192, 1) router_tc_kernel(const __grid_constant
 
 struct alignas(64) RWParams {
   CUtensorMap x_map;   // x [T, d], box {64 (d), 64 (tokens)}
-  CUtensorMap l_map;   // dl16 [T, E8], box {64 (experts), 64 (tokens)}
+  CUtensorMap l_map;   // dl16 [T, E8], box {64 (experts), 64 (tokens)}; narrow: {16, 64}, 32 B swizzle
   float* part;         // [n_chunks][E][d]
   uint32_t* status;
   unsigned long long timeout_ns;
   int T, d, E, N, chunk, n_dt;
   uint32_t idesc, tmem_cols, stage_bytes;
   int nstages, stall;
+  int narrow;          // E <= 16: N = 16, dl16 rows of 32 bytes
 };
+
+// Shared-memory descriptor of an MN-major operand in the 32-byte swizzle: atoms of 8 K rows x 32
+// bytes (16 bf16 along MN), `sbo` bytes between consecutive 8-row groups.  The operand is a single
+// 16-element chunk along MN, so the leading-byte offset (the stride between such chunks) is unused.
+__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((2048u >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 6ull << 61;   // SWIZZLE_32B
+  return d;
+}
 
 __global__ void __launch_bounds__(192, 1) router_wgrad_tc_kernel(const __grid_constant__ RWParams P) {
   pdl_prologue();
@@ -381,7 +395,10 @@ __global__ void __launch_bounds__(192, 1) router_wgrad_tc_kernel(const __grid_co
       const int tk = t0 + kb * 64;
       tma_load_2d(sA, &P.x_map, &full[stage], d0, tk);
       tma_load_2d(sA + 8192, &P.x_map, &full[stage], d0 + 64, tk);
-      for (int j = 0; j < P.N / 64; ++j) tma_load_2d(sB + j * 8192, &P.l_map, &full[stage], 64 * j, tk);
+      if (P.narrow) tma_load_2d(sB, &P.l_map, &full[stage], 0, tk);
+      else
+        for (int j = 0; j < P.N / 64; ++j)
+          tma_load_2d(sB + j * 8192, &P.l_map, &full[stage], 64 * j, tk);
       outstanding |= 1u << stage;
       out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
       if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
@@ -398,9 +415,10 @@ __global__ void __launch_bounds__(192, 1) router_wgrad_tc_kernel(const __grid_co
       const uint32_t sa = smem_u32(smem + stage * P.stage_bytes);
       const uint32_t sb = sa + 16384;
 #pragma unroll
-      for (int k = 0; k < 4; ++k)   // both operands MN-major: a K step of 16 rows is 2 KB
+      for (int k = 0; k < 4; ++k)   // both operands MN-major: a K step of 16 rows is 2 KB (B narrow: 512 B)
         umma_bf16(tmem_base, sw128_desc(sa + k * 2048, 8192, 1024),
-                  sw128_desc(sb + k * 2048, 8192, 1024), P.idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                  P.narrow ? sw32_desc(sb + k * 512, 256) : sw128_desc(sb + k * 2048, 8192, 1024),
+                  P.idesc, (kb > 0 || k > 0) ? 1u : 0u);
       issued = true;
       umma_commit(&empty[stage]);
       if (++stage == RSTAGES) { stage = 0; phase ^= 1u; }
@@ -527,7 +545,12 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
   RWParams P;
   memset(&P, 0, sizeof(P));
   const int E8 = (int)round_up(D.E, 8);
-  if (!map2(&P.x_map, x, D.d, D.T, 64, 64) || !map2(&P.l_map, dl16, E8, D.T, 64, 64))
+  // At most 16 experts: N = 16 MMAs (their cost grows with N) over dl16 rows fetched as 16-element
+  // boxes in the 32-byte swizzle, instead of N = 64 with 56 or 48 zero columns.
+  P.narrow = E8 <= 16;
+  if (!map2(&P.x_map, x, D.d, D.T, 64, 64) ||
+      !(P.narrow ? map2_sw32(&P.l_map, dl16, E8, D.T, 16, 64)
+                 : map2(&P.l_map, dl16, E8, D.T, 64, 64)))
     return MOE_ERR_CUDA;
   P.part = part;
   P.status = status;
@@ -536,7 +559,7 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
   P.T = D.T;
   P.d = D.d;
   P.E = D.E;
-  P.N = (int)round_up(D.E, 64);                 // 64..256
+  P.N = P.narrow ? 16 : (int)round_up(D.E, 64);   // 16, or 64..256
   P.n_dt = (D.d + 127) / 128;
   // token chunks: at most two CTAs per SM in all (one wave: a partial second wave of a few CTAs
   // would double the time), within the partial buffer (D.n_tchunk chunks)
@@ -548,7 +571,7 @@ moe_status launch_router_wgrad_tc(const Dims& D, const __nv_bfloat16* dl16, cons
   uint32_t cols = 64;
   while ((int)cols < P.N) cols <<= 1;
   P.tmem_cols = cols;
-  P.stage_bytes = 16384u + (uint32_t)P.N * 128u;
+  P.stage_bytes = 16384u + (P.narrow ? 64u * 32u : (uint32_t)P.N * 128u);   // x, then dl16
   const int nk_cta = P.chunk / 64;
   const size_t fixed = 1024 + 2 * 8 + 16;
   const size_t fit = (RSMEM_SPLIT - fixed) / (P.stage_bytes + 2 * 8);

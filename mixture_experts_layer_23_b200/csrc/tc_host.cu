@@ -18,9 +18,9 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-// bf16 map, 128-byte swizzle.  dims/box innermost first; rank 2 or 3.
+// bf16 map, 128-byte swizzle (32-byte with swz32).  dims/box innermost first; rank 2 or 3.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-              const uint32_t* box, int elem) {
+              const uint32_t* box, int elem, bool swz32) {
   EncodeTiledFn enc = encoder();
   if (!enc || !base) return false;
   cuuint64_t gd[3], gs[2];
@@ -32,7 +32,8 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   gs[0] = dims[0] * elem;
   if (rank == 3) gs[1] = dims[0] * dims[1] * elem;
   return enc(m, elem == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swz32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -41,6 +42,12 @@ bool map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint3
   const uint64_t d[2] = {inner, rows};
   const uint32_t b[2] = {box_inner, box_rows};
   return make_map(m, base, 2, d, b);
+}
+bool map2_sw32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+               uint32_t box_inner, uint32_t box_rows) {
+  const uint64_t d[2] = {inner, rows};
+  const uint32_t b[2] = {box_inner, box_rows};
+  return make_map(m, base, 2, d, b, 2, true);
 }
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
                  uint32_t box_inner, uint32_t box_mid) {

@@ -12,12 +12,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encoder();
-// Tensor map with 128-byte swizzle over bf16 (elem 2) or fp32 (elem 4) data; dims and box
-// innermost first, rank 2 or 3.
+// Tensor map with 128-byte swizzle (32-byte with swz32) over bf16 (elem 2) or fp32 (elem 4) data;
+// dims and box innermost first, rank 2 or 3.
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint32_t* box,
-              int elem = 2);
+              int elem = 2, bool swz32 = false);
 bool map2(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
           uint32_t box_rows);
+// bf16, 32-byte swizzle: boxes 16 elements wide
+bool map2_sw32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+               uint32_t box_rows);
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
           uint32_t box_inner, uint32_t box_mid);
 bool map3_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
